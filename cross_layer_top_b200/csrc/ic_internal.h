@@ -1,0 +1,89 @@
+// Host-side internals of libindexcache: the context and the kernel launchers.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "ic_errors.h"
+
+struct ic_ctx {
+    int device = 0;
+    int num_sms = 148;
+    size_t scratch_limit = 0;       // bound on the prefill score scratch (bytes)
+    float* scores = nullptr;        // score scratch (fp32 rows)
+    size_t scores_cap = 0;          // bytes
+    float* attn_part = nullptr;     // split-attention partials
+    size_t attn_part_cap = 0;       // bytes
+    int* dev_err = nullptr;         // device error word (first error wins)
+    std::string last_error;
+    bool timing = false;
+    struct EventPair {
+        int kernel;
+        cudaEvent_t start, stop;
+    };
+    std::vector<EventPair> pool;    // reusable event pairs
+    size_t pending = 0;             // pairs recorded since the last harvest
+    double total_ms[IC_K_COUNT] = {0};
+    int64_t launches[IC_K_COUNT] = {0};
+    int64_t launch_count = 0;
+};
+
+struct ic_pattern {
+    std::string c;
+    std::vector<int32_t> src;
+};
+
+namespace ic {
+
+// Records the message on ctx (or the global slot) and returns code.
+int fail(ic_ctx* ctx, int code, const char* fmt, ...);
+int cuda_fail(ic_ctx* ctx, cudaError_t e, const char* what);
+
+// Brackets one kernel launch with timing events when timing is enabled and
+// counts it.  Usage: LaunchScope ls(ctx, IC_K_TOPK, stream); kernel<<<>>>; ls.done();
+struct LaunchScope {
+    ic_ctx* ctx;
+    int kernel;
+    cudaStream_t stream;
+    size_t slot;
+    LaunchScope(ic_ctx* c, int k, cudaStream_t s);
+    cudaError_t done();
+};
+
+// Grows a scratch buffer to at least `bytes`.  Returns IC_OK / IC_ERR_NOMEM.
+int ensure_buffer(ic_ctx* ctx, void** buf, size_t* cap, size_t bytes);
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled_fn();
+
+// 2-D bf16 tensor map over [rows, cols] (cols contiguous) with a
+// box of {64 columns, box_rows rows} and the 128-byte swizzle.
+int make_tmap_bf16_2d(ic_ctx* ctx, CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                      uint32_t box_rows);
+// Same for an 8-bit tensor, box {128 columns, box_rows rows}, no swizzle.
+int make_tmap_u8_2d(ic_ctx* ctx, CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
+                    uint32_t box_cols, uint32_t box_rows);
+
+// ----------------------------------------------------------------- launchers
+int launch_index_score_prefill(ic_ctx* ctx, const void* qI, const void* kI, const void* w, int L,
+                               int H_I, int d_I, int row_begin, int row_end, float* scores,
+                               int64_t ld, cudaStream_t stream);
+int launch_index_score_decode(ic_ctx* ctx, const void* q, const void* w, const uint8_t* kI8,
+                              const float* kI_scale, const int32_t* seq_len, int B, int S_max,
+                              int H_I, int d_I, float* scores, int64_t ld, cudaStream_t stream);
+int launch_topk(ic_ctx* ctx, const float* scores, int64_t ld, int rows, int k, int causal_base,
+                const int32_t* row_len, int max_len, int32_t* idx_out, int64_t ld_out,
+                cudaStream_t stream);
+int launch_sparse_attn(ic_ctx* ctx, const void* Q, const void* K, const void* V,
+                       const int32_t* idx, int rows, int Hq, int d, int k, int rows_per_seq,
+                       int64_t kv_seq_stride, int kv_len, float scale, void* out,
+                       cudaStream_t stream);
+
+}  // namespace ic

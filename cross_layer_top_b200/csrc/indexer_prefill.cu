@@ -1,0 +1,378 @@
+// Prefill lightning-indexer score on tcgen05 tensor cores.
+//
+// Computes, for query rows t in [row_begin, row_end) and keys s <= t,
+//   I[t,s] = sum_j w[t,j] * ReLU(q_I[t,j,:] . k_I[s,:])
+// ("IndexCache：跨层复用稀疏索引，以及它为什么能被训练", §2.1, the DSA
+// lightning-indexer score; "IndexCache: Accelerating Sparse Attention via
+// Cross-Layer Index Reuse", §2.1: the indexer scores all preceding tokens).
+//
+// Design (sm_100a):
+//  * The contraction is arranged "keys as M": A = a tile of 128 keys of k_I
+//    (K-major, 128-byte swizzle, loaded by TMA), B = the (token, head) rows
+//    of q_I for a block of query tokens (K-major, same swizzle).  One UMMA
+//    (M=128, N=256, K=16, bf16 in, fp32 accumulate) gives per-head dot
+//    products D[s, (t,j)] in TMEM: lane = key, column = (token, head).
+//  * The epilogue thread that owns TMEM lane s therefore holds all heads of
+//    (t, s) in its own registers: ReLU, the w[t,j] weighting and the sum over
+//    heads run without any cross-thread reduction, and only I[t,s] (fp32)
+//    is stored.  The per-head [H_I, L, L] tensor never reaches HBM.
+//  * A work item is TQ = 2 * 256/H_I query tokens; its q_I block stays in
+//    shared memory while the causal key tiles 0..t_last/128 stream through
+//    a TMA ring.  Two 256-column TMEM accumulators ping-pong so the epilogue
+//    of one overlaps the MMAs of the other.
+//  * Warp roles (384 threads, one CTA per SM, persistent): warp 0 = TMA
+//    producer, warp 1 = MMA issuer, warp 2 = TMEM allocator, warps 4..11 =
+//    epilogue (warp w reads TMEM lanes 32*(w%4).., columns half (w-4)/4).
+//  * Work items are handed out longest-first (latest rows first), round
+//    robin over the persistent CTAs.
+//  * Every mbarrier wait is bounded; on timeout the CTA aborts cleanly
+//    (drains its TMA loads and MMAs, frees TMEM) and latches an error code.
+#include "ic_device.cuh"
+#include "ic_internal.h"
+
+namespace ic {
+
+template <int H_I, int NATOM>
+struct PrefillShape {
+    static constexpr int BM = 128;                 // keys per tile (UMMA M, TMEM lanes)
+    static constexpr int BN = 256;                 // (token, head) columns per accumulator
+    static constexpr int NACC = 2;                 // TMEM accumulators (2 x 256 = 512 columns)
+    static constexpr int TOK_PER_ACC = BN / H_I;
+    static constexpr int TQ = NACC * TOK_PER_ACC;  // query tokens per work item
+    static constexpr int A_ATOM = BM * 128;        // one 64-element K slice of a key tile
+    static constexpr int A_STAGE = NATOM * A_ATOM;
+    static constexpr int B_ATOM = BN * 128;
+    static constexpr int B_ACC = NATOM * B_ATOM;
+    static constexpr int B_BYTES = NACC * B_ACC;
+    static constexpr int W_BYTES = 8 * 1024;       // per epilogue warp: 256 fp32 weights
+    static constexpr int BAR_BYTES = 256;
+    static constexpr int SMEM_CAP = 232448;
+    static constexpr int KST_RAW = (SMEM_CAP - B_BYTES - W_BYTES - BAR_BYTES) / A_STAGE;
+    static constexpr int KSTAGES = KST_RAW > 6 ? 6 : KST_RAW;
+    static constexpr int SMEM = B_BYTES + KSTAGES * A_STAGE + W_BYTES + BAR_BYTES;
+    static_assert(KSTAGES >= 2, "shared memory too small for the key ring");
+    static_assert(SMEM <= SMEM_CAP, "shared memory budget");
+    static_assert(64 % H_I == 0, "H_I must divide 64");
+};
+
+// Score 64 consecutive accumulator columns held in va (cols 0..31) and vb
+// (cols 32..63); wcol points at the fp32 weights of those 64 columns
+// (token-major, head-minor, same order as the columns).  Produces one score
+// per token covered (64 / H_I tokens).
+template <int H_I>
+__device__ __forceinline__ void score64(const uint32_t (&va)[32], const uint32_t (&vb)[32],
+                                        const float* wcol, float (&out)[64 / H_I]) {
+    constexpr int NT = 64 / H_I;
+#pragma unroll
+    for (int tt = 0; tt < NT; ++tt) {
+        float p[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int j = 0; j < H_I; j += 4) {
+            const int c = tt * H_I + j;
+            const float4 wv = *reinterpret_cast<const float4*>(wcol + c);
+            const float x0 = __uint_as_float(c + 0 < 32 ? va[(c + 0) & 31] : vb[(c + 0) & 31]);
+            const float x1 = __uint_as_float(c + 1 < 32 ? va[(c + 1) & 31] : vb[(c + 1) & 31]);
+            const float x2 = __uint_as_float(c + 2 < 32 ? va[(c + 2) & 31] : vb[(c + 2) & 31]);
+            const float x3 = __uint_as_float(c + 3 < 32 ? va[(c + 3) & 31] : vb[(c + 3) & 31]);
+            p[0] = fmaf(wv.x, fmaxf(x0, 0.f), p[0]);
+            p[1] = fmaf(wv.y, fmaxf(x1, 0.f), p[1]);
+            p[2] = fmaf(wv.z, fmaxf(x2, 0.f), p[2]);
+            p[3] = fmaf(wv.w, fmaxf(x3, 0.f), p[3]);
+        }
+        out[tt] = (p[0] + p[1]) + (p[2] + p[3]);
+    }
+}
+
+template <int H_I, int NATOM>
+__global__ void __launch_bounds__(384, 1)
+    k_index_score_prefill(const __grid_constant__ CUtensorMap tm_q,
+                          const __grid_constant__ CUtensorMap tm_k,
+                          const __nv_bfloat16* __restrict__ w, float* __restrict__ scores,
+                          long long ld, int L, int row_begin, int row_end, int n_items,
+                          int* __restrict__ err) {
+    using S = PrefillShape<H_I, NATOM>;
+    constexpr int KST = S::KSTAGES;
+    extern __shared__ __align__(1024) uint8_t smem[];
+    uint8_t* sB = smem;
+    uint8_t* sA = smem + S::B_BYTES;
+    float* sW = reinterpret_cast<float*>(sA + KST * S::A_STAGE);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(sW) + S::W_BYTES);
+    uint64_t* a_full = bars;
+    uint64_t* a_empty = bars + KST;
+    uint64_t* q_full = bars + 2 * KST;
+    uint64_t* q_empty = q_full + 1;
+    uint64_t* acc_full = q_full + 2;   // [2]
+    uint64_t* acc_empty = q_full + 4;  // [2]
+    uint64_t* done_bar = q_full + 6;
+    uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+    const int warp = threadIdx.x >> 5;
+    const int lane = threadIdx.x & 31;
+
+    if (threadIdx.x == 0) {
+        *abort_flag = 0;
+        if (smem_u32(smem) & 1023u) {
+            *abort_flag = 1;
+            atomicCAS(err, 0, kDevSmemMisaligned);
+        }
+        for (int i = 0; i < KST; ++i) {
+            mbar_init(&a_full[i], 1);
+            mbar_init(&a_empty[i], 1);
+        }
+        mbar_init(q_full, 1);
+        mbar_init(q_empty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&acc_full[i], 1);
+            mbar_init(&acc_empty[i], 8);  // one arrival per epilogue warp
+        }
+        mbar_init(done_bar, 1);
+        fence_mbar_init();
+        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
+    }
+    if (warp == 2) {
+        tmem_alloc(tmem_slot, 512);
+        tmem_relinquish();
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const bool start_ok = (*abort_flag == 0);
+
+    if (warp == 0 && lane == 0 && start_ok) {
+        // ------------------------------------------------ TMA producer
+        int st = 0;
+        uint32_t ph = 0, q_it = 0;
+        int last_ph[KST];
+#pragma unroll
+        for (int i = 0; i < KST; ++i) last_ph[i] = -1;
+        int q_last = -1;
+        bool ok = true;
+        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+            const int t0 = row_begin + (n_items - 1 - it) * S::TQ;
+            const int t_last = min(t0 + S::TQ, row_end) - 1;
+            const int n_tiles = t_last / S::BM + 1;
+            if (!mbar_wait(q_empty, (q_it & 1) ^ 1, abort_flag, err, kDevTimeoutProducer)) {
+                ok = false;
+                break;
+            }
+            mbar_arrive_expect_tx(q_full, S::B_BYTES);
+#pragma unroll
+            for (int a = 0; a < S::NACC; ++a)
+#pragma unroll
+                for (int k = 0; k < NATOM; ++k)
+                    tma_load_2d(sB + a * S::B_ACC + k * S::B_ATOM, &tm_q, q_full, k * 64,
+                                (t0 + a * S::TOK_PER_ACC) * H_I);
+            q_last = q_it & 1;
+            ++q_it;
+            for (int kt = 0; kt < n_tiles; ++kt) {
+                if (!mbar_wait(&a_empty[st], ph ^ 1, abort_flag, err, kDevTimeoutProducer)) {
+                    ok = false;
+                    break;
+                }
+                mbar_arrive_expect_tx(&a_full[st], S::A_STAGE);
+#pragma unroll
+                for (int k = 0; k < NATOM; ++k)
+                    tma_load_2d(sA + st * S::A_STAGE + k * S::A_ATOM, &tm_k, &a_full[st], k * 64,
+                                kt * S::BM);
+                last_ph[st] = static_cast<int>(ph);
+                if (++st == KST) {
+                    st = 0;
+                    ph ^= 1;
+                }
+            }
+        }
+        // No TMA write may still be landing in shared memory when the CTA exits.
+        for (int i = 0; i < KST; ++i)
+            if (last_ph[i] >= 0) mbar_wait_drain(&a_full[i], static_cast<uint32_t>(last_ph[i]));
+        if (q_last >= 0) mbar_wait_drain(q_full, static_cast<uint32_t>(q_last));
+    } else if (warp == 1 && lane == 0 && start_ok) {
+        // ------------------------------------------------ MMA issuer
+        constexpr uint32_t IDESC = idesc_bf16_f32(S::BM, S::BN);
+        int st = 0;
+        uint32_t ph = 0, q_it = 0;
+        uint32_t acc_it[2] = {0, 0};
+        bool ok = true;
+        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+            const int t0 = row_begin + (n_items - 1 - it) * S::TQ;
+            const int t_last = min(t0 + S::TQ, row_end) - 1;
+            const int n_tiles = t_last / S::BM + 1;
+            if (!mbar_wait(q_full, q_it & 1, abort_flag, err, kDevTimeoutMma)) {
+                ok = false;
+                break;
+            }
+            ++q_it;
+            tc_fence_after();
+            for (int kt = 0; kt < n_tiles && ok; ++kt) {
+                if (!mbar_wait(&a_full[st], ph, abort_flag, err, kDevTimeoutMma)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    if (!mbar_wait(&acc_empty[a], (acc_it[a] & 1) ^ 1, abort_flag, err,
+                                   kDevTimeoutMma)) {
+                        ok = false;
+                        break;
+                    }
+                    tc_fence_after();
+                    const uint32_t d_tmem = tmem + static_cast<uint32_t>(a * S::BN);
+#pragma unroll
+                    for (int k = 0; k < NATOM; ++k)
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t ad = sdesc_k_sw128(
+                                smem_u32(sA + st * S::A_STAGE + k * S::A_ATOM + kk * 32));
+                            const uint64_t bd = sdesc_k_sw128(
+                                smem_u32(sB + a * S::B_ACC + k * S::B_ATOM + kk * 32));
+                            umma_bf16(d_tmem, ad, bd, IDESC, (k | kk) != 0 ? 1u : 0u);
+                        }
+                    umma_commit(&acc_full[a]);
+                    ++acc_it[a];
+                }
+                if (!ok) break;
+                umma_commit(&a_empty[st]);
+                if (++st == KST) {
+                    st = 0;
+                    ph ^= 1;
+                }
+            }
+            if (!ok) break;
+            umma_commit(q_empty);
+        }
+        // Every MMA this thread issued completes before TMEM is released.
+        umma_commit(done_bar);
+        if (!mbar_wait_drain(done_bar, 0)) atomicCAS(err, 0, kDevTimeoutDrain);
+    } else if (warp >= 4 && start_ok) {
+        // ------------------------------------------------ epilogue
+        const int ew = warp - 4;  // 0..7
+        const int lq = warp & 3;  // TMEM lane quarter
+        const int cg = ew >> 2;   // column half of each accumulator
+        float* wW = sW + ew * 256;  // this warp's weights: [acc][128 columns]
+        uint32_t acc_it[2] = {0, 0};
+        bool ok = true;
+        constexpr int TOK_PER_HALF = 128 / H_I;  // tokens in this warp's 128 columns
+        for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
+            const int t0 = row_begin + (n_items - 1 - it) * S::TQ;
+            const int t_last = min(t0 + S::TQ, row_end) - 1;
+            const int n_tiles = t_last / S::BM + 1;
+            // weights of this warp's columns, widened to fp32 (private copy)
+            __syncwarp();
+#pragma unroll
+            for (int a = 0; a < 2; ++a) {
+                const int tok0 = t0 + a * S::TOK_PER_ACC + cg * TOK_PER_HALF;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int c = lane * 4 + q;  // column within the half
+                    const int t = tok0 + c / H_I;
+                    wW[a * 128 + c] =
+                        t < L ? __bfloat162float(w[static_cast<size_t>(t) * H_I + (c % H_I)]) : 0.f;
+                }
+            }
+            __syncwarp();
+            for (int kt = 0; kt < n_tiles && ok; ++kt) {
+                const int s = kt * S::BM + lq * 32 + lane;
+#pragma unroll
+                for (int a = 0; a < 2; ++a) {
+                    bool got = mbar_wait(&acc_full[a], acc_it[a] & 1, abort_flag, err,
+                                         kDevTimeoutEpilogue);
+                    got = __all_sync(0xffffffffu, got);
+                    if (!got) {
+                        ok = false;
+                        break;
+                    }
+                    ++acc_it[a];
+                    tc_fence_after();
+                    const uint32_t taddr = tmem + (static_cast<uint32_t>(lq * 32) << 16) +
+                                           static_cast<uint32_t>(a * S::BN + cg * 128);
+                    const int tok_base = a * S::TOK_PER_ACC + cg * TOK_PER_HALF;
+                    uint32_t va[32], vb[32];
+                    float sc[64 / H_I];
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        tmem_ld32(taddr + h * 64, va);
+                        tmem_ld32(taddr + h * 64 + 32, vb);
+                        tmem_ld_wait();
+                        if (h == 1) {
+                            // all of this accumulator is in registers: hand it back
+                            tc_fence_before();
+                            __syncwarp();
+                            if (lane == 0) mbar_arrive(&acc_empty[a]);
+                        }
+                        score64<H_I>(va, vb, wW + a * 128 + h * 64, sc);
+#pragma unroll
+                        for (int tt = 0; tt < 64 / H_I; ++tt) {
+                            const int t = t0 + tok_base + h * (64 / H_I) + tt;
+                            if (t < row_end && s <= t)
+                                scores[static_cast<long long>(t - row_begin) * ld + s] = sc[tt];
+                        }
+                    }
+                }
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 2) {
+        tc_fence_after();
+        tmem_dealloc(tmem, 512);
+    }
+}
+
+template <int H_I, int NATOM>
+static int launch_prefill_t(ic_ctx* ctx, const void* qI, const void* kI, const void* w, int L,
+                            int d_I, int row_begin, int row_end, float* scores, int64_t ld,
+                            cudaStream_t stream) {
+    using S = PrefillShape<H_I, NATOM>;
+    auto kern = k_index_score_prefill<H_I, NATOM>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e =
+            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
+        if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaFuncSetAttribute(index_score)");
+        attr_set = true;
+    }
+    CUtensorMap tm_q, tm_k;
+    int rc = make_tmap_bf16_2d(ctx, &tm_q, qI, static_cast<uint64_t>(L) * H_I, d_I, S::BN);
+    if (rc) return rc;
+    rc = make_tmap_bf16_2d(ctx, &tm_k, kI, static_cast<uint64_t>(L), d_I, S::BM);
+    if (rc) return rc;
+    const int n_items = (row_end - row_begin + S::TQ - 1) / S::TQ;
+    const int grid = n_items < ctx->num_sms ? n_items : ctx->num_sms;
+    LaunchScope ls(ctx, IC_K_INDEX_SCORE, stream);
+    k_index_score_prefill<H_I, NATOM><<<grid, 384, S::SMEM, stream>>>(
+        tm_q, tm_k, static_cast<const __nv_bfloat16*>(w), scores, static_cast<long long>(ld), L,
+        row_begin, row_end, n_items, ctx->dev_err);
+    cudaError_t e = ls.done();
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "index_score launch");
+    return IC_OK;
+}
+
+int launch_index_score_prefill(ic_ctx* ctx, const void* qI, const void* kI, const void* w, int L,
+                               int H_I, int d_I, int row_begin, int row_end, float* scores,
+                               int64_t ld, cudaStream_t stream) {
+    if (row_end <= row_begin) return IC_OK;
+    const bool one_atom = d_I <= 64;
+#define IC_PREFILL_CASE(H)                                                                      \
+    case H:                                                                                     \
+        return one_atom ? launch_prefill_t<H, 1>(ctx, qI, kI, w, L, d_I, row_begin, row_end,    \
+                                                 scores, ld, stream)                            \
+                        : launch_prefill_t<H, 2>(ctx, qI, kI, w, L, d_I, row_begin, row_end,    \
+                                                 scores, ld, stream);
+    switch (H_I) {
+        IC_PREFILL_CASE(4)
+        IC_PREFILL_CASE(8)
+        IC_PREFILL_CASE(16)
+        IC_PREFILL_CASE(32)
+        IC_PREFILL_CASE(64)
+        default:
+            return fail(ctx, IC_ERR_UNSUPPORTED, "index_score: H_I=%d not in {4,8,16,32,64}", H_I);
+    }
+#undef IC_PREFILL_CASE
+}
+
+}  // namespace ic

@@ -1,0 +1,361 @@
+// Sparse MQA attention over gathered K/V rows:
+//   o[r,h,:] = sum_{s in T_r} softmax_s(scale * Q[r,h,:].K[s,:]) V[s,:]
+// ("IndexCache：跨层复用稀疏索引，以及它为什么能被训练", §3: each layer keeps
+// its own Q/K/V and attends at the shared positions T_t; "IndexCache:
+// Accelerating Sparse Attention via Cross-Layer Index Reuse", Figure 2 step
+// SPARSEATTN).  One K/V head is shared by all Hq <= 16 query heads.
+//
+// Design: one CTA (4 warps) per (query row, key split).  The 16 query heads
+// form the M = 16 rows of mma.m16n8k16 tiles, so one gathered K/V row serves
+// every head.  Each warp owns chunks of 16 index slots and runs its own
+// 3-stage cp.async ring: the 16 selected K rows and V rows (d*2 bytes each,
+// 16-byte pieces, XOR-swizzled in shared memory so ldmatrix is
+// conflict-free) are gathered while the previous chunk computes
+// S = Q K^T, an online softmax (fp32, base-2 exponent with the scale folded
+// in) and O += P V.  The four warps' (m, l, O) are merged through shared
+// memory; with one split the CTA writes bf16 output, otherwise fp32
+// partials that k_attn_combine merges (decode: few rows, many splits).
+// Invalid slots (-1, or outside [0, kv_len): latched as an error) are
+// masked and gather nothing.
+#include "ic_device.cuh"
+#include "ic_internal.h"
+
+namespace ic {
+
+template <int D>
+struct AttnShape {
+    static constexpr int WARPS = 4;
+    static constexpr int THREADS = WARPS * 32;
+    static constexpr int CH = 16;  // index slots per warp chunk
+    static constexpr int STAGES = 3;
+    static constexpr int ROWB = D * 2;
+    static constexpr int PIECES = D / 8;  // 16-byte pieces per row
+    static constexpr int CHUNK_BYTES = CH * ROWB;
+    static constexpr int STAGE_BYTES = 2 * CHUNK_BYTES;  // K and V
+    static constexpr int WARP_BYTES = STAGES * STAGE_BYTES;
+    static constexpr int Q_BYTES = 16 * ROWB;
+    static constexpr int MAXK = 2048;
+    static constexpr int OFF_Q = 0;
+    static constexpr int OFF_IDX = Q_BYTES;
+    static constexpr int OFF_ST = OFF_IDX + MAXK * 4;
+    static constexpr int SMEM = OFF_ST + WARPS * WARP_BYTES;
+    // merge buffers (alias the stages once every warp is done)
+    static constexpr int MERGE_BYTES = WARPS * (16 * D + 32) * 4;
+    static_assert(MERGE_BYTES <= WARPS * WARP_BYTES, "merge buffer must fit in the stages");
+};
+
+// byte offset of 16-byte piece `c` of row `row` in a swizzled [rows][D] tile
+template <int D>
+__device__ __forceinline__ uint32_t swz(int row, int c) {
+    return static_cast<uint32_t>(row * (D * 2) + ((c ^ (row & 7)) << 4));
+}
+
+template <int D>
+__global__ void __launch_bounds__(AttnShape<D>::THREADS)
+    k_sparse_attn(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
+                  const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ idx, int Hq,
+                  int k, int rows_per_seq, long long kv_seq_stride, int kv_len, float scale_log2,
+                  int nsplit, int kps, __nv_bfloat16* __restrict__ out,
+                  float* __restrict__ part, int* __restrict__ err) {
+    using S = AttnShape<D>;
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int r = blockIdx.x, split = blockIdx.y;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int slot0 = split * kps;
+    const int nk = max(0, min(k, slot0 + kps) - slot0);
+    int32_t* sIdx = reinterpret_cast<int32_t*>(smem + S::OFF_IDX);
+    const uint32_t sQ = smem_u32(smem + S::OFF_Q);
+    const long long seq = rows_per_seq > 0 ? r / rows_per_seq : 0;
+    const __nv_bfloat16* Kb = K + seq * kv_seq_stride;
+    const __nv_bfloat16* Vb = V + seq * kv_seq_stride;
+
+    // index slots of this split (validated) and the query heads
+    const int32_t* irow = idx + static_cast<long long>(r) * k + slot0;
+    bool bad = false;
+    for (int i = tid; i < nk; i += S::THREADS) {
+        int v = irow[i];
+        if (v < -1 || v >= kv_len) {
+            bad = true;
+            v = -1;
+        }
+        sIdx[i] = v;
+    }
+    if (bad) atomicCAS(err, 0, kDevBadIndex);
+    const __nv_bfloat16* qrow = Q + static_cast<long long>(r) * Hq * D;
+    for (int p = tid; p < 16 * S::PIECES; p += S::THREADS) {
+        const int h = p / S::PIECES, c = p % S::PIECES;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (h < Hq) v = *reinterpret_cast<const uint4*>(qrow + h * D + c * 8);
+        *reinterpret_cast<uint4*>(smem + S::OFF_Q + swz<D>(h, c)) = v;
+    }
+    __syncthreads();
+
+    // Q fragments (A operand, 16 heads x D)
+    uint32_t qa[D / 16][4];
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        const int m = lane >> 3;
+        const int row = (m & 1) * 8 + (lane & 7);
+        const int c = 2 * kk + (m >> 1);
+        ldsm_x4(sQ + swz<D>(row, c), qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
+    }
+
+    const uint32_t wst = smem_u32(smem + S::OFF_ST + warp * S::WARP_BYTES);
+    const int nch = (nk + S::CH - 1) / S::CH;
+    // chunks of this warp: warp, warp + WARPS, ...
+    const int my_n = nch > warp ? (nch - warp + S::WARPS - 1) / S::WARPS : 0;
+
+    auto issue = [&](int j) {
+        if (j < my_n) {
+            const int c0 = (warp + j * S::WARPS) * S::CH;
+            const uint32_t kb = wst + (j % S::STAGES) * S::STAGE_BYTES;
+            const uint32_t vb = kb + S::CHUNK_BYTES;
+#pragma unroll
+            for (int p = lane; p < S::CH * S::PIECES; p += 32) {
+                const int key = p / S::PIECES, c = p % S::PIECES;
+                const int slot = c0 + key;
+                const int s = slot < nk ? sIdx[slot] : -1;
+                const bool ok = s >= 0;
+                const long long off = static_cast<long long>(ok ? s : 0) * D + c * 8;
+                cp_async16(kb + swz<D>(key, c), Kb + off, ok);
+                cp_async16(vb + swz<D>(key, c), Vb + off, ok);
+            }
+        }
+        cp_async_commit();
+    };
+
+    float o[D / 8][4];
+#pragma unroll
+    for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // rows g and g+8
+
+#pragma unroll
+    for (int j = 0; j < S::STAGES - 1; ++j) issue(j);
+
+    for (int j = 0; j < my_n; ++j) {
+        cp_async_wait<S::STAGES - 2>();
+        __syncwarp();
+        const uint32_t kb = wst + (j % S::STAGES) * S::STAGE_BYTES;
+        const uint32_t vb = kb + S::CHUNK_BYTES;
+        const int c0 = (warp + j * S::WARPS) * S::CH;
+
+        float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const int m = lane >> 3;
+            const int key = (m >> 1) * 8 + (lane & 7);
+            const int c = 2 * kk + (m & 1);
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4(kb + swz<D>(key, c), b0, b1, b2, b3);
+            mma_bf16_16816(s[0], qa[kk], b0, b1);
+            mma_bf16_16816(s[1], qa[kk], b2, b3);
+        }
+        // mask invalid slots, scale into the base-2 domain
+        float x[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int col = nt * 8 + 2 * (lane & 3) + (e & 1);
+                const int slot = c0 + col;
+                const bool ok = slot < nk && sIdx[slot] >= 0;
+                x[nt][e] = ok ? s[nt][e] * scale_log2 : -INFINITY;
+            }
+        float mx0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+        float mx1 = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
+        // reference points that stay finite while a row has seen nothing
+        const float r0 = n0 == -INFINITY ? 0.f : n0;
+        const float r1 = n1 == -INFINITY ? 0.f : n1;
+        const float a0 = exp2f(m0 - r0), a1 = exp2f(m1 - r1);
+        m0 = n0;
+        m1 = n1;
+        float p[2][4];
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            p[nt][0] = exp2f(x[nt][0] - r0);
+            p[nt][1] = exp2f(x[nt][1] - r0);
+            p[nt][2] = exp2f(x[nt][2] - r1);
+            p[nt][3] = exp2f(x[nt][3] - r1);
+        }
+        l0 = l0 * a0 + (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+        l1 = l1 * a1 + (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) {
+            o[i][0] *= a0;
+            o[i][1] *= a0;
+            o[i][2] *= a1;
+            o[i][3] *= a1;
+        }
+        uint32_t pa[4];
+        pa[0] = pack_bf16x2(p[0][0], p[0][1]);
+        pa[1] = pack_bf16x2(p[0][2], p[0][3]);
+        pa[2] = pack_bf16x2(p[1][0], p[1][1]);
+        pa[3] = pack_bf16x2(p[1][2], p[1][3]);
+#pragma unroll
+        for (int dn = 0; dn < D / 16; ++dn) {
+            const int m = lane >> 3;
+            const int key = (m & 1) * 8 + (lane & 7);
+            const int c = 2 * dn + (m >> 1);
+            uint32_t b0, b1, b2, b3;
+            ldsm_x4_t(vb + swz<D>(key, c), b0, b1, b2, b3);
+            mma_bf16_16816(o[2 * dn], pa, b0, b1);
+            mma_bf16_16816(o[2 * dn + 1], pa, b2, b3);
+        }
+        __syncwarp();
+        issue(j + S::STAGES - 1);
+    }
+    cp_async_wait<0>();
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
+    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
+    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    __syncthreads();  // every warp is done with its stages: reuse them for the merge
+
+    float* mO = reinterpret_cast<float*>(smem + S::OFF_ST);  // [WARPS][16][D]
+    float* mML = mO + S::WARPS * 16 * D;                     // [WARPS][32]: m[16], l[16]
+    {
+        const int g = lane >> 2, cc = 2 * (lane & 3);
+        float* ow = mO + warp * 16 * D;
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) {
+            *reinterpret_cast<float2*>(ow + g * D + i * 8 + cc) = make_float2(o[i][0], o[i][1]);
+            *reinterpret_cast<float2*>(ow + (g + 8) * D + i * 8 + cc) = make_float2(o[i][2], o[i][3]);
+        }
+        if ((lane & 3) == 0) {
+            mML[warp * 32 + g] = m0;
+            mML[warp * 32 + g + 8] = m1;
+            mML[warp * 32 + 16 + g] = l0;
+            mML[warp * 32 + 16 + g + 8] = l1;
+        }
+    }
+    __syncthreads();
+    const int hmax = nsplit == 1 ? Hq : 16;
+    for (int e = tid; e < hmax * D; e += S::THREADS) {
+        const int h = e / D, dd = e % D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < S::WARPS; ++w) M = fmaxf(M, mML[w * 32 + h]);
+        float acc = 0.f, lsum = 0.f;
+        if (M != -INFINITY) {
+#pragma unroll
+            for (int w = 0; w < S::WARPS; ++w) {
+                const float f = exp2f(mML[w * 32 + h] - M);
+                acc += mO[w * 16 * D + h * D + dd] * f;
+                lsum += mML[w * 32 + 16 + h] * f;
+            }
+        }
+        if (nsplit == 1) {
+            const float v = lsum > 0.f ? acc / lsum : 0.f;
+            out[(static_cast<long long>(r) * Hq + h) * D + dd] = __float2bfloat16_rn(v);
+        } else {
+            float* pr = part + (static_cast<long long>(r) * nsplit + split) * (16 * D + 32);
+            pr[h * D + dd] = acc;
+            if (dd == 0) {
+                pr[16 * D + h] = M;
+                pr[16 * D + 16 + h] = lsum;
+            }
+        }
+    }
+}
+
+// Merge the per-split partials of each row: out = sum_s O_s 2^(m_s - M) / sum_s l_s 2^(m_s - M).
+template <int D>
+__global__ void __launch_bounds__(256)
+    k_attn_combine(const float* __restrict__ part, int Hq, int nsplit,
+                   __nv_bfloat16* __restrict__ out) {
+    const int r = blockIdx.x;
+    const float* pr = part + static_cast<long long>(r) * nsplit * (16 * D + 32);
+    for (int e = threadIdx.x; e < Hq * D; e += blockDim.x) {
+        const int h = e / D, dd = e % D;
+        float M = -INFINITY;
+        for (int s = 0; s < nsplit; ++s) M = fmaxf(M, pr[s * (16 * D + 32) + 16 * D + h]);
+        float acc = 0.f, lsum = 0.f;
+        if (M != -INFINITY) {
+            for (int s = 0; s < nsplit; ++s) {
+                const float* ps = pr + s * (16 * D + 32);
+                const float f = exp2f(ps[16 * D + h] - M);
+                acc += ps[h * D + dd] * f;
+                lsum += ps[16 * D + 16 + h] * f;
+            }
+        }
+        out[(static_cast<long long>(r) * Hq + h) * D + dd] =
+            __float2bfloat16_rn(lsum > 0.f ? acc / lsum : 0.f);
+    }
+}
+
+template <int D>
+static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* V,
+                         const int32_t* idx, int rows, int Hq, int k, int rows_per_seq,
+                         int64_t kv_seq_stride, int kv_len, float scale, void* out,
+                         cudaStream_t stream) {
+    using S = AttnShape<D>;
+    static bool attr_set = false;
+    if (!attr_set) {
+        cudaError_t e = cudaFuncSetAttribute(k_sparse_attn<D>,
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
+        if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaFuncSetAttribute(sparse_attn)");
+        attr_set = true;
+    }
+    // Split the index slots across CTAs when there are too few rows to fill
+    // the GPU (decode): aim for ~4 CTAs per SM, at least 64 slots per split.
+    int nsplit = 1;
+    const int target = 4 * ctx->num_sms;
+    if (rows < target) {
+        nsplit = (target + rows - 1) / rows;
+        const int max_split = (k + 63) / 64;
+        if (nsplit > max_split) nsplit = max_split;
+        if (nsplit < 1) nsplit = 1;
+    }
+    int kps = (k + nsplit - 1) / nsplit;
+    kps = (kps + S::CH - 1) / S::CH * S::CH;
+    nsplit = (k + kps - 1) / kps;
+    float* part = nullptr;
+    if (nsplit > 1) {
+        const size_t bytes = static_cast<size_t>(rows) * nsplit * (16 * D + 32) * sizeof(float);
+        int rc = ensure_buffer(ctx, reinterpret_cast<void**>(&ctx->attn_part), &ctx->attn_part_cap,
+                               bytes);
+        if (rc) return rc;
+        part = ctx->attn_part;
+    }
+    const float scale_log2 = scale * 1.4426950408889634f;
+    {
+        LaunchScope ls(ctx, IC_K_ATTN, stream);
+        dim3 grid(rows, nsplit);
+        k_sparse_attn<D><<<grid, S::THREADS, S::SMEM, stream>>>(
+            static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
+            static_cast<const __nv_bfloat16*>(V), idx, Hq, k, rows_per_seq,
+            static_cast<long long>(kv_seq_stride), kv_len, scale_log2, nsplit, kps,
+            static_cast<__nv_bfloat16*>(out), part, ctx->dev_err);
+        cudaError_t e = ls.done();
+        if (e != cudaSuccess) return cuda_fail(ctx, e, "sparse_attn launch");
+    }
+    if (nsplit > 1) {
+        LaunchScope ls(ctx, IC_K_ATTN_COMBINE, stream);
+        k_attn_combine<D><<<rows, 256, 0, stream>>>(part, Hq, nsplit,
+                                                    static_cast<__nv_bfloat16*>(out));
+        cudaError_t e = ls.done();
+        if (e != cudaSuccess) return cuda_fail(ctx, e, "attn_combine launch");
+    }
+    return IC_OK;
+}
+
+int launch_sparse_attn(ic_ctx* ctx, const void* Q, const void* K, const void* V,
+                       const int32_t* idx, int rows, int Hq, int d, int k, int rows_per_seq,
+                       int64_t kv_seq_stride, int kv_len, float scale, void* out,
+                       cudaStream_t stream) {
+    if (rows <= 0) return IC_OK;
+    if (d == 128)
+        return launch_attn_t<128>(ctx, Q, K, V, idx, rows, Hq, k, rows_per_seq, kv_seq_stride,
+                                  kv_len, scale, out, stream);
+    if (d == 64)
+        return launch_attn_t<64>(ctx, Q, K, V, idx, rows, Hq, k, rows_per_seq, kv_seq_stride,
+                                 kv_len, scale, out, stream);
+    return fail(ctx, IC_ERR_UNSUPPORTED, "sparse_attn: d=%d not in {64,128}", d);
+}
+
+}  // namespace ic

@@ -1,0 +1,233 @@
+/*
+ * indexcache.h — C ABI of libindexcache.so, the B200 (sm_100a) hot path of
+ * DeepSeek Sparse Attention with IndexCache (cross-layer top-k index reuse).
+ *
+ * The operations follow two web pages, cited by title and section:
+ *   [IC] "IndexCache: Accelerating Sparse Attention via Cross-Layer Index
+ *        Reuse" (paper summary): method details (pattern c in {F,S}^N,
+ *        f(l) = max{j<l : c_j = F}, first layer F), Figure 2 (inference
+ *        loop: F layers run the indexer and top-k and overwrite the cache,
+ *        S layers copy the cached indices, every layer runs sparse
+ *        attention), §2.1 (top-k with k = 2048, FP8 indexer arithmetic),
+ *        §3.1.1 (uniform interleave).
+ *   [RN] "IndexCache：跨层复用稀疏索引，以及它为什么能被训练" (reading notes):
+ *        §2.1 indexer score I[t,s] = sum_j w[t,j] ReLU(q_I[t,j] . k_I[s]);
+ *        §2.2 the cache holds the current index tensor only; §3 sparse
+ *        attention o_t = sum_{s in T_t} softmax(Q_t.K_s/sqrt(d)) V_s;
+ *        §10.1 decode scans the whole indexer key cache per token; §11 S
+ *        layers keep no indexer key cache.
+ *
+ * Conventions (all calls):
+ *  - Tensors are caller-owned DEVICE pointers, row-major and contiguous,
+ *    with the sizes passed explicitly.  bf16 tensors are passed as void*.
+ *    Tensors read by TMA (q_I, k_I) must be 16-byte aligned.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream).  They return after enqueueing work.
+ *  - Every call returns IC_OK (0) or an IC_ERR_* code and never throws.  The
+ *    message of the last failure is ic_last_error(ctx).  Argument errors are
+ *    detected on the host before anything is enqueued.  Errors found on the
+ *    device (a bounded wait that ran out, an index outside [-1, kv_len))
+ *    are latched in the context and reported by ic_sync_status().
+ *  - Positions are 0-based; causal means s <= t (the query sees itself).
+ *  - Index rows hold min(k, n) selected positions in ascending order
+ *    followed by -1 padding; ties in score go to the lower position.
+ *  - A context (ic_ctx) owns scratch memory (score rows, split-attention
+ *    partials) and the device error flag.  It is not thread-safe: use one
+ *    context per host thread / stream.
+ */
+#ifndef INDEXCACHE_H
+#define INDEXCACHE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define IC_OK 0
+#define IC_ERR_INVALID_ARG 1  /* null pointer, negative size, misaligned pointer */
+#define IC_ERR_PATTERN 2      /* pattern not over {F,S} or first layer not F */
+#define IC_ERR_SHAPE 3        /* inconsistent sizes (e.g. k < 1) */
+#define IC_ERR_UNSUPPORTED 4  /* a size outside what the kernels are built for */
+#define IC_ERR_CUDA 5         /* a CUDA runtime/driver call failed */
+#define IC_ERR_TIMEOUT 6      /* a bounded device wait ran out */
+#define IC_ERR_NOMEM 7        /* scratch allocation failed */
+#define IC_ERR_DEVICE 8       /* a device-side check failed (bad index) */
+
+#define IC_PREFILL 0
+#define IC_DECODE 1
+
+/* Kernel ids for the timing counters. */
+#define IC_K_INDEX_SCORE 0        /* prefill indexer score (tcgen05) */
+#define IC_K_INDEX_SCORE_DECODE 1 /* decode FP8 indexer-key scan (tcgen05) */
+#define IC_K_TOPK 2               /* per-row top-k select */
+#define IC_K_ATTN 3               /* sparse MQA attention (gather + softmax) */
+#define IC_K_ATTN_COMBINE 4       /* split-attention combine */
+#define IC_K_COUNT 5
+
+typedef struct ic_ctx ic_ctx;
+typedef struct ic_pattern ic_pattern;
+
+/* ---------------------------------------------------------------- context */
+
+/* Library version, major*10000 + minor*100 + patch. */
+int ic_version(void);
+
+/* Create a context on CUDA `device`.  `scratch_bytes` bounds the score
+ * scratch used by ic_index_fp (0 = 2 GiB); rows are processed in chunks
+ * that fit.  Scratch is allocated lazily on first use.  *out receives the
+ * context.  Errors: IC_ERR_INVALID_ARG (out NULL), IC_ERR_CUDA. */
+int ic_ctx_create(ic_ctx **out, int device, size_t scratch_bytes);
+
+/* Free the context and its scratch (synchronizes the device first). */
+int ic_ctx_destroy(ic_ctx *ctx);
+
+/* Message of the last failure on `ctx` (or of the last ic_ctx_create /
+ * ic_create_pattern failure when ctx is NULL).  Never NULL. */
+const char *ic_last_error(const ic_ctx *ctx);
+
+/* Synchronize `stream`, then read and clear the context's device error
+ * flag.  Returns IC_OK, IC_ERR_TIMEOUT, IC_ERR_DEVICE or IC_ERR_CUDA. */
+int ic_sync_status(ic_ctx *ctx, void *stream);
+
+/* Kernel timing counters (tracing).  When enabled, every kernel the context
+ * launches is bracketed by CUDA events on its launch stream.
+ * ic_ctx_get_timing synchronizes on the last recorded event and returns the
+ * summed device time (ms) and launch count for kernel id `kernel`.
+ * ic_ctx_reset_timing clears all counters. */
+int ic_ctx_set_timing(ic_ctx *ctx, int enable);
+int ic_ctx_get_timing(ic_ctx *ctx, int kernel, double *total_ms, int64_t *launches);
+int ic_ctx_reset_timing(ic_ctx *ctx);
+/* Number of kernels this context has launched since creation (all ids). */
+int64_t ic_ctx_launch_count(const ic_ctx *ctx);
+
+/* ---------------------------------------------------------------- pattern */
+
+/* [IC] method details: parse c[0..n_layers) over {'F','S'}; c[0] must be
+ * 'F'.  Errors: IC_ERR_INVALID_ARG, IC_ERR_PATTERN.  Host only. */
+int ic_create_pattern(const char *c, int n_layers, ic_pattern **out);
+
+/* [IC] §3.1.1 uniform interleave: layer l is F iff l % r == 0. */
+int ic_pattern_uniform(int n_layers, int r, ic_pattern **out);
+
+int ic_pattern_destroy(ic_pattern *p);
+int ic_pattern_size(const ic_pattern *p);                     /* n_layers, or -1 */
+int ic_pattern_string(const ic_pattern *p, char *buf, int buflen); /* NUL-terminated */
+
+/* src_out[l] = l for an F layer, f(l) = max{j<l : c_j=F} for an S layer.
+ * src_out is a HOST array of n_layers ints. */
+int ic_pattern_src(const ic_pattern *p, int32_t *src_out);
+
+/* ------------------------------------------------------- prefill indexer */
+
+/* [RN] §2.1 lightning-indexer scores of query rows t in [row_begin,row_end):
+ *   scores[(t - row_begin)*ld + s] = sum_j w[t,j] * ReLU(q_I[t,j,:] . k_I[s,:])
+ * for s <= t; entries with s > t are not written.
+ *   q_I: bf16 [L, H_I, d_I];  k_I: bf16 [L, d_I];  w: bf16 [L, H_I].
+ *   scores: fp32, ld >= row_end, ld % 4 == 0.
+ * Supported: H_I in {4,8,16,32,64}, d_I in {32,64,128}.  fp32 accumulation
+ * on the tensor cores; exact whenever every partial sum is (e.g. small
+ * integers).  Errors: IC_ERR_INVALID_ARG, IC_ERR_UNSUPPORTED, IC_ERR_CUDA. */
+int ic_index_score(ic_ctx *ctx, const void *qI, const void *kI, const void *w, int L, int H_I,
+                   int d_I, int row_begin, int row_end, float *scores, int64_t ld, void *stream);
+
+/* Per-row top-k ([IC] notation T_t = Top-k(I_t)).  Row r has n_r candidates
+ * scores[r*ld + 0 .. n_r-1], with n_r = row_len[r] when row_len (device,
+ * int32 [rows]) is non-NULL, else n_r = causal_base + r + 1.  Writes
+ * idx_out[r*ld_out + 0..k-1]: the min(k, n_r) positions of the largest
+ * scores, ascending, ties to the lower position, then -1.  Rows with
+ * n_r <= k read no scores.  1 <= k <= 2048.  -0.0 equals +0.0. */
+int ic_topk(ic_ctx *ctx, const float *scores, int64_t ld, int rows, int k, int causal_base,
+            const int32_t *row_len, int32_t *idx_out, int64_t ld_out, void *stream);
+
+/* One prefill F layer ([IC] Figure 2, steps "I <- INDEXER(X); T <-
+ * Top-k(I); cache <- T"): idx_out int32 [L, k] (the index cache) receives
+ * T_t for every t.  Rows t < k need no score (T_t = {0..t}).  Scores go
+ * through the context's scratch in row chunks. */
+int ic_index_fp(ic_ctx *ctx, const void *qI, const void *kI, const void *w, int L, int H_I,
+                int d_I, int k, int32_t *idx_out, void *stream);
+
+/* S layer ([IC] Figure 2 "T <- cache"): the cached tensor itself is used, no
+ * copy and no kernel.  *idx_out = idx_cache. */
+int ic_index_reuse(const int32_t *idx_cache, const int32_t **idx_out);
+
+/* -------------------------------------------------------- decode indexer */
+
+/* [RN] §2.1 score for one new query per sequence against its FP8 indexer
+ * key cache ([IC] §2.1 FP8 indexer; [RN] §10.1 full scan per token):
+ *   scores[b*ld + s] = sum_j w[b,j] * ReLU(q[b,j,:] . (e4m3(kI8[b,s,:]) * kI_scale[b,s]))
+ * for s < seq_len[b].  q: bf16 [B, H_I, d_I]; w: bf16 [B, H_I];
+ * kI8: e4m3 bytes [B, S_max, d_I]; kI_scale: fp32 [B, S_max], > 0;
+ * seq_len: device int32 [B], 1 <= seq_len[b] <= S_max.  ld >= S_max.
+ * Supported: H_I in {32,64}, d_I = 128. */
+int ic_index_score_decode(ic_ctx *ctx, const void *q, const void *w, const uint8_t *kI8,
+                          const float *kI_scale, const int32_t *seq_len, int B, int S_max, int H_I,
+                          int d_I, float *scores, int64_t ld, void *stream);
+
+/* Decode F layer: scores then top-k over each sequence's seq_len[b]
+ * candidates; idx_out int32 [B, k]. */
+int ic_index_fp_decode(ic_ctx *ctx, const void *q, const void *w, const uint8_t *kI8,
+                       const float *kI_scale, const int32_t *seq_len, int B, int S_max, int H_I,
+                       int d_I, int k, int32_t *idx_out, void *stream);
+
+/* ------------------------------------------------------ sparse attention */
+
+/* [RN] §3 sparse MQA attention, every layer:
+ *   out[r,h,:] = sum_{s in idx[r,:], s >= 0} softmax_s(scale * Q[r,h,:].K[s,:]) V[s,:]
+ * Q: bf16 [rows, Hq, d]; out: bf16 [rows, Hq, d]; idx: int32 [rows, k].
+ * K, V: bf16; query row r reads the block of sequence r / rows_per_seq at
+ * K + (r / rows_per_seq) * kv_seq_stride (elements), whose rows are
+ * [kv_len, d].  One shared K/V head.  Entries -1 are skipped; an entry
+ * outside [-1, kv_len) is skipped and latched as IC_ERR_DEVICE.  A row with
+ * no valid entry produces zeros.  scale <= 0 means 1/sqrt(d).
+ * Supported: d in {64,128}, 1 <= Hq <= 16, 1 <= k <= 2048. */
+int ic_sparse_attn(ic_ctx *ctx, const void *Q, const void *K, const void *V, const int32_t *idx,
+                   int rows, int Hq, int d, int k, int rows_per_seq, int64_t kv_seq_stride,
+                   int kv_len, float scale, void *out, void *stream);
+
+/* ------------------------------------------------------------ layer stack */
+
+typedef struct ic_layer_io {
+    /* F layers only (NULL on S layers, [RN] §11: S layers own no indexer).
+     * prefill: qI bf16 [L,H_I,d_I], kI bf16 [L,d_I], w bf16 [L,H_I].
+     * decode:  qI bf16 [B,H_I,d_I] (the new token's query), w bf16 [B,H_I],
+     *          kI8 e4m3 [B,S_max,d_I], kI_scale fp32 [B,S_max]. */
+    const void *qI;
+    const void *kI;
+    const void *w;
+    const uint8_t *kI8;
+    const float *kI_scale;
+    /* every layer: Q bf16 [rows,Hq,d]; K, V bf16 (prefill [L,d], decode
+     * [B,S_max,d]); out bf16 [rows,Hq,d]. */
+    const void *Q;
+    const void *K;
+    const void *V;
+    void *out;
+    /* optional: device int32 [rows,k] that receives a copy of the index
+     * tensor this layer attended with (for checking the reuse invariant). */
+    int32_t *idx_snapshot;
+} ic_layer_io;
+
+typedef struct ic_stack_dims {
+    int mode;               /* IC_PREFILL or IC_DECODE */
+    int L;                  /* prefill: sequence length (rows = L) */
+    int B;                  /* decode: sequences (rows = B) */
+    int S_max;              /* decode: capacity of each sequence's caches */
+    const int32_t *seq_len; /* decode: device int32 [B], candidates incl. the new token */
+    int H_I, d_I, k, Hq, d;
+    float scale;            /* softmax scale; <= 0 means 1/sqrt(d) */
+} ic_stack_dims;
+
+/* [IC] Figure 2: for l = 0..N-1, if c_l = F run the indexer and top-k into
+ * idx_cache (device int32 [rows, k], overwritten), else reuse idx_cache as
+ * it stands; then sparse attention of layer l with its own Q/K/V at those
+ * indices.  Everything is enqueued on `stream` with no host sync. */
+int ic_run_stack(ic_ctx *ctx, const ic_pattern *pattern, const ic_layer_io *layers,
+                 const ic_stack_dims *dims, int32_t *idx_cache, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* INDEXCACHE_H */

@@ -1,0 +1,151 @@
+"""GPU parity of the decode path (FP8 indexer-key scan, top-k over whole
+sequences, split attention) against the CPU oracle."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from cross_layer_top_b200 import synth
+
+pytestmark = pytest.mark.gpu
+
+SEL_RTOL = 1e-3
+
+
+@pytest.fixture(scope="module")
+def ic():
+    from cross_layer_top_b200 import indexcache
+    return indexcache
+
+
+@pytest.fixture(scope="module")
+def ctx(ic):
+    c = ic.Context(0)
+    yield c
+    c.close()
+
+
+def f32(t):
+    return synth.bf16_to_f32_numpy(t)
+
+
+def _decode_inputs(B, S_max, H_I, seed, lens=None, integer=False):
+    gen = torch.Generator().manual_seed(seed)
+    if integer:
+        q = torch.randint(-3, 4, (B, H_I, 128), generator=gen).bfloat16()
+        w = torch.tensor([-1.0, -0.5, 0.5, 1.0])[torch.randint(0, 4, (B, H_I), generator=gen)].bfloat16()
+        # e4m3 bytes of small integers and halves: 0, +-0.5, +-1, +-1.5, +-2, +-3
+        table = torch.tensor([0x00, 0x30, 0xB0, 0x38, 0xB8, 0x3C, 0xBC, 0x40, 0xC0, 0x44, 0xC4],
+                             dtype=torch.uint8)
+        k8 = table[torch.randint(0, len(table), (B, S_max, 128), generator=gen)]
+        sc = torch.tensor([1.0, 0.5, 2.0, 0.25])[torch.randint(0, 4, (B, S_max), generator=gen)]
+    else:
+        q = torch.randn((B, H_I, 128), generator=gen).bfloat16()
+        w = (torch.randn((B, H_I), generator=gen) / 8).bfloat16()
+        k8, sc = synth.fp8_e4m3_quantize_per_token(torch.randn((B, S_max, 128), generator=gen))
+    if lens is None:
+        lens = [S_max] * B
+    return q, w, k8.contiguous(), sc.float().contiguous(), torch.tensor(lens, dtype=torch.int32)
+
+
+@pytest.mark.parametrize("H_I", [64, 32])
+def test_decode_scores_integer_bit_exact(ic, ctx, H_I):
+    B, S_max = 3, 1000
+    q, w, k8, sc, lens = _decode_inputs(B, S_max, H_I, 1, lens=[1000, 129, 1], integer=True)
+    ld = 1024
+    out = torch.full((B, ld), float("nan"), device="cuda")
+    ic.ic_index_score_decode(ctx, q.cuda(), w.cuda(), k8.cuda(), sc.cuda(), lens.cuda(), out)
+    ctx.sync_status()
+    got = out.cpu().numpy()
+    for b in range(B):
+        n = int(lens[b])
+        ref = oracle.decode_scores(f32(q[b]), f32(w[b]), k8[b].numpy(), sc[b].numpy(), S=n)
+        assert np.array_equal(got[b, :n].astype(np.float64), ref)
+        assert np.all(np.isnan(got[b, n:]))
+
+
+def test_decode_scores_gaussian_close(ic, ctx):
+    B, S_max = 4, 6000
+    q, w, k8, sc, lens = _decode_inputs(B, S_max, 64, 2, lens=[6000, 5999, 4097, 3])
+    out = torch.zeros((B, 6016), device="cuda")
+    ic.ic_index_score_decode(ctx, q.cuda(), w.cuda(), k8.cuda(), sc.cuda(), lens.cuda(), out)
+    ctx.sync_status()
+    got = out.cpu().numpy()
+    for b in range(B):
+        n = int(lens[b])
+        ref = oracle.decode_scores(f32(q[b]), f32(w[b]), k8[b].numpy(), sc[b].numpy(), S=n)
+        assert np.all(np.abs(got[b, :n] - ref) <= 1e-4 * np.abs(ref).max() + 1e-6)
+
+
+def test_decode_index_selected_set(ic, ctx):
+    B, S_max, k = 4, 70001, 2048
+    q, w, k8, sc, lens = _decode_inputs(B, S_max, 64, 3, lens=[70001, 2048, 2049, 33333])
+    idx = torch.empty((B, k), dtype=torch.int32, device="cuda")
+    ic.ic_index_fp_decode(ctx, q.cuda(), w.cuda(), k8.cuda(), sc.cuda(), lens.cuda(), k, idx)
+    ctx.sync_status()
+    got = idx.cpu().numpy()
+    for b in range(B):
+        n = int(lens[b])
+        ref = oracle.decode_scores(f32(q[b]), f32(w[b]), k8[b].numpy(), sc[b].numpy(), S=n)
+        m = min(n, k)
+        sel = got[b, :m]
+        assert np.all(got[b, m:] == -1) and np.all(np.diff(sel) > 0) and sel.max() < n
+        if n > k:
+            kth = oracle.kth_score(ref, k)
+            assert ref[sel].min() >= kth - SEL_RTOL * abs(kth)
+
+
+def test_decode_workload_sampled(ic, ctx):
+    """Decode workload shapes (32 sequences x 65537 candidates, H_I=64,
+    k=2048): one F layer, 6 sequences checked against the oracle."""
+    cfg = synth.CONFIGS["decode"]
+    lay = synth.decode_layer(cfg, 0, "cuda")
+    B, k = cfg.B, cfg.k
+    idx = torch.empty((B, k), dtype=torch.int32, device="cuda")
+    ic.ic_index_fp_decode(ctx, lay["q"], lay["w"], lay["kI8"], lay["kI_scale"], lay["seq_len"], k,
+                          idx)
+    ctx.sync_status()
+    got = idx.cpu().numpy()
+    for b in [0, 1, 15, 30, 31]:
+        ref = oracle.decode_scores(f32(lay["q"][b]), f32(lay["w"][b]), lay["kI8"][b].cpu().numpy(),
+                                   lay["kI_scale"][b].cpu().numpy())
+        kth = oracle.kth_score(ref, k)
+        sel = got[b]
+        assert np.all(np.diff(sel) > 0)
+        assert ref[sel].min() >= kth - SEL_RTOL * abs(kth)
+
+
+def test_decode_stack(ic, ctx):
+    """Decode F/S stack through ic_run_stack: snapshots obey the reuse rule,
+    F-layer selections and every layer's attention match the oracle."""
+    cfg = synth.DecodeConfig("small_decode", 3, 4999, "FSSFS", 64, 128, 256, 16, 128, 9)
+    B, S, k = cfg.B, cfg.S, cfg.k
+    layers, olay = [], []
+    for l in range(cfg.n_layers):
+        lay = synth.decode_layer(cfg, l, "cuda")
+        lay["out"] = torch.empty((B, cfg.Hq, cfg.d), dtype=torch.bfloat16, device="cuda")
+        lay["idx_snapshot"] = torch.empty((B, k), dtype=torch.int32, device="cuda")
+        layers.append(lay)
+    seq_len = layers[0]["seq_len"]
+    pat = ic.ic_create_pattern(cfg.pattern)
+    dims = ic.stack_dims(ic.IC_DECODE, cfg.H_I, cfg.d_I, k, cfg.Hq, cfg.d, B=B, S_max=S,
+                         seq_len=seq_len)
+    cache = torch.empty((B, k), dtype=torch.int32, device="cuda")
+    ic.ic_run_stack(ctx, pat, layers, dims, cache)
+    ctx.sync_status()
+    src = oracle.pattern_src(cfg.pattern)
+    snaps = [lay["idx_snapshot"].cpu().numpy() for lay in layers]
+    for l in range(cfg.n_layers):
+        assert np.array_equal(snaps[l], snaps[src[l]])
+        lay = layers[l]
+        if cfg.pattern[l] == "F":
+            for b in range(B):
+                ref = oracle.decode_scores(f32(lay["q"][b]), f32(lay["w"][b]),
+                                           lay["kI8"][b].cpu().numpy(),
+                                           lay["kI_scale"][b].cpu().numpy())
+                kth = oracle.kth_score(ref, k)
+                assert ref[snaps[l][b]].min() >= kth - SEL_RTOL * abs(kth)
+        ref_out = oracle.sparse_attn(f32(lay["Q"]), f32(lay["K"]), f32(lay["V"]), snaps[l],
+                                     rows_per_seq=1)
+        got = lay["out"].float().cpu().numpy().astype(np.float64)
+        assert np.all(np.abs(got - ref_out) <= 2e-2 + 1e-2 * np.abs(ref_out))
