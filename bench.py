@@ -1,0 +1,502 @@
+"""Benchmark of the IndexCache hot path on B200 GPUs.
+
+One step = one pass of the whole F/S layer stack (indexer + top-k on F
+layers, index reuse on S layers, sparse MQA attention on every layer) over
+one synthetic sequence of the prefill workload: L = 16384, pattern
+FSSSFSSS, H_I = 64, d_I = 128, k = 2048, 16 query heads, d = 128.  Inputs
+are resident in HBM when the timed region starts; the L2 is flushed
+(a 512 MB write) between timed steps, outside the timed events.
+
+Launch: ``python bench.py [--gpus N --steps K --warmup W]``; for N > 1 under
+torchrun, one rank per GPU, each rank running its own independent sequence
+(weak scaling, no data-path collective; NCCL carries only the barrier and
+the max-over-ranks of the step time).
+
+``--impl reference`` times the CPU oracle (the plain C reference) on the
+host cores instead, on a bounded row sample of the same workload.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "indexer scored pairs/s + top-k rows/s; F/S layer-stack prefill & decode ms"
+WORKLOAD = "prefill"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FLOP_PER_PAIR_PER_HEAD_DIM = 2  # multiply-add
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return p, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def scored_pairs(L, k, n_f):
+    """Causal pairs (t, s <= t) the F layers must score: rows t >= k (rows
+    t < k keep all of 0..t without a score)."""
+    per_layer = L * (L + 1) // 2 - k * (k + 1) // 2 if L > k else 0
+    return per_layer * n_f
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling (200 ms) while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index):
+        self.dev = device_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax = float(parts[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------- our arm
+def make_prefill_inputs(cfg, rank, device):
+    """All layer tensors of one sequence; each rank draws its own sequence."""
+    import dataclasses
+    from cross_layer_top_b200 import synth
+    cfg = dataclasses.replace(cfg, seed=cfg.seed + 7919 * rank)
+    layers = []
+    for l in range(cfg.n_layers):
+        lay = synth.prefill_layer(cfg, l, device)
+        lay["out"] = torch.empty((cfg.L, cfg.Hq, cfg.d), dtype=torch.bfloat16, device=device)
+        layers.append(lay)
+    return layers
+
+
+def run_ours(args, rank, world, local_rank):
+    from cross_layer_top_b200 import indexcache as ic
+    from cross_layer_top_b200 import synth
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    peaks, peak_src = load_peaks()
+    cfg = synth.CONFIGS[WORKLOAD]
+    L, k = cfg.L, cfg.k
+    n_f = cfg.pattern.count("F")
+    ctx = ic.Context(local_rank)
+    pat = ic.ic_create_pattern(cfg.pattern)
+    layers = make_prefill_inputs(cfg, rank, dev)
+    dims = ic.stack_dims(ic.IC_PREFILL, cfg.H_I, cfg.d_I, k, cfg.Hq, cfg.d, L=L)
+    cache = torch.empty((L, k), dtype=torch.int32, device=dev)
+    arr = ic.make_stack_layers(layers)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        ic.ic_run_stack(ctx, pat, None, dims, cache, layer_array=arr)
+
+    for _ in range(args.warmup):
+        step()
+    ctx.sync_status()
+    dist_barrier(world)
+    torch.cuda.synchronize()
+
+    # ------------------------------------------------ timed region (device)
+    ctx.reset_timing()
+    ctx.set_timing(True)
+    launches0 = ctx.launch_count()
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    for i in range(args.steps):
+        flush.fill_(float(i))  # L2 flush, outside the timed events
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    clk = clocks.stop()
+    ctx.set_timing(False)
+    ctx.sync_status()
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    total_ms = sum(step_ms)
+    gpu_launches = ctx.launch_count() - launches0
+    ktimes = {}
+    for kid, name in enumerate(ic.KERNEL_NAMES):
+        ms, n = ctx.get_timing(kid)
+        ktimes[name] = {"ms": ms, "launches": n}
+    total_ms = dist_max(total_ms, world)
+
+    pairs_step = scored_pairs(L, k, n_f)
+    value = pairs_step * args.steps * world / (total_ms / 1e3)
+    ms_per_step = total_ms / args.steps
+
+    # ------------------------------------------------ roofline of the dominant kernel
+    idx_k = ktimes["index_score"]
+    att_k = ktimes["sparse_attn"]
+    top_k = ktimes["topk"]
+    roof = {}
+    if idx_k["launches"]:
+        avg_ms = idx_k["ms"] / idx_k["launches"]
+        pairs_launch = pairs_step * args.steps / idx_k["launches"]
+        tflops = 2 * cfg.H_I * cfg.d_I * pairs_launch / (avg_ms / 1e3) / 1e12
+        peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+        roof["index_score"] = {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak,
+                               "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
+                               "traffic": None, "peak_kind": "sustained bf16, " + peak_src,
+                               "avg_launch_ms": round(avg_ms, 4),
+                               "flop_per_launch": 2 * cfg.H_I * cfg.d_I * pairs_launch}
+    if att_k["launches"]:
+        avg_ms = att_k["ms"] / att_k["launches"]
+        # algorithmic bytes per launch: the k gathered K and V rows per query
+        # row plus the Q row read and the output row written
+        bytes_launch = L * (k * 2 * cfg.d * 2 + 2 * cfg.Hq * cfg.d * 2)
+        gbs = bytes_launch / (avg_ms / 1e3) / 1e9
+        roof["sparse_attn"] = {"bound": "hbm", "achieved": round(gbs, 1),
+                               "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                               "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                               "peak_kind": "HBM copy, " + peak_src,
+                               "avg_launch_ms": round(avg_ms, 4), "bytes_per_launch": bytes_launch,
+                               "note": "gathered rows mostly hit L2 (8 MB K/V per layer)"}
+    dominant = max(("index_score", "sparse_attn"), key=lambda n: ktimes[n]["ms"])
+    roofline = dict(roof.get(dominant, {}))
+    roofline["kernel"] = dominant
+
+    topk_rows = (L - k) * n_f * args.steps
+    extra = {
+        "kernels_ms_per_step": {n: round(v["ms"] / args.steps, 4) for n, v in ktimes.items()},
+        "indexer_pairs_per_s": (pairs_step * args.steps / (idx_k["ms"] / 1e3)) if idx_k["ms"] else None,
+        "topk_rows_per_s": (topk_rows / (top_k["ms"] / 1e3)) if top_k["ms"] else None,
+        "stack_prefill_ms": round(ms_per_step, 4),
+        "step_ms": [round(x, 4) for x in step_ms],
+        "roofline_all": roof,
+    }
+
+    # ------------------------------------------------ e2e through the C ABI with host buffers
+    e2e = None
+    if not args.no_e2e:
+        e2e = run_e2e(args, ctx, pat, dims, cfg, layers, cache, world, pairs_step, stream)
+
+    # ------------------------------------------------ decode step (extra evidence)
+    if not args.no_decode:
+        extra["decode"] = run_decode(args, ctx, peaks, peak_src, local_rank)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = cpu_baseline(cfg, budget_s=args.cpu_budget)
+
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "pairs/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms_per_step,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": "prefill stack: 1 sequence/GPU, L=16384, pattern FSSSFSSS, "
+                               "H_I=64, d_I=128, k=2048, 16 query heads, 1 KV head, d=128",
+                   "global_batch": world, "seq_len": L, "parallelism": "dp%d" % world,
+                   "l2": "flushed between timed steps (512 MB write)"},
+        "e2e": e2e,
+        "gpu_launches": gpu_launches,
+        "roofline": roofline,
+        "cpu_baseline": cpu,
+        "clocks": clk,
+        "extra": extra,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    ctx.close()
+
+
+def run_e2e(args, ctx, pat, dims, cfg, layers, cache, world, pairs_step, stream):
+    """Same metric through ic_run_stack with host inputs: every step copies
+    all layer inputs host->device (pinned) and every layer output back."""
+    from cross_layer_top_b200 import indexcache as ic
+    host_in, host_out = [], []
+    h2d = d2h = 0
+    for lay in layers:
+        hi = {}
+        for n, t in lay.items():
+            if n == "out":
+                continue
+            hi[n] = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+            hi[n].copy_(t)
+            h2d += t.numel() * t.element_size()
+        host_in.append(hi)
+        host_out.append(torch.empty(lay["out"].shape, dtype=lay["out"].dtype, pin_memory=True))
+        d2h += lay["out"].numel() * lay["out"].element_size()
+    arr = ic.make_stack_layers(layers)
+
+    def step():
+        for lay, hi in zip(layers, host_in):
+            for n, t in hi.items():
+                lay[n].copy_(t, non_blocking=True)
+        ic.ic_run_stack(ctx, pat, None, dims, cache, layer_array=arr)
+        for lay, ho in zip(layers, host_out):
+            ho.copy_(lay["out"], non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = dist_max(a.elapsed_time(b), world)
+    return {"value": pairs_step * args.steps * world / (ms / 1e3), "unit": "pairs/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "ms_per_step": ms / args.steps}
+
+
+def run_decode(args, ctx, peaks, peak_src, local_rank):
+    """One decode step of the batched-decode workload (32 sequences x 65537
+    candidates, 16 layers FSSS x4): step ms, FP8 indexer-key scan GB/s and
+    the attention gather GB/s against the HBM peak."""
+    from cross_layer_top_b200 import indexcache as ic
+    from cross_layer_top_b200 import synth
+    cfg = synth.CONFIGS["decode"]
+    dev = torch.device("cuda", local_rank)
+    B, S, k = cfg.B, cfg.S, cfg.k
+    layers = []
+    for l in range(cfg.n_layers):
+        lay = synth.decode_layer(cfg, l, dev)
+        lay["out"] = torch.empty((B, cfg.Hq, cfg.d), dtype=torch.bfloat16, device=dev)
+        layers.append(lay)
+    seq_len = layers[0]["seq_len"]
+    pat = ic.ic_create_pattern(cfg.pattern)
+    dims = ic.stack_dims(ic.IC_DECODE, cfg.H_I, cfg.d_I, k, cfg.Hq, cfg.d, B=B, S_max=S,
+                         seq_len=seq_len)
+    cache = torch.empty((B, k), dtype=torch.int32, device=dev)
+    arr = ic.make_stack_layers(layers, ic.IC_DECODE)
+    flush = torch.empty(512 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    for _ in range(args.warmup):
+        ic.ic_run_stack(ctx, pat, None, dims, cache, layer_array=arr)
+    ctx.sync_status()
+    steps = max(args.steps, 5)
+    ctx.reset_timing()
+    ctx.set_timing(True)
+    stream = torch.cuda.current_stream()
+    tot = 0.0
+    for i in range(steps):
+        flush.fill_(float(i))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        ic.ic_run_stack(ctx, pat, None, dims, cache, layer_array=arr)
+        b.record(stream)
+        b.synchronize()
+        tot += a.elapsed_time(b)
+    ctx.set_timing(False)
+    ctx.sync_status()
+    kt = {n: ctx.get_timing(i) for i, n in enumerate(ic.KERNEL_NAMES)}
+    n_f = cfg.pattern.count("F")
+    scan_bytes = B * S * (cfg.d_I + 4) + B * S * 4  # e4m3 keys + scales read, fp32 scores written
+    scan_ms, scan_n = kt["index_score_decode"]
+    att_ms, att_n = kt["sparse_attn"]
+    gather_bytes = B * k * 2 * cfg.d * 2
+    res = {"workload": "decode: 32 sequences x (65536 cached + 1 new) tokens, 16 layers FSSS x4, "
+                       "FP8 e4m3 indexer keys + fp32 per-token scale, k=2048",
+           "step_ms": tot / steps,
+           "kernels_ms_per_step": {n: round(v[0] / steps, 4) for n, v in kt.items()}}
+    if scan_n:
+        gbs = scan_bytes / (scan_ms / scan_n / 1e3) / 1e9
+        res["scan"] = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                       "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                       "bytes_per_launch": scan_bytes, "avg_launch_ms": scan_ms / scan_n,
+                       "peak_kind": "HBM copy, " + peak_src}
+    if att_n:
+        gbs = gather_bytes / (att_ms / att_n / 1e3) / 1e9
+        res["gather"] = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
+                         "bytes_per_launch": gather_bytes, "avg_launch_ms": att_ms / att_n}
+    del layers
+    torch.cuda.empty_cache()
+    return res
+
+
+# ------------------------------------------------------- the oracle on CPU
+def cpu_baseline(cfg, budget_s=15.0, rows_idx=None, rows_att=None):
+    """Time the CPU oracle on a bounded row sample of the prefill stack and
+    scale to the stack's scored pairs/s.  The indexer cost of row t is
+    proportional to t+1, attention cost is per row."""
+    import oracle
+    from cross_layer_top_b200 import synth
+    L, k = cfg.L, cfg.k
+    n_f, n_l = cfg.pattern.count("F"), cfg.n_layers
+    lay = synth.prefill_layer(cfg, 0, "cpu")
+    q = synth.bf16_to_f32_numpy(lay["qI"])
+    kk = synth.bf16_to_f32_numpy(lay["kI"])
+    w = synth.bf16_to_f32_numpy(lay["w"])
+    Q = synth.bf16_to_f32_numpy(lay["Q"])
+    K = synth.bf16_to_f32_numpy(lay["K"])
+    V = synth.bf16_to_f32_numpy(lay["V"])
+    rng = np.random.default_rng(0)
+    threads = os.cpu_count()
+    # indexer: grow the sample until about half the budget is spent
+    n_rows = rows_idx or 8
+    while True:
+        rows = np.sort(rng.integers(k, L, n_rows)).astype(np.int32)
+        t0 = time.perf_counter()
+        idx = oracle.index_topk(q, kk, w, k, rows)
+        dt_idx = time.perf_counter() - t0
+        if rows_idx or dt_idx > budget_s / 4 or n_rows >= 4096:
+            break
+        n_rows *= 4
+    pairs_sampled = int(np.sum(rows.astype(np.int64) + 1))
+    sec_per_pair = dt_idx / pairs_sampled
+    n_att = rows_att or 64
+    while True:
+        arows = rng.integers(0, L, n_att).astype(np.int32)
+        t0 = time.perf_counter()
+        oracle.sparse_attn(Q, K, V, np.tile(idx[:1], (n_att, 1)), rows=arows)
+        dt_att = time.perf_counter() - t0
+        if rows_att or dt_att > budget_s / 4 or n_att >= 65536:
+            break
+        n_att *= 4
+    sec_per_att_row = dt_att / n_att
+    pairs = scored_pairs(L, k, n_f)
+    est_step_s = pairs * sec_per_pair + n_l * L * sec_per_att_row
+    return {"value": pairs / est_step_s, "unit": "pairs/s", "cores": threads, "kind": "oracle",
+            "sample": "%d indexer rows (t in [k, L), %d scored pairs) + %d attention rows of the "
+                      "prefill workload; stack time extrapolated by pairs and rows"
+                      % (n_rows, pairs_sampled, n_att),
+            "est_step_s": est_step_s, "measured_s": dt_idx + dt_att}
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the CPU oracle (plain C, fp64, OpenMP over rows)."""
+    if rank != 0:
+        return
+    from cross_layer_top_b200 import synth
+    cfg = synth.CONFIGS[WORKLOAD]
+    budget = min(16.0, max(4.0, 150.0 / max(1, args.steps + args.warmup)))
+    vals = []
+    cb = None
+    for i in range(args.warmup + args.steps):
+        cb = cpu_baseline(cfg, budget_s=budget)
+        if i >= args.warmup:
+            vals.append(cb["value"])
+    value = statistics.median(vals) if vals else cb["value"]
+    step_ms = scored_pairs(cfg.L, cfg.k, cfg.pattern.count("F")) / value * 1e3
+    line = {"metric": METRIC, "value": value, "unit": "pairs/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_ms,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "impl": "reference",
+            "config": {"workload": "prefill stack: 1 sequence, L=16384, pattern FSSSFSSS, H_I=64, "
+                                   "d_I=128, k=2048, 16 query heads, 1 KV head, d=128",
+                       "global_batch": 1, "seq_len": cfg.L, "parallelism": "host cores"},
+            "cpu_baseline": {"value": value, "unit": "pairs/s", "kind": "oracle",
+                             "cores": cb["cores"], "sample": cb["sample"]},
+            "e2e": {"value": value, "unit": "pairs/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------ distributed
+def dist_barrier(world):
+    if world > 1:
+        torch.distributed.barrier()
+
+
+def dist_max(x, world):
+    if world == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=16.0)
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours":
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
