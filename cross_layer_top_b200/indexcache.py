@@ -78,6 +78,7 @@ _SIGS = {
     "ic_index_reuse": ([_vp, ctypes.POINTER(_vp)], _i),
     "ic_index_score_decode": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _i64, _vp], _i),
     "ic_index_fp_decode": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp], _i),
+    "ic_index_fp_decode_noalloc": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp], _i),
     "ic_sparse_attn": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64, _i, _f, _vp, _vp], _i),
     "ic_run_stack": ([_vp, _vp, ctypes.POINTER(ic_layer_io), ctypes.POINTER(ic_stack_dims), _vp,
                       _vp], _i),
@@ -272,6 +273,15 @@ def ic_index_fp_decode(ctx: Context, q, w, kI8, kI_scale, seq_len, k: int, idx_o
     _check(_lib.ic_index_fp_decode(ctx.handle, _ptr(q), _ptr(w), _ptr(kI8), _ptr(kI_scale),
                                    _ptr(seq_len), B, S_max, H_I, d_I, k, _ptr(idx_out),
                                    _stream(stream)), ctx)
+
+
+def ic_index_fp_decode_noalloc(q, w, kI8, kI_scale, seq_len, k: int, idx_out, stream=None):
+    """Decode F layer without any device allocation (fixed library scratch)."""
+    B, H_I, d_I = q.shape
+    S_max = kI8.shape[1]
+    _check(_lib.ic_index_fp_decode_noalloc(_ptr(q), _ptr(w), _ptr(kI8), _ptr(kI_scale),
+                                           _ptr(seq_len), B, S_max, H_I, d_I, k, _ptr(idx_out),
+                                           _stream(stream)))
 
 
 def ic_sparse_attn(ctx: Context, Q, K, V, idx, out, rows_per_seq: int = 0, kv_seq_stride: int = 0,

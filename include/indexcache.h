@@ -171,6 +171,24 @@ int ic_index_fp_decode(ic_ctx *ctx, const void *q, const void *w, const uint8_t 
                        const float *kI_scale, const int32_t *seq_len, int B, int S_max, int H_I,
                        int d_I, int k, int32_t *idx_out, void *stream);
 
+/* Allocation-free variant of ic_index_fp_decode, for callers that cannot
+ * call cudaMalloc on their decode path: engines that give all free HBM to
+ * their own KV-cache pool (an allocation could fail, and it synchronizes the
+ * device in a latency-bound per-token loop), or a decode step replayed from
+ * a captured stream.  The pages have no counterpart to this entry point.
+ * Same arguments, results and support as ic_index_fp_decode, without a
+ * context.  The fp32 score rows live in a fixed 16 MiB array in the
+ * library's device memory (every GPU that loads the library holds it until
+ * exit): B * round_up(S_max, 64) must be <= 4194304, else IC_ERR_UNSUPPORTED
+ * with a message.  The first call on a device resolves that array's address
+ * (cudaGetSymbolAddress) and should come before any stream capture.  All
+ * calls share the array: calls whose kernels overlap on the GPU race.
+ * Device-side wait timeouts are not reported (the call never
+ * synchronizes).  Error messages: ic_last_error(NULL). */
+int ic_index_fp_decode_noalloc(const void *q, const void *w, const uint8_t *kI8,
+                               const float *kI_scale, const int32_t *seq_len, int B, int S_max,
+                               int H_I, int d_I, int k, int32_t *idx_out, void *stream);
+
 /* ------------------------------------------------------ sparse attention */
 
 /* [RN] §3 sparse MQA attention, every layer:
