@@ -313,10 +313,14 @@ def run_e2e(args, ctx, pat, dims, cfg, layers, cache, world, pairs_step, stream)
 def run_decode(args, ctx, peaks, peak_src, local_rank):
     """One decode step of the batched-decode workload (32 sequences x 65537
     candidates, 16 layers FSSS x4): step ms, FP8 indexer-key scan GB/s and
-    the attention gather GB/s against the HBM peak."""
+    the attention gather GB/s against the HBM peak.  --decode-layers N keeps
+    the first N layers (for profiling captures that must stay small)."""
+    import dataclasses
     from cross_layer_top_b200 import indexcache as ic
     from cross_layer_top_b200 import synth
     cfg = synth.CONFIGS["decode"]
+    if args.decode_layers:
+        cfg = dataclasses.replace(cfg, pattern=cfg.pattern[:args.decode_layers])
     dev = torch.device("cuda", local_rank)
     B, S, k = cfg.B, cfg.S, cfg.k
     layers = []
@@ -477,6 +481,9 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=16.0)
+    ap.add_argument("--decode-only", action="store_true",
+                    help="time only the decode workload (not the contract line)")
+    ap.add_argument("--decode-layers", type=int, default=0)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -485,6 +492,16 @@ def main():
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.decode_only:
+        torch.cuda.set_device(local_rank)
+        from cross_layer_top_b200 import indexcache as ic
+        ctx = ic.Context(local_rank)
+        peaks, peak_src = load_peaks()
+        res = run_decode(args, ctx, peaks, peak_src, local_rank)
+        if rank == 0:
+            print(json.dumps({"decode_only": True, "decode": res}), flush=True)
+        ctx.close()
         return
     if world > 1:
         import datetime

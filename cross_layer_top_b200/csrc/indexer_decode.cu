@@ -51,21 +51,30 @@ struct DecodeShape {
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
+// Two e4m3 bytes (low bytes of the two 16-bit lanes of y) -> bf16x2, exactly.
+// The e4m3 sign goes to bit 15 and its 7 exponent/mantissa bits to bits
+// 10..4, i.e. a bf16 whose exponent field is the e4m3 exponent field
+// unbiased: value * 2^-120 (for an e4m3 subnormal, the matching bf16
+// subnormal).  One bf16x2 multiply by 2^120 restores the value; it is exact
+// (a power-of-two scaling into the normal range).  The e4m3 NaN bytes
+// (0x7F, 0xFF) are not NaN afterwards (+-480); caches hold none.
+__device__ __forceinline__ uint32_t e4m3x2_lanes_to_bf16x2(uint32_t y) {
+    const uint32_t bits = ((y << 4) & 0x07F007F0u) | ((y << 8) & 0x80008000u);
+    const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&bits);
+    const __nv_bfloat162 s = __halves2bfloat162(__ushort_as_bfloat16(0x7B80),
+                                                __ushort_as_bfloat16(0x7B80));  // 2^120
+    const __nv_bfloat162 r = __hmul2(v, s);
+    return *reinterpret_cast<const uint32_t*>(&r);
+}
+
 // 16 e4m3 values (one 16-byte chunk) -> 16 bf16 values, exactly.
 __device__ __forceinline__ void e4m3x16_to_bf16(const uint4 in, uint4& lo, uint4& hi) {
     const uint32_t w[4] = {in.x, in.y, in.z, in.w};
     uint32_t o[8];
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-            const unsigned short pair = static_cast<unsigned short>(w[i] >> (16 * h));
-            uint32_t f16x2;
-            asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(f16x2) : "h"(pair));
-            const __half2 hv = *reinterpret_cast<const __half2*>(&f16x2);
-            const float2 f = __half22float2(hv);
-            o[2 * i + h] = pack_bf16x2(f.x, f.y);
-        }
+        o[2 * i] = e4m3x2_lanes_to_bf16x2(__byte_perm(w[i], 0u, 0x4140));      // bytes 0, 1
+        o[2 * i + 1] = e4m3x2_lanes_to_bf16x2(__byte_perm(w[i], 0u, 0x4342));  // bytes 2, 3
     }
     lo = make_uint4(o[0], o[1], o[2], o[3]);
     hi = make_uint4(o[4], o[5], o[6], o[7]);
@@ -265,11 +274,29 @@ __global__ void __launch_bounds__(384, 1)
         int acc = 0;
         uint32_t acc_it[S::NACC] = {0, 0, 0, 0};
         int cur_b = -1;
-        bool ok = true;
-        for (long long g = g_begin; g < g_end && ok; ++g) {
+        // the next tile (after g) that holds candidates, or g_end
+        auto next_valid = [&](long long g) -> long long {
+            for (++g; g < g_end; ++g) {
+                const int b = static_cast<int>(g / tps), j = static_cast<int>(g % tps);
+                if (j * S::BM < seq_len[b]) return g;
+            }
+            return g_end;
+        };
+        // this thread's per-token scale in tile g (0 past the sequence end)
+        auto load_scale = [&](long long g) -> float {
+            if (g >= g_end) return 0.f;
+            const int b = static_cast<int>(g / tps), j = static_cast<int>(g % tps);
+            const int s = j * S::BM + lq * 32 + lane;
+            return s < seq_len[b] ? __ldg(kscale + static_cast<long long>(b) * S_max + s) : 0.f;
+        };
+        // scales are loaded two tiles ahead so their latency hides behind the MMAs
+        long long g = next_valid(g_begin - 1);
+        long long g1 = next_valid(g), g2 = next_valid(g1);
+        float sc0 = load_scale(g), sc1 = load_scale(g1);
+        while (g < g_end) {
+            const float sc2 = load_scale(g2);
             const int b = static_cast<int>(g / tps), j = static_cast<int>(g % tps);
             const int n = seq_len[b];
-            if (j * S::BM >= n) continue;
             if (b != cur_b) {
                 __syncwarp();
                 for (int h = lane; h < H_I; h += 32)
@@ -278,14 +305,10 @@ __global__ void __launch_bounds__(384, 1)
                 cur_b = b;
             }
             const int s = j * S::BM + lq * 32 + lane;
-            const float sc = s < n ? __ldg(kscale + static_cast<long long>(b) * S_max + s) : 0.f;
             bool got = mbar_wait(&acc_full[acc], acc_it[acc] & 1, abort_flag, err,
                                  kDevTimeoutEpilogue);
             got = __all_sync(0xffffffffu, got);
-            if (!got) {
-                ok = false;
-                break;
-            }
+            if (!got) break;
             tc_fence_after();
             const uint32_t taddr =
                 tmem + (static_cast<uint32_t>(lq * 32) << 16) + static_cast<uint32_t>(acc * H_I);
@@ -306,9 +329,14 @@ __global__ void __launch_bounds__(384, 1)
                 p[2] = fmaf(wv.z, fmaxf(__uint_as_float(src[(h + 2) & 31]), 0.f), p[2]);
                 p[3] = fmaf(wv.w, fmaxf(__uint_as_float(src[(h + 3) & 31]), 0.f), p[3]);
             }
-            if (s < n) scores[static_cast<long long>(b) * ld + s] = sc * ((p[0] + p[1]) + (p[2] + p[3]));
+            if (s < n) scores[static_cast<long long>(b) * ld + s] = sc0 * ((p[0] + p[1]) + (p[2] + p[3]));
             ++acc_it[acc];
             if (++acc == S::NACC) acc = 0;
+            sc0 = sc1;
+            sc1 = sc2;
+            g = g1;
+            g1 = g2;
+            g2 = next_valid(g2);
         }
     }
 

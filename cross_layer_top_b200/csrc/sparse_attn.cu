@@ -5,18 +5,20 @@
 // Accelerating Sparse Attention via Cross-Layer Index Reuse", Figure 2 step
 // SPARSEATTN).  One K/V head is shared by all Hq <= 16 query heads.
 //
-// Design: one CTA (4 warps) per (query row, key split).  The 16 query heads
-// form the M = 16 rows of mma.m16n8k16 tiles, so one gathered K/V row serves
-// every head.  Each warp owns chunks of 16 index slots and runs its own
-// 3-stage cp.async ring: the 16 selected K rows and V rows (d*2 bytes each,
-// 16-byte pieces, XOR-swizzled in shared memory so ldmatrix is
-// conflict-free) are gathered while the previous chunk computes
-// S = Q K^T, an online softmax (fp32, base-2 exponent with the scale folded
-// in) and O += P V.  The four warps' (m, l, O) are merged through shared
-// memory; with one split the CTA writes bf16 output, otherwise fp32
-// partials that k_attn_combine merges (decode: few rows, many splits).
-// Invalid slots (-1, or outside [0, kv_len): latched as an error) are
-// masked and gather nothing.
+// Design: one CTA (4 warps, two CTAs per SM) per (query row, key split).
+// The 16 query heads form the M = 16 rows of mma.m16n8k16 tiles, so one
+// gathered K/V row serves every head.  Each warp owns chunks of 16 index
+// slots and a 3-deep ring: lane l always copies the same 16-byte piece
+// (l mod d/8) of its rows with cp.async (zero-filled for masked slots),
+// XOR-swizzled by row so ldmatrix is conflict-free, while the warp computes
+// an earlier chunk: S = Q K^T, an online softmax in the
+// base-2 domain with the scale folded in and a lazy rescale (the running
+// reference only moves when a logit exceeds it by 2^8, so O is rarely
+// rescaled), and O += P V.  Slots holding -1 (or an out-of-range index,
+// which is also latched as an error) are masked and gather zeros; the
+// chunks after the last valid slot are skipped.  The four warps' (m, l, O)
+// merge through shared memory; one split writes bf16 output, several
+// splits write fp32 partials merged by k_attn_combine (decode).
 #include "ic_device.cuh"
 #include "ic_internal.h"
 
@@ -29,22 +31,24 @@ struct AttnShape {
     static constexpr int CH = 16;  // index slots per warp chunk
     static constexpr int STAGES = 3;
     static constexpr int ROWB = D * 2;
-    static constexpr int PIECES = D / 8;  // 16-byte pieces per row
-    static constexpr int CHUNK_BYTES = CH * ROWB;
-    static constexpr int STAGE_BYTES = 2 * CHUNK_BYTES;  // K and V
+    static constexpr int ROWP = ROWB;  // row pitch; 16-byte pieces XOR-swizzled by row
+    static constexpr int STAGE_BYTES = 2 * CH * ROWP;  // K rows then V rows
     static constexpr int WARP_BYTES = STAGES * STAGE_BYTES;
-    static constexpr int Q_BYTES = 16 * ROWB;
+    static constexpr int Q_BYTES = 16 * ROWP;
     static constexpr int MAXK = 2048;
     static constexpr int OFF_Q = 0;
     static constexpr int OFF_IDX = Q_BYTES;
-    static constexpr int OFF_ST = OFF_IDX + MAXK * 4;
+    static constexpr int OFF_LAST = OFF_IDX + MAXK * 4;
+    static constexpr int OFF_ST = OFF_LAST + 128;
     static constexpr int SMEM = OFF_ST + WARPS * WARP_BYTES;
-    // merge buffers (alias the stages once every warp is done)
     static constexpr int MERGE_BYTES = WARPS * (16 * D + 32) * 4;
+    static constexpr float kRescaleThreshold = 8.0f;  // log2 units
     static_assert(MERGE_BYTES <= WARPS * WARP_BYTES, "merge buffer must fit in the stages");
 };
 
-// byte offset of 16-byte piece `c` of row `row` in a swizzled [rows][D] tile
+// byte offset of 16-byte piece c of row `row` in a [rows][d] bf16 tile whose
+// pieces are XOR-swizzled by (row mod 8): ldmatrix reads 8 rows of one piece
+// column from 8 different bank groups
 template <int D>
 __device__ __forceinline__ uint32_t swz(int row, int c) {
     return static_cast<uint32_t>(row * (D * 2) + ((c ^ (row & 7)) << 4));
@@ -64,14 +68,18 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
     const int slot0 = split * kps;
     const int nk = max(0, min(k, slot0 + kps) - slot0);
     int32_t* sIdx = reinterpret_cast<int32_t*>(smem + S::OFF_IDX);
+    int* s_last = reinterpret_cast<int*>(smem + S::OFF_LAST);
     const uint32_t sQ = smem_u32(smem + S::OFF_Q);
     const long long seq = rows_per_seq > 0 ? r / rows_per_seq : 0;
     const __nv_bfloat16* Kb = K + seq * kv_seq_stride;
     const __nv_bfloat16* Vb = V + seq * kv_seq_stride;
 
-    // index slots of this split (validated) and the query heads
+    if (tid == 0) *s_last = -1;
+    __syncthreads();
+    // index slots of this split (validated), the last valid slot, the query heads
     const int32_t* irow = idx + static_cast<long long>(r) * k + slot0;
     bool bad = false;
+    int last = -1;
     for (int i = tid; i < nk; i += S::THREADS) {
         int v = irow[i];
         if (v < -1 || v >= kv_len) {
@@ -79,18 +87,20 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
             v = -1;
         }
         sIdx[i] = v;
+        if (v >= 0) last = i;
     }
     if (bad) atomicCAS(err, 0, kDevBadIndex);
+    if (last >= 0) atomicMax(s_last, last);
     const __nv_bfloat16* qrow = Q + static_cast<long long>(r) * Hq * D;
-    for (int p = tid; p < 16 * S::PIECES; p += S::THREADS) {
-        const int h = p / S::PIECES, c = p % S::PIECES;
+    for (int p = tid; p < 16 * (D / 8); p += S::THREADS) {
+        const int h = p / (D / 8), c = p % (D / 8);
         uint4 v = make_uint4(0, 0, 0, 0);
         if (h < Hq) v = *reinterpret_cast<const uint4*>(qrow + h * D + c * 8);
         *reinterpret_cast<uint4*>(smem + S::OFF_Q + swz<D>(h, c)) = v;
     }
     __syncthreads();
+    const int nk_eff = *s_last + 1;  // slots after the last valid one hold nothing
 
-    // Q fragments (A operand, 16 heads x D)
     uint32_t qa[D / 16][4];
 #pragma unroll
     for (int kk = 0; kk < D / 16; ++kk) {
@@ -101,24 +111,34 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
     }
 
     const uint32_t wst = smem_u32(smem + S::OFF_ST + warp * S::WARP_BYTES);
-    const int nch = (nk + S::CH - 1) / S::CH;
-    // chunks of this warp: warp, warp + WARPS, ...
+    const int nch = (nk_eff + S::CH - 1) / S::CH;
     const int my_n = nch > warp ? (nch - warp + S::WARPS - 1) / S::WARPS : 0;
+    uint32_t vmask[S::STAGES];
 
+    // lane l copies piece (l % PPR) of rows l / PPR, + RPI, ... of K and V
+    constexpr int PPR = D / 8;        // 16-byte pieces per row
+    constexpr int RPI = 32 / PPR;     // rows per warp instruction
+    const int piece = lane % PPR, prow = lane / PPR;
     auto issue = [&](int j) {
         if (j < my_n) {
+            const int st = j % S::STAGES;
             const int c0 = (warp + j * S::WARPS) * S::CH;
-            const uint32_t kb = wst + (j % S::STAGES) * S::STAGE_BYTES;
-            const uint32_t vb = kb + S::CHUNK_BYTES;
+            {
+                const int slot = c0 + (lane & 15);
+                const bool v = slot < nk && sIdx[slot] >= 0;
+                vmask[st] = __ballot_sync(0xffffffffu, v && lane < 16) & 0xffffu;
+            }
+            const uint32_t kdst = wst + st * S::STAGE_BYTES;
+            const uint32_t vdst = kdst + S::CH * S::ROWP;
 #pragma unroll
-            for (int p = lane; p < S::CH * S::PIECES; p += 32) {
-                const int key = p / S::PIECES, c = p % S::PIECES;
-                const int slot = c0 + key;
-                const int s = slot < nk ? sIdx[slot] : -1;
-                const bool ok = s >= 0;
-                const long long off = static_cast<long long>(ok ? s : 0) * D + c * 8;
-                cp_async16(kb + swz<D>(key, c), Kb + off, ok);
-                cp_async16(vb + swz<D>(key, c), Vb + off, ok);
+            for (int i = 0; i < S::CH / RPI; ++i) {
+                const int row = prow + i * RPI;
+                const int slot = c0 + row;
+                const int sidx = slot < nk ? sIdx[slot] : -1;
+                const bool ok = sidx >= 0;
+                const long long off = static_cast<long long>(ok ? sidx : 0) * D + piece * 8;
+                cp_async16(kdst + swz<D>(row, piece), Kb + off, ok);
+                cp_async16(vdst + swz<D>(row, piece), Vb + off, ok);
             }
         }
         cp_async_commit();
@@ -131,13 +151,14 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
 
 #pragma unroll
     for (int j = 0; j < S::STAGES - 1; ++j) issue(j);
-
     for (int j = 0; j < my_n; ++j) {
-        cp_async_wait<S::STAGES - 2>();
+        const int st = j % S::STAGES;
+        cp_async_wait<S::STAGES - 2>();  // chunk j has landed
         __syncwarp();
-        const uint32_t kb = wst + (j % S::STAGES) * S::STAGE_BYTES;
-        const uint32_t vb = kb + S::CHUNK_BYTES;
-        const int c0 = (warp + j * S::WARPS) * S::CH;
+        issue(j + S::STAGES - 1);  // into the stage of chunk j-1, whose reads are done
+        const uint32_t kb = wst + st * S::STAGE_BYTES;
+        const uint32_t vb = kb + S::CH * S::ROWP;
+        const uint32_t cmask = vmask[st];
 
         float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
@@ -150,16 +171,13 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
             mma_bf16_16816(s[0], qa[kk], b0, b1);
             mma_bf16_16816(s[1], qa[kk], b2, b3);
         }
-        // mask invalid slots, scale into the base-2 domain
         float x[2][4];
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
                 const int col = nt * 8 + 2 * (lane & 3) + (e & 1);
-                const int slot = c0 + col;
-                const bool ok = slot < nk && sIdx[slot] >= 0;
-                x[nt][e] = ok ? s[nt][e] * scale_log2 : -INFINITY;
+                x[nt][e] = ((cmask >> col) & 1u) ? s[nt][e] * scale_log2 : -INFINITY;
             }
         float mx0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
         float mx1 = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
@@ -167,13 +185,29 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        const float n0 = fmaxf(m0, mx0), n1 = fmaxf(m1, mx1);
-        // reference points that stay finite while a row has seen nothing
-        const float r0 = n0 == -INFINITY ? 0.f : n0;
-        const float r1 = n1 == -INFINITY ? 0.f : n1;
-        const float a0 = exp2f(m0 - r0), a1 = exp2f(m1 - r1);
-        m0 = n0;
-        m1 = n1;
+        // lazy rescale: move the reference only when a logit passes it by 2^8
+        if (mx0 > m0 + S::kRescaleThreshold) {
+            const float a = exp2f(m0 - mx0);  // 0 while nothing was seen
+            l0 *= a;
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) {
+                o[i][0] *= a;
+                o[i][1] *= a;
+            }
+            m0 = mx0;
+        }
+        if (mx1 > m1 + S::kRescaleThreshold) {
+            const float a = exp2f(m1 - mx1);
+            l1 *= a;
+#pragma unroll
+            for (int i = 0; i < D / 8; ++i) {
+                o[i][2] *= a;
+                o[i][3] *= a;
+            }
+            m1 = mx1;
+        }
+        const float r0 = m0 == -INFINITY ? 0.f : m0;
+        const float r1 = m1 == -INFINITY ? 0.f : m1;
         float p[2][4];
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
@@ -182,15 +216,8 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
             p[nt][2] = exp2f(x[nt][2] - r1);
             p[nt][3] = exp2f(x[nt][3] - r1);
         }
-        l0 = l0 * a0 + (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
-        l1 = l1 * a1 + (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
-#pragma unroll
-        for (int i = 0; i < D / 8; ++i) {
-            o[i][0] *= a0;
-            o[i][1] *= a0;
-            o[i][2] *= a1;
-            o[i][3] *= a1;
-        }
+        l0 += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+        l1 += (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
         uint32_t pa[4];
         pa[0] = pack_bf16x2(p[0][0], p[0][1]);
         pa[1] = pack_bf16x2(p[0][2], p[0][3]);
@@ -206,8 +233,6 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
             mma_bf16_16816(o[2 * dn], pa, b0, b1);
             mma_bf16_16816(o[2 * dn + 1], pa, b2, b3);
         }
-        __syncwarp();
-        issue(j + S::STAGES - 1);
     }
     cp_async_wait<0>();
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
@@ -263,28 +288,36 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
     }
 }
 
-// Merge the per-split partials of each row: out = sum_s O_s 2^(m_s - M) / sum_s l_s 2^(m_s - M).
+// Merge the per-split partials of each row:
+//   out = sum_s O_s 2^(m_s - M) / sum_s l_s 2^(m_s - M),  M = max_s m_s.
+// The per-(split, head) factors are computed once into shared memory.
 template <int D>
 __global__ void __launch_bounds__(256)
     k_attn_combine(const float* __restrict__ part, int Hq, int nsplit,
                    __nv_bfloat16* __restrict__ out) {
+    __shared__ float sf[64][16];
+    __shared__ float sinv[16];
     const int r = blockIdx.x;
     const float* pr = part + static_cast<long long>(r) * nsplit * (16 * D + 32);
-    for (int e = threadIdx.x; e < Hq * D; e += blockDim.x) {
-        const int h = e / D, dd = e % D;
+    if (threadIdx.x < 16) {
+        const int h = threadIdx.x;
         float M = -INFINITY;
         for (int s = 0; s < nsplit; ++s) M = fmaxf(M, pr[s * (16 * D + 32) + 16 * D + h]);
-        float acc = 0.f, lsum = 0.f;
-        if (M != -INFINITY) {
-            for (int s = 0; s < nsplit; ++s) {
-                const float* ps = pr + s * (16 * D + 32);
-                const float f = exp2f(ps[16 * D + h] - M);
-                acc += ps[h * D + dd] * f;
-                lsum += ps[16 * D + 16 + h] * f;
-            }
+        float L = 0.f;
+        for (int s = 0; s < nsplit; ++s) {
+            const float* ps = pr + s * (16 * D + 32);
+            const float f = M == -INFINITY ? 0.f : exp2f(ps[16 * D + h] - M);
+            sf[s][h] = f;
+            L += ps[16 * D + 16 + h] * f;
         }
-        out[(static_cast<long long>(r) * Hq + h) * D + dd] =
-            __float2bfloat16_rn(lsum > 0.f ? acc / lsum : 0.f);
+        sinv[h] = L > 0.f ? 1.f / L : 0.f;
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < Hq * D; e += blockDim.x) {
+        const int h = e / D, dd = e % D;
+        float acc = 0.f;
+        for (int s = 0; s < nsplit; ++s) acc += pr[s * (16 * D + 32) + h * D + dd] * sf[s][h];
+        out[(static_cast<long long>(r) * Hq + h) * D + dd] = __float2bfloat16_rn(acc * sinv[h]);
     }
 }
 
@@ -302,17 +335,19 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
         attr_set = true;
     }
     // Split the index slots across CTAs when there are too few rows to fill
-    // the GPU (decode): aim for ~4 CTAs per SM, at least 64 slots per split.
+    // the GPU (decode): aim for ~4 CTAs per SM, whole warp rounds per split.
+    constexpr int unit = S::CH * S::WARPS;
     int nsplit = 1;
     const int target = 4 * ctx->num_sms;
     if (rows < target) {
         nsplit = (target + rows - 1) / rows;
-        const int max_split = (k + 63) / 64;
+        const int max_split = (k + unit - 1) / unit;
         if (nsplit > max_split) nsplit = max_split;
+        if (nsplit > 64) nsplit = 64;
         if (nsplit < 1) nsplit = 1;
     }
     int kps = (k + nsplit - 1) / nsplit;
-    kps = (kps + S::CH - 1) / S::CH * S::CH;
+    kps = (kps + unit - 1) / unit * unit;
     nsplit = (k + kps - 1) / kps;
     float* part = nullptr;
     if (nsplit > 1) {

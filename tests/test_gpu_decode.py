@@ -149,3 +149,32 @@ def test_decode_stack(ic, ctx):
                                      rows_per_seq=1)
         got = lay["out"].float().cpu().numpy().astype(np.float64)
         assert np.all(np.abs(got - ref_out) <= 2e-2 + 1e-2 * np.abs(ref_out))
+
+
+def test_decode_every_e4m3_byte_exact(ic, ctx):
+    """Each key row holds one nonzero e4m3 byte b at position j < 32; heads
+    0..31 read +k[j] (q = e_j, w = 1) and heads 32..63 read -k[j] (q = -e_j,
+    w = 0.5), so the score is k[j] for k[j] > 0 and 0.5*|k[j]| otherwise —
+    exact in fp32.  Rows cover all 254 finite byte values (subnormals and
+    both signs) at every position: the widening to bf16 must be exact."""
+    B, S = 1, 254 * 32
+    vals = [b for b in range(256) if b not in (0x7F, 0xFF)]
+    k8 = torch.zeros((B, S, 128), dtype=torch.uint8)
+    s = 0
+    for j in range(32):
+        for b in vals:
+            k8[0, s, j] = b
+            s += 1
+    q = torch.zeros((B, 64, 128))
+    for h in range(32):
+        q[0, h, h] = 1.0
+        q[0, 32 + h, h] = -1.0
+    w = torch.tensor([[1.0] * 32 + [0.5] * 32])
+    sc = torch.full((B, S), 2.0)
+    lens = torch.tensor([S], dtype=torch.int32)
+    q, w = q.bfloat16(), w.bfloat16()
+    out = torch.zeros((B, S), device="cuda")
+    ic.ic_index_score_decode(ctx, q.cuda(), w.cuda(), k8.cuda(), sc.cuda(), lens.cuda(), out)
+    ctx.sync_status()
+    ref = oracle.decode_scores(f32(q[0]), f32(w[0]), k8[0].numpy(), sc[0].numpy())
+    assert np.array_equal(out.cpu().numpy()[0].astype(np.float64), ref)
