@@ -437,6 +437,8 @@ extern "C" int ic_sparse_attn(ic_ctx* ctx, const void* Q, const void* K, const v
         return fail(ctx, IC_ERR_SHAPE, "sparse_attn: rows=%d Hq=%d k=%d kv_len=%d", rows, Hq, k,
                     kv_len);
     if (d != 64 && d != 128) return fail(ctx, IC_ERR_UNSUPPORTED, "sparse_attn: d=%d", d);
+    if (kv_len > (1 << 24))
+        return fail(ctx, IC_ERR_UNSUPPORTED, "sparse_attn: kv_len=%d above 2^24", kv_len);
     if (rows == 0) return IC_OK;
     if (!Q || !K || !V || !idx || !out) return fail(ctx, IC_ERR_INVALID_ARG, "sparse_attn: NULL");
     if (!aligned16(Q) || !aligned16(K) || !aligned16(V))

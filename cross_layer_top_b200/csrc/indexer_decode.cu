@@ -9,15 +9,16 @@
 // Accelerating Sparse Attention via Cross-Layer Index Reuse", §2.1).
 //
 // Design (sm_100a), one persistent CTA per SM, HBM-bound by construction:
-//  * warp 0 (TMA): streams raw e4m3 key tiles (128 keys x 128 B) through a
-//    5-deep ring, and the sequence's q rows (bf16, 128-byte swizzle) when
-//    the sequence changes;
-//  * warps 4..7 (convert): widen each e4m3 tile to bf16 — exact, every e4m3
+//  * warp 0 (TMA): streams raw e4m3 key tiles (128 keys x 128 B, one
+//    contiguous 16 KB block each, so one bulk copy) through a 5-deep ring,
+//    and the sequence's q rows (bf16, 128-byte swizzle, a tensor copy)
+//    when the sequence changes;
+//  * warps 4..11 (convert): widen each e4m3 tile to bf16 — exact, every e4m3
 //    value is a bf16 value — and write it in the K-major 128-byte-swizzle
 //    layout the tensor core reads, then fence the async proxy;
 //  * warp 1 (MMA): UMMA M=128 keys x N=H_I heads x K=128, fp32 in TMEM, four
 //    accumulators in flight;
-//  * warps 8..11 (epilogue): the thread owning TMEM lane s applies ReLU,
+//  * warps 12..15 (epilogue): the thread owning TMEM lane s applies ReLU,
 //    the w weights, the head sum and the per-token scale, and stores I[b,s].
 // Each CTA scans a contiguous range of (sequence, key tile) pairs, so q is
 // reloaded only when its range crosses into the next sequence.  All waits
@@ -41,12 +42,15 @@ struct DecodeShape {
     static constexpr int NACC = 4;
     static constexpr int TMEM_COLS = NACC * H_I < 32 ? 32 : NACC * H_I;
     static constexpr int W_BYTES = 4 * H_I * 4;  // per epilogue warp
+    static constexpr int SC_RING = 4;             // scale prefetch depth (tiles)
+    static constexpr int SC_BYTES = SC_RING * BM * 4;
     static constexpr int BAR_BYTES = 256;
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + A_ST * A_STAGE;
     static constexpr int OFF_RAW = OFF_B + B_BYTES;
     static constexpr int OFF_W = OFF_RAW + RAW_ST * RAW;
-    static constexpr int OFF_BAR = OFF_W + W_BYTES;
+    static constexpr int OFF_SC = OFF_W + W_BYTES;
+    static constexpr int OFF_BAR = OFF_SC + SC_BYTES;
     static constexpr int SMEM = OFF_BAR + BAR_BYTES;
     static_assert(SMEM <= 232448, "shared memory budget");
 };
@@ -59,7 +63,8 @@ struct DecodeShape {
 // (a power-of-two scaling into the normal range).  The e4m3 NaN bytes
 // (0x7F, 0xFF) are not NaN afterwards (+-480); caches hold none.
 __device__ __forceinline__ uint32_t e4m3x2_lanes_to_bf16x2(uint32_t y) {
-    const uint32_t bits = ((y << 4) & 0x07F007F0u) | ((y << 8) & 0x80008000u);
+    // (low 7 bits << 4) | (sign << 8) == (y << 4) + sign * (256 - 16)
+    const uint32_t bits = (y & 0x00800080u) * 240u + (y << 4);
     const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&bits);
     const __nv_bfloat162 s = __halves2bfloat162(__ushort_as_bfloat16(0x7B80),
                                                 __ushort_as_bfloat16(0x7B80));  // 2^120
@@ -80,10 +85,49 @@ __device__ __forceinline__ void e4m3x16_to_bf16(const uint4 in, uint4& lo, uint4
     hi = make_uint4(o[4], o[5], o[6], o[7]);
 }
 
+// Walks a CTA's contiguous range of (sequence b, key tile j) pairs in order,
+// visiting only tiles that hold candidates (j * BM < seq_len[b]) and
+// skipping a sequence's empty tail in one step.  One division at the start,
+// none afterwards.
+template <int BM>
+struct TileWalk {
+    long long g, g_end;
+    int b, j, n, tps;
+    const int32_t* seq_len;
+    __device__ __forceinline__ void init(long long g0, long long ge, int tps_, const int32_t* sl) {
+        g = g0;
+        g_end = ge;
+        tps = tps_;
+        seq_len = sl;
+        b = static_cast<int>(g0 / tps_);
+        j = static_cast<int>(g0 - static_cast<long long>(b) * tps_);
+        n = g < g_end ? seq_len[b] : 0;
+        settle();
+    }
+    __device__ __forceinline__ void settle() {
+        while (g < g_end && j * BM >= n) {
+            g += tps - j;
+            ++b;
+            j = 0;
+            if (g < g_end) n = seq_len[b];
+        }
+    }
+    __device__ __forceinline__ bool done() const { return g >= g_end; }
+    __device__ __forceinline__ void next() {
+        ++g;
+        if (++j == tps) {
+            j = 0;
+            ++b;
+            if (g < g_end) n = seq_len[b];
+        }
+        settle();
+    }
+};
+
 template <int H_I>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     k_index_score_decode(const __grid_constant__ CUtensorMap tm_q,
-                         const __grid_constant__ CUtensorMap tm_k8,
+                         const uint8_t* __restrict__ k8,
                          const __nv_bfloat16* __restrict__ w, const float* __restrict__ kscale,
                          const int32_t* __restrict__ seq_len, int B, int S_max, int tps,
                          float* __restrict__ scores, long long ld, int* __restrict__ err) {
@@ -119,10 +163,10 @@ __global__ void __launch_bounds__(384, 1)
         }
         for (int i = 0; i < S::RAW_ST; ++i) {
             mbar_init(&raw_full[i], 1);
-            mbar_init(&raw_empty[i], 128);
+            mbar_init(&raw_empty[i], 8);  // one arrival per converter warp
         }
         for (int i = 0; i < S::A_ST; ++i) {
-            mbar_init(&a_full[i], 128);
+            mbar_init(&a_full[i], 8);
             mbar_init(&a_empty[i], 1);
         }
         for (int i = 0; i < S::NACC; ++i) {
@@ -134,7 +178,6 @@ __global__ void __launch_bounds__(384, 1)
         mbar_init(done_bar, 1);
         fence_mbar_init();
         tma_prefetch_desc(&tm_q);
-        tma_prefetch_desc(&tm_k8);
     }
     if (warp == 2) {
         tmem_alloc(tmem_slot, S::TMEM_COLS);
@@ -154,9 +197,9 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int i = 0; i < S::RAW_ST; ++i) last_ph[i] = -1;
         int q_last = -1, cur_b = -1;
-        for (long long g = g_begin; g < g_end; ++g) {
-            const int b = static_cast<int>(g / tps), j = static_cast<int>(g % tps);
-            if (j * S::BM >= seq_len[b]) continue;
+        TileWalk<S::BM> tw;
+        for (tw.init(g_begin, g_end, tps, seq_len); !tw.done(); tw.next()) {
+            const int b = tw.b, j = tw.j;
             if (b != cur_b) {
                 if (!mbar_wait(q_empty, (q_it & 1) ^ 1, abort_flag, err, kDevTimeoutProducer)) break;
                 mbar_arrive_expect_tx(q_full, S::B_BYTES);
@@ -167,9 +210,14 @@ __global__ void __launch_bounds__(384, 1)
                 cur_b = b;
             }
             if (!mbar_wait(&raw_empty[rs], rph ^ 1, abort_flag, err, kDevTimeoutProducer)) break;
-            mbar_arrive_expect_tx(&raw_full[rs], S::RAW);
-            tma_load_2d(sRaw + rs * S::RAW, &tm_k8, &raw_full[rs], 0,
-                        b * S_max + j * S::BM);
+            // the tile's 128 key rows are one contiguous block: a single bulk
+            // copy, clamped at the end of the cache (rows past it stay stale
+            // and are never stored)
+            const long long row0 = static_cast<long long>(b) * S_max + j * S::BM;
+            const long long left = static_cast<long long>(B) * S_max - row0;
+            const uint32_t bytes = static_cast<uint32_t>(left < S::BM ? left : S::BM) * S::DI;
+            mbar_arrive_expect_tx(&raw_full[rs], bytes);
+            bulk_load(smem_u32(sRaw + rs * S::RAW), k8 + row0 * S::DI, bytes, &raw_full[rs]);
             last_ph[rs] = static_cast<int>(rph);
             if (++rs == S::RAW_ST) {
                 rs = 0;
@@ -187,9 +235,9 @@ __global__ void __launch_bounds__(384, 1)
         uint32_t acc_it[S::NACC] = {0, 0, 0, 0};
         int cur_b = -1;
         bool ok = true;
-        for (long long g = g_begin; g < g_end && ok; ++g) {
-            const int b = static_cast<int>(g / tps), j = static_cast<int>(g % tps);
-            if (j * S::BM >= seq_len[b]) continue;
+        TileWalk<S::BM> tw;
+        for (tw.init(g_begin, g_end, tps, seq_len); !tw.done() && ok; tw.next()) {
+            const int b = tw.b;
             if (b != cur_b) {
                 if (cur_b >= 0) umma_commit(q_empty);  // previous q no longer read
                 if (!mbar_wait(q_full, q_it & 1, abort_flag, err, kDevTimeoutMma)) break;
@@ -224,15 +272,14 @@ __global__ void __launch_bounds__(384, 1)
         }
         umma_commit(done_bar);
         if (!mbar_wait_drain(done_bar, 0)) atomicCAS(err, 0, kDevTimeoutDrain);
-    } else if (warp >= 4 && warp < 8 && start_ok) {
+    } else if (warp >= 4 && warp < 12 && start_ok) {
         // ------------------------------------------------ e4m3 -> bf16
-        const int t = threadIdx.x - 128;  // 0..127
+        const int t = threadIdx.x - 128;  // 0..255
         int rs = 0, as = 0;
         uint32_t rph = 0, aph = 0;
         bool ok = true;
-        for (long long g = g_begin; g < g_end && ok; ++g) {
-            const int b = static_cast<int>(g / tps), j = static_cast<int>(g % tps);
-            if (j * S::BM >= seq_len[b]) continue;
+        TileWalk<S::BM> tw;
+        for (tw.init(g_begin, g_end, tps, seq_len); !tw.done() && ok; tw.next()) {
             bool got = mbar_wait(&raw_full[rs], rph, abort_flag, err, kDevTimeoutEpilogue);
             got = got && mbar_wait(&a_empty[as], aph ^ 1, abort_flag, err, kDevTimeoutEpilogue);
             got = __all_sync(0xffffffffu, got);
@@ -243,8 +290,8 @@ __global__ void __launch_bounds__(384, 1)
             const uint8_t* raw = sRaw + rs * S::RAW;
             uint8_t* dst = sA + as * S::A_STAGE;
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int c = i * 128 + t;       // 16-byte chunk id in the raw tile
+            for (int i = 0; i < 4; ++i) {
+                const int c = i * 256 + t;       // 16-byte chunk id in the raw tile
                 const int row = c >> 3, c8 = c & 7;
                 const uint4 v = *reinterpret_cast<const uint4*>(raw + c * 16);
                 uint4 lo, hi;
@@ -254,10 +301,14 @@ __global__ void __launch_bounds__(384, 1)
                 *reinterpret_cast<uint4*>(atom + ((ch ^ (row & 7)) << 4)) = lo;
                 *reinterpret_cast<uint4*>(atom + (((ch + 1) ^ (row & 7)) << 4)) = hi;
             }
-            // generic-proxy writes must be visible to the tensor core
+            // generic-proxy writes must be visible to the tensor core; one
+            // arrival per warp keeps the barriers' arrival traffic small
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-            mbar_arrive(&a_full[as]);
-            mbar_arrive(&raw_empty[rs]);
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) {
+                mbar_arrive(&a_full[as]);
+                mbar_arrive(&raw_empty[rs]);
+            }
             if (++rs == S::RAW_ST) {
                 rs = 0;
                 rph ^= 1;
@@ -267,36 +318,38 @@ __global__ void __launch_bounds__(384, 1)
                 aph ^= 1;
             }
         }
-    } else if (warp >= 8 && start_ok) {
+    } else if (warp >= 12 && start_ok) {
         // ------------------------------------------------ epilogue
         const int lq = warp & 3;
         float* wW = sW + lq * H_I;
         int acc = 0;
         uint32_t acc_it[S::NACC] = {0, 0, 0, 0};
         int cur_b = -1;
-        // the next tile (after g) that holds candidates, or g_end
-        auto next_valid = [&](long long g) -> long long {
-            for (++g; g < g_end; ++g) {
-                const int b = static_cast<int>(g / tps), j = static_cast<int>(g % tps);
-                if (j * S::BM < seq_len[b]) return g;
+        // this thread's per-token scales are prefetched SC_RING-1 tiles ahead
+        // (walker `tp`) with cp.async into a per-thread shared-memory ring
+        // (zero past the sequence end), so no register waits on a global load
+        const uint32_t sc_ring = smem_u32(smem + S::OFF_SC) + (lq * 32 + lane) * 4;
+        TileWalk<S::BM> tw, tp;
+        tw.init(g_begin, g_end, tps, seq_len);
+        tp.init(g_begin, g_end, tps, seq_len);
+        auto prefetch_scale = [&](int slot) {
+            if (!tp.done()) {
+                const int s = tp.j * S::BM + lq * 32 + lane;
+                const bool ok = s < tp.n;
+                const float* src = kscale + static_cast<long long>(tp.b) * S_max + (ok ? s : 0);
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(
+                                 sc_ring + slot * S::BM * 4),
+                             "l"(src), "r"(ok ? 4 : 0)
+                             : "memory");
+                tp.next();
             }
-            return g_end;
+            cp_async_commit();
         };
-        // this thread's per-token scale in tile g (0 past the sequence end)
-        auto load_scale = [&](long long g) -> float {
-            if (g >= g_end) return 0.f;
-            const int b = static_cast<int>(g / tps), j = static_cast<int>(g % tps);
-            const int s = j * S::BM + lq * 32 + lane;
-            return s < seq_len[b] ? __ldg(kscale + static_cast<long long>(b) * S_max + s) : 0.f;
-        };
-        // scales are loaded two tiles ahead so their latency hides behind the MMAs
-        long long g = next_valid(g_begin - 1);
-        long long g1 = next_valid(g), g2 = next_valid(g1);
-        float sc0 = load_scale(g), sc1 = load_scale(g1);
-        while (g < g_end) {
-            const float sc2 = load_scale(g2);
-            const int b = static_cast<int>(g / tps), j = static_cast<int>(g % tps);
-            const int n = seq_len[b];
+        int it = 0;
+        for (int p = 0; p < S::SC_RING - 1; ++p) prefetch_scale(p);
+        for (; !tw.done(); tw.next()) {
+            prefetch_scale((it + S::SC_RING - 1) % S::SC_RING);
+            const int b = tw.b, j = tw.j, n = tw.n;
             if (b != cur_b) {
                 __syncwarp();
                 for (int h = lane; h < H_I; h += 32)
@@ -329,15 +382,15 @@ __global__ void __launch_bounds__(384, 1)
                 p[2] = fmaf(wv.z, fmaxf(__uint_as_float(src[(h + 2) & 31]), 0.f), p[2]);
                 p[3] = fmaf(wv.w, fmaxf(__uint_as_float(src[(h + 3) & 31]), 0.f), p[3]);
             }
-            if (s < n) scores[static_cast<long long>(b) * ld + s] = sc0 * ((p[0] + p[1]) + (p[2] + p[3]));
+            cp_async_wait<S::SC_RING - 1>();  // this tile's scale has landed
+            float sc;
+            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(sc) : "r"(sc_ring + (it % S::SC_RING) * S::BM * 4));
+            if (s < n) scores[static_cast<long long>(b) * ld + s] = sc * ((p[0] + p[1]) + (p[2] + p[3]));
             ++acc_it[acc];
             if (++acc == S::NACC) acc = 0;
-            sc0 = sc1;
-            sc1 = sc2;
-            g = g1;
-            g1 = g2;
-            g2 = next_valid(g2);
+            ++it;
         }
+        cp_async_wait<0>();  // no prefetch may still be landing at exit
     }
 
     tc_fence_before();
@@ -360,17 +413,15 @@ static int launch_decode_t(ic_ctx* ctx, const void* q, const void* w, const uint
         if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaFuncSetAttribute(index_decode)");
         attr_set = true;
     }
-    CUtensorMap tm_q, tm_k8;
+    CUtensorMap tm_q;
     int rc = make_tmap_bf16_2d(ctx, &tm_q, q, static_cast<uint64_t>(B) * H_I, 128, H_I);
-    if (rc) return rc;
-    rc = make_tmap_u8_2d(ctx, &tm_k8, kI8, static_cast<uint64_t>(B) * S_max, 128, 128, 128);
     if (rc) return rc;
     const int tps = (S_max + S::BM - 1) / S::BM;
     const long long total = static_cast<long long>(B) * tps;
     const int grid = total < ctx->num_sms ? static_cast<int>(total) : ctx->num_sms;
     LaunchScope ls(ctx, IC_K_INDEX_SCORE_DECODE, stream);
-    k_index_score_decode<H_I><<<grid, 384, S::SMEM, stream>>>(
-        tm_q, tm_k8, static_cast<const __nv_bfloat16*>(w), kI_scale, seq_len, B, S_max, tps,
+    k_index_score_decode<H_I><<<grid, 512, S::SMEM, stream>>>(
+        tm_q, kI8, static_cast<const __nv_bfloat16*>(w), kI_scale, seq_len, B, S_max, tps,
         scores, static_cast<long long>(ld), ctx->dev_err);
     cudaError_t e = ls.done();
     if (e != cudaSuccess) return cuda_fail(ctx, e, "index_score_decode launch");

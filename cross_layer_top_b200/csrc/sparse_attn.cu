@@ -5,10 +5,10 @@
 // Accelerating Sparse Attention via Cross-Layer Index Reuse", Figure 2 step
 // SPARSEATTN).  One K/V head is shared by all Hq <= 16 query heads.
 //
-// Design: one CTA (4 warps, two CTAs per SM) per (query row, key split).
+// Design: one CTA (6 warps, two CTAs per SM) per (query row, key split).
 // The 16 query heads form the M = 16 rows of mma.m16n8k16 tiles, so one
 // gathered K/V row serves every head.  Each warp owns chunks of 16 index
-// slots and a 3-deep ring: lane l always copies the same 16-byte piece
+// slots and a 2-deep ring: lane l always copies the same 16-byte piece
 // (l mod d/8) of its rows with cp.async (zero-filled for masked slots),
 // XOR-swizzled by row so ldmatrix is conflict-free, while the warp computes
 // an earlier chunk: S = Q K^T, an online softmax in the
@@ -22,14 +22,22 @@
 #include "ic_device.cuh"
 #include "ic_internal.h"
 
+// Warps per CTA and gather-ring depth (compile-time tuning knobs).
+#ifndef IC_ATTN_WARPS
+#define IC_ATTN_WARPS 6
+#endif
+#ifndef IC_ATTN_STAGES
+#define IC_ATTN_STAGES 2
+#endif
+
 namespace ic {
 
 template <int D>
 struct AttnShape {
-    static constexpr int WARPS = 4;
+    static constexpr int WARPS = IC_ATTN_WARPS;
     static constexpr int THREADS = WARPS * 32;
     static constexpr int CH = 16;  // index slots per warp chunk
-    static constexpr int STAGES = 3;
+    static constexpr int STAGES = IC_ATTN_STAGES;
     static constexpr int ROWB = D * 2;
     static constexpr int ROWP = ROWB;  // row pitch; 16-byte pieces XOR-swizzled by row
     static constexpr int STAGE_BYTES = 2 * CH * ROWP;  // K rows then V rows
@@ -80,8 +88,9 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
     const int32_t* irow = idx + static_cast<long long>(r) * k + slot0;
     bool bad = false;
     int last = -1;
-    for (int i = tid; i < nk; i += S::THREADS) {
-        int v = irow[i];
+    const int nk_pad = (nk + S::CH - 1) / S::CH * S::CH;  // whole chunks, padded with -1
+    for (int i = tid; i < nk_pad; i += S::THREADS) {
+        int v = i < nk ? irow[i] : -1;
         if (v < -1 || v >= kv_len) {
             bad = true;
             v = -1;
@@ -113,32 +122,29 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
     const uint32_t wst = smem_u32(smem + S::OFF_ST + warp * S::WARP_BYTES);
     const int nch = (nk_eff + S::CH - 1) / S::CH;
     const int my_n = nch > warp ? (nch - warp + S::WARPS - 1) / S::WARPS : 0;
-    uint32_t vmask[S::STAGES];
 
-    // lane l copies piece (l % PPR) of rows l / PPR, + RPI, ... of K and V
+    // lane l copies piece (l % PPR) of rows l / PPR, + RPI, ... of K and V;
+    // its destination offsets inside a stage are fixed, so precompute them
     constexpr int PPR = D / 8;        // 16-byte pieces per row
     constexpr int RPI = 32 / PPR;     // rows per warp instruction
+    constexpr int NI = S::CH / RPI;   // copy instructions per lane per tensor
     const int piece = lane % PPR, prow = lane / PPR;
+    uint32_t dsto[NI];
+#pragma unroll
+    for (int i = 0; i < NI; ++i) dsto[i] = swz<D>(prow + i * RPI, piece);
+    const char* Kc = reinterpret_cast<const char*>(Kb) + piece * 16;
+    const char* Vc = reinterpret_cast<const char*>(Vb) + piece * 16;
     auto issue = [&](int j) {
         if (j < my_n) {
-            const int st = j % S::STAGES;
             const int c0 = (warp + j * S::WARPS) * S::CH;
-            {
-                const int slot = c0 + (lane & 15);
-                const bool v = slot < nk && sIdx[slot] >= 0;
-                vmask[st] = __ballot_sync(0xffffffffu, v && lane < 16) & 0xffffu;
-            }
-            const uint32_t kdst = wst + st * S::STAGE_BYTES;
-            const uint32_t vdst = kdst + S::CH * S::ROWP;
+            const uint32_t kdst = wst + (j % S::STAGES) * S::STAGE_BYTES;
 #pragma unroll
-            for (int i = 0; i < S::CH / RPI; ++i) {
-                const int row = prow + i * RPI;
-                const int slot = c0 + row;
-                const int sidx = slot < nk ? sIdx[slot] : -1;
+            for (int i = 0; i < NI; ++i) {
+                const int sidx = sIdx[c0 + prow + i * RPI];
                 const bool ok = sidx >= 0;
-                const long long off = static_cast<long long>(ok ? sidx : 0) * D + piece * 8;
-                cp_async16(kdst + swz<D>(row, piece), Kb + off, ok);
-                cp_async16(vdst + swz<D>(row, piece), Vb + off, ok);
+                const uint32_t off = static_cast<uint32_t>(ok ? sidx : 0) * S::ROWB;
+                cp_async16(kdst + dsto[i], Kc + off, ok);
+                cp_async16(kdst + S::CH * S::ROWP + dsto[i], Vc + off, ok);
             }
         }
         cp_async_commit();
@@ -147,7 +153,9 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
     float o[D / 8][4];
 #pragma unroll
     for (int i = 0; i < D / 8; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;  // rows g and g+8
+    // running references (log2 domain, scale folded in) and partial sums,
+    // rows g = lane/4 and g + 8
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
 #pragma unroll
     for (int j = 0; j < S::STAGES - 1; ++j) issue(j);
@@ -158,7 +166,8 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
         issue(j + S::STAGES - 1);  // into the stage of chunk j-1, whose reads are done
         const uint32_t kb = wst + st * S::STAGE_BYTES;
         const uint32_t vb = kb + S::CH * S::ROWP;
-        const uint32_t cmask = vmask[st];
+        const int c0 = (warp + j * S::WARPS) * S::CH;
+        const uint32_t cmask = __ballot_sync(0xffffffffu, sIdx[c0 + (lane & 15)] >= 0) & 0xffffu;
 
         float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
 #pragma unroll
@@ -171,23 +180,26 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
             mma_bf16_16816(s[0], qa[kk], b0, b1);
             mma_bf16_16816(s[1], qa[kk], b2, b3);
         }
-        float x[2][4];
+        if (cmask != 0xffffu) {  // warp-uniform: only chunks with masked slots
 #pragma unroll
-        for (int nt = 0; nt < 2; ++nt)
+            for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-                const int col = nt * 8 + 2 * (lane & 3) + (e & 1);
-                x[nt][e] = ((cmask >> col) & 1u) ? s[nt][e] * scale_log2 : -INFINITY;
-            }
-        float mx0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
-        float mx1 = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
+                for (int e = 0; e < 4; ++e) {
+                    const int col = nt * 8 + 2 * (lane & 3) + (e & 1);
+                    if (!((cmask >> col) & 1u)) s[nt][e] = -INFINITY;
+                }
+        }
+        float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+        float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+        mx0 *= scale_log2;  // scale > 0 keeps the order
+        mx1 *= scale_log2;
         // lazy rescale: move the reference only when a logit passes it by 2^8
         if (mx0 > m0 + S::kRescaleThreshold) {
-            const float a = exp2f(m0 - mx0);  // 0 while nothing was seen
+            const float a = ex2_approx(m0 - mx0);  // 0 while nothing was seen
             l0 *= a;
 #pragma unroll
             for (int i = 0; i < D / 8; ++i) {
@@ -197,7 +209,7 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
             m0 = mx0;
         }
         if (mx1 > m1 + S::kRescaleThreshold) {
-            const float a = exp2f(m1 - mx1);
+            const float a = ex2_approx(m1 - mx1);
             l1 *= a;
 #pragma unroll
             for (int i = 0; i < D / 8; ++i) {
@@ -206,15 +218,15 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
             }
             m1 = mx1;
         }
-        const float r0 = m0 == -INFINITY ? 0.f : m0;
-        const float r1 = m1 == -INFINITY ? 0.f : m1;
+        const float n0 = m0 == -INFINITY ? 0.f : -m0;
+        const float n1 = m1 == -INFINITY ? 0.f : -m1;
         float p[2][4];
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-            p[nt][0] = exp2f(x[nt][0] - r0);
-            p[nt][1] = exp2f(x[nt][1] - r0);
-            p[nt][2] = exp2f(x[nt][2] - r1);
-            p[nt][3] = exp2f(x[nt][3] - r1);
+            p[nt][0] = ex2_approx(fmaf(s[nt][0], scale_log2, n0));
+            p[nt][1] = ex2_approx(fmaf(s[nt][1], scale_log2, n0));
+            p[nt][2] = ex2_approx(fmaf(s[nt][2], scale_log2, n1));
+            p[nt][3] = ex2_approx(fmaf(s[nt][3], scale_log2, n1));
         }
         l0 += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
         l1 += (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
@@ -269,7 +281,7 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
         if (M != -INFINITY) {
 #pragma unroll
             for (int w = 0; w < S::WARPS; ++w) {
-                const float f = exp2f(mML[w * 32 + h] - M);
+                const float f = ex2_approx(mML[w * 32 + h] - M);
                 acc += mO[w * 16 * D + h * D + dd] * f;
                 lsum += mML[w * 32 + 16 + h] * f;
             }
@@ -306,7 +318,7 @@ __global__ void __launch_bounds__(256)
         float L = 0.f;
         for (int s = 0; s < nsplit; ++s) {
             const float* ps = pr + s * (16 * D + 32);
-            const float f = M == -INFINITY ? 0.f : exp2f(ps[16 * D + h] - M);
+            const float f = M == -INFINITY ? 0.f : ex2_approx(ps[16 * D + h] - M);
             sf[s][h] = f;
             L += ps[16 * D + 16 + h] * f;
         }
