@@ -112,9 +112,8 @@ class ClockSampler:
 # ------------------------------------------------------------- our arm
 def make_prefill_inputs(cfg, rank, device):
     """All layer tensors of one sequence; each rank draws its own sequence."""
-    import dataclasses
     from cross_layer_top_b200 import synth
-    cfg = dataclasses.replace(cfg, seed=cfg.seed + 7919 * rank)
+    cfg = rank_config(cfg, rank)
     layers = []
     for l in range(cfg.n_layers):
         lay = synth.prefill_layer(cfg, l, device)
@@ -145,6 +144,11 @@ def run_ours(args, rank, world, local_rank):
     def step():
         ic.ic_run_stack(ctx, pat, None, dims, cache, layer_array=arr)
 
+    # the clock sampler starts before the warm-up so that it is producing
+    # samples (under load) by the time the timed region begins
+    clocks = ClockSampler(local_rank)
+    clocks.start()
+    time.sleep(0.3)
     for _ in range(args.warmup):
         step()
     ctx.sync_status()
@@ -155,8 +159,6 @@ def run_ours(args, rank, world, local_rank):
     ctx.reset_timing()
     ctx.set_timing(True)
     launches0 = ctx.launch_count()
-    clocks = ClockSampler(local_rank)
-    clocks.start()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for _ in range(args.steps)]
     dist_barrier(world)
@@ -181,7 +183,7 @@ def run_ours(args, rank, world, local_rank):
     total_ms = dist_max(total_ms, world)
 
     pairs_step = scored_pairs(L, k, n_f)
-    value = pairs_step * args.steps * world / (total_ms / 1e3)
+    value = weak_scaling_value(pairs_step, args.steps, world, total_ms)
     ms_per_step = total_ms / args.steps
 
     # ------------------------------------------------ roofline of the dominant kernel
@@ -231,8 +233,13 @@ def run_ours(args, rank, world, local_rank):
         e2e = run_e2e(args, ctx, pat, dims, cfg, layers, cache, world, pairs_step, stream)
 
     # ------------------------------------------------ decode step (extra evidence)
+    del layers, arr
+    torch.cuda.empty_cache()
     if not args.no_decode:
         extra["decode"] = run_decode(args, ctx, peaks, peak_src, local_rank)
+    if not args.no_extended:
+        extra["long_prefill"] = run_long_prefill(args, ctx, peaks, local_rank)
+        extra["decode_retention_sweep"] = run_decode_sweep(args, ctx, local_rank)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -379,6 +386,100 @@ def run_decode(args, ctx, peaks, peak_src, local_rank):
     return res
 
 
+def _time_stack(ctx, pat, dims, cache, arr, steps, stream):
+    from cross_layer_top_b200 import indexcache as ic
+    ctx.reset_timing()
+    ctx.set_timing(True)
+    tot = 0.0
+    for _ in range(steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        ic.ic_run_stack(ctx, pat, None, dims, cache, layer_array=arr)
+        b.record(stream)
+        b.synchronize()
+        tot += a.elapsed_time(b)
+    ctx.set_timing(False)
+    ctx.sync_status()
+    kt = {n: ctx.get_timing(i)[0] / steps for i, n in enumerate(ic.KERNEL_NAMES)}
+    return tot / steps, kt
+
+
+def run_long_prefill(args, ctx, peaks, local_rank):
+    """The long-prefill workload (L = 131072, FSSS), and the same layers
+    with an all-F pattern: stack ms and the indexer's share of the all-F
+    stack (indexer score + top-k time over stack time)."""
+    from cross_layer_top_b200 import indexcache as ic
+    from cross_layer_top_b200 import synth
+    cfg = synth.CONFIGS["long_prefill_allF"]
+    dev = torch.device("cuda", local_rank)
+    L, k = cfg.L, cfg.k
+    layers = []
+    for l in range(cfg.n_layers):
+        lay = synth.prefill_layer(cfg, l, dev, indexer=True)
+        lay["out"] = torch.empty((L, cfg.Hq, cfg.d), dtype=torch.bfloat16, device=dev)
+        layers.append(lay)
+    dims = ic.stack_dims(ic.IC_PREFILL, cfg.H_I, cfg.d_I, k, cfg.Hq, cfg.d, L=L)
+    cache = torch.empty((L, k), dtype=torch.int32, device=dev)
+    arr = ic.make_stack_layers(layers)
+    stream = torch.cuda.current_stream()
+    res = {"workload": "long prefill: 1 sequence, L=131072, 4 layers, H_I=64, d_I=128, k=2048, "
+                       "16 query heads, d=128"}
+    for pattern in ("FSSS", "FFFF"):
+        pat = ic.ic_create_pattern(pattern)
+        ic.ic_run_stack(ctx, pat, None, dims, cache, layer_array=arr)  # warm-up
+        ms, kt = _time_stack(ctx, pat, dims, cache, arr, 2, stream)
+        pairs = scored_pairs(L, k, pattern.count("F"))
+        ent = {"stack_ms": ms, "kernels_ms": {n: round(v, 3) for n, v in kt.items()},
+               "scored_pairs_per_s": pairs / (ms / 1e3)}
+        if kt["index_score"]:
+            tf = 2 * cfg.H_I * cfg.d_I * pairs / (kt["index_score"] / 1e3) / 1e12
+            ent["indexer_tflops"] = round(tf, 1)
+            ent["indexer_frac_of_sustained_bf16"] = round(
+                tf / peaks.get("bf16_tflops_sustained", 1400.0), 4)
+        ent["indexer_share"] = round((kt["index_score"] + kt["topk"]) / ms, 4)
+        res[pattern] = ent
+    res["speedup_FSSS_vs_FFFF"] = res["FFFF"]["stack_ms"] / res["FSSS"]["stack_ms"]
+    del layers, arr, cache
+    torch.cuda.empty_cache()
+    return res
+
+
+def run_decode_sweep(args, ctx, local_rank):
+    """200K-context decode: 8 sequences x 200001 candidates, 47 layers, one
+    decode step at uniform retention 1/1, 1/2, 1/4, 1/8 (the same layer
+    tensors; S layers ignore their indexer inputs)."""
+    from cross_layer_top_b200 import indexcache as ic
+    from cross_layer_top_b200 import synth
+    cfg = synth.CONFIGS["decode_sweep_r1"]
+    dev = torch.device("cuda", local_rank)
+    B, S, k = cfg.B, cfg.S, cfg.k
+    layers = []
+    for l in range(cfg.n_layers):
+        lay = synth.decode_layer(cfg, l, dev, indexer=True)
+        lay["out"] = torch.empty((B, cfg.Hq, cfg.d), dtype=torch.bfloat16, device=dev)
+        layers.append(lay)
+    seq_len = layers[0]["seq_len"]
+    dims = ic.stack_dims(ic.IC_DECODE, cfg.H_I, cfg.d_I, k, cfg.Hq, cfg.d, B=B, S_max=S,
+                         seq_len=seq_len)
+    cache = torch.empty((B, k), dtype=torch.int32, device=dev)
+    arr = ic.make_stack_layers(layers, ic.IC_DECODE)
+    stream = torch.cuda.current_stream()
+    res = {"workload": "decode: 8 sequences x (200000 cached + 1 new) tokens, 47 layers, "
+                       "FP8 indexer keys, k=2048"}
+    for r in (1, 2, 4, 8):
+        pat = ic.ic_pattern_uniform(cfg.n_layers, r)
+        for _ in range(2):
+            ic.ic_run_stack(ctx, pat, None, dims, cache, layer_array=arr)
+        ms, kt = _time_stack(ctx, pat, dims, cache, arr, 5, stream)
+        res["r%d" % r] = {"pattern_F_layers": str(pat).count("F"), "step_ms": ms,
+                          "tokens_per_s": B / (ms / 1e3),
+                          "kernels_ms": {n: round(v, 4) for n, v in kt.items()}}
+    res["speedup_r4_vs_r1"] = res["r1"]["step_ms"] / res["r4"]["step_ms"]
+    del layers, arr, cache
+    torch.cuda.empty_cache()
+    return res
+
+
 # ------------------------------------------------------- the oracle on CPU
 def cpu_baseline(cfg, budget_s=15.0, rows_idx=None, rows_att=None):
     """Time the CPU oracle on a bounded row sample of the prefill stack and
@@ -463,24 +564,39 @@ def dist_barrier(world):
         torch.distributed.barrier()
 
 
-def dist_max(x, world):
+def dist_max(x, world, device="cuda"):
+    """Max over ranks (plumbing only: the step time and nothing else)."""
     if world == 1:
         return x
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    t = torch.tensor([x], dtype=torch.float64, device=device)
     torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
     return float(t.item())
+
+
+def rank_config(cfg, rank):
+    """Weak scaling: every rank runs its own independent sequence of the same
+    shape (a different seed), with no data-path exchange."""
+    import dataclasses
+    return dataclasses.replace(cfg, seed=cfg.seed + 7919 * rank)
+
+
+def weak_scaling_value(units_per_step_per_rank, steps, world, max_rank_ms):
+    """Whole-job throughput: units processed by all ranks / max rank time."""
+    return units_per_step_per_rank * steps * world / (max_rank_ms / 1e3)
 
 
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--steps", type=int, default=40)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=16.0)
+    ap.add_argument("--no-extended", action="store_true",
+                    help="skip the long-prefill and 200K-decode retention-sweep timings")
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the decode workload (not the contract line)")
     ap.add_argument("--decode-layers", type=int, default=0)

@@ -17,8 +17,9 @@
 // rescaled), and O += P V.  Slots holding -1 (or an out-of-range index,
 // which is also latched as an error) are masked and gather zeros; the
 // chunks after the last valid slot are skipped.  The four warps' (m, l, O)
-// merge through shared memory; one split writes bf16 output, several
-// splits write fp32 partials merged by k_attn_combine (decode).
+// merge through shared memory; one split writes bf16 output; with several
+// splits (decode) each CTA writes an fp32 partial and the row's last CTA to
+// finish merges them (counter + threadfence, no second launch).
 #include "ic_device.cuh"
 #include "ic_internal.h"
 
@@ -68,7 +69,7 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
                   const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ idx, int Hq,
                   int k, int rows_per_seq, long long kv_seq_stride, int kv_len, float scale_log2,
                   int nsplit, int kps, __nv_bfloat16* __restrict__ out,
-                  float* __restrict__ part, int* __restrict__ err) {
+                  float* __restrict__ part, int* __restrict__ row_done, int* __restrict__ err) {
     using S = AttnShape<D>;
     extern __shared__ __align__(128) uint8_t smem[];
     const int r = blockIdx.x, split = blockIdx.y;
@@ -298,39 +299,43 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
             }
         }
     }
-}
+    if (nsplit == 1) return;
 
-// Merge the per-split partials of each row:
-//   out = sum_s O_s 2^(m_s - M) / sum_s l_s 2^(m_s - M),  M = max_s m_s.
-// The per-(split, head) factors are computed once into shared memory.
-template <int D>
-__global__ void __launch_bounds__(256)
-    k_attn_combine(const float* __restrict__ part, int Hq, int nsplit,
-                   __nv_bfloat16* __restrict__ out) {
-    __shared__ float sf[64][16];
-    __shared__ float sinv[16];
-    const int r = blockIdx.x;
-    const float* pr = part + static_cast<long long>(r) * nsplit * (16 * D + 32);
-    if (threadIdx.x < 16) {
-        const int h = threadIdx.x;
+    // The last CTA of the row to finish merges every split's partial:
+    //   out = sum_s O_s 2^(m_s - M) / sum_s l_s 2^(m_s - M),  M = max_s m_s.
+    // Publication: partials -> __threadfence -> counter increment; the CTA
+    // that takes the counter to nsplit resets it for the next launch.
+    __threadfence();
+    __syncthreads();
+    int* s_flag = s_last;  // reuse: the slot scan is long finished
+    if (tid == 0) *s_flag = atomicAdd(&row_done[r], 1) == nsplit - 1;
+    __syncthreads();
+    if (!*s_flag) return;
+    __threadfence();
+    const float* part_row = part + static_cast<long long>(r) * nsplit * (16 * D + 32);
+    float* sf = mO;                // [nsplit][16] factors (merge buffer is free again)
+    float* sinv = mO + 64 * 16;    // [16]
+    if (tid < 16) {
+        const int h = tid;
         float M = -INFINITY;
-        for (int s = 0; s < nsplit; ++s) M = fmaxf(M, pr[s * (16 * D + 32) + 16 * D + h]);
+        for (int q = 0; q < nsplit; ++q) M = fmaxf(M, __ldcg(part_row + q * (16 * D + 32) + 16 * D + h));
         float L = 0.f;
-        for (int s = 0; s < nsplit; ++s) {
-            const float* ps = pr + s * (16 * D + 32);
-            const float f = M == -INFINITY ? 0.f : ex2_approx(ps[16 * D + h] - M);
-            sf[s][h] = f;
-            L += ps[16 * D + 16 + h] * f;
+        for (int q = 0; q < nsplit; ++q) {
+            const float* ps = part_row + q * (16 * D + 32);
+            const float f = M == -INFINITY ? 0.f : ex2_approx(__ldcg(ps + 16 * D + h) - M);
+            sf[q * 16 + h] = f;
+            L += __ldcg(ps + 16 * D + 16 + h) * f;
         }
         sinv[h] = L > 0.f ? 1.f / L : 0.f;
     }
     __syncthreads();
-    for (int e = threadIdx.x; e < Hq * D; e += blockDim.x) {
+    for (int e = tid; e < Hq * D; e += S::THREADS) {
         const int h = e / D, dd = e % D;
         float acc = 0.f;
-        for (int s = 0; s < nsplit; ++s) acc += pr[s * (16 * D + 32) + h * D + dd] * sf[s][h];
+        for (int q = 0; q < nsplit; ++q) acc += __ldcg(part_row + q * (16 * D + 32) + h * D + dd) * sf[q * 16 + h];
         out[(static_cast<long long>(r) * Hq + h) * D + dd] = __float2bfloat16_rn(acc * sinv[h]);
     }
+    if (tid == 0) row_done[r] = 0;
 }
 
 template <int D>
@@ -347,27 +352,37 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
         attr_set = true;
     }
     // Split the index slots across CTAs when there are too few rows to fill
-    // the GPU (decode): aim for ~4 CTAs per SM, whole warp rounds per split.
-    constexpr int unit = S::CH * S::WARPS;
+    // the GPU (decode): about one wave at two CTAs per SM, whole chunks per
+    // split, at most 64 splits.
     int nsplit = 1;
-    const int target = 4 * ctx->num_sms;
+    const int target = 2 * ctx->num_sms;
     if (rows < target) {
-        nsplit = (target + rows - 1) / rows;
-        const int max_split = (k + unit - 1) / unit;
+        nsplit = target / rows;
+        const int max_split = (k + S::CH - 1) / S::CH;
         if (nsplit > max_split) nsplit = max_split;
         if (nsplit > 64) nsplit = 64;
         if (nsplit < 1) nsplit = 1;
     }
     int kps = (k + nsplit - 1) / nsplit;
-    kps = (kps + unit - 1) / unit * unit;
+    kps = (kps + S::CH - 1) / S::CH * S::CH;
     nsplit = (k + kps - 1) / kps;
     float* part = nullptr;
+    int* row_done = nullptr;
     if (nsplit > 1) {
-        const size_t bytes = static_cast<size_t>(rows) * nsplit * (16 * D + 32) * sizeof(float);
+        // partials, then one completion counter per row (zeroed here once;
+        // every launch leaves them at zero)
+        const size_t pbytes = static_cast<size_t>(rows) * nsplit * (16 * D + 32) * sizeof(float);
+        const size_t bytes = pbytes + static_cast<size_t>(rows) * sizeof(int);
+        const bool fresh = ctx->attn_part_cap < bytes || !ctx->attn_part;
         int rc = ensure_buffer(ctx, reinterpret_cast<void**>(&ctx->attn_part), &ctx->attn_part_cap,
                                bytes);
         if (rc) return rc;
         part = ctx->attn_part;
+        row_done = reinterpret_cast<int*>(reinterpret_cast<char*>(part) + pbytes);
+        if (fresh) {
+            cudaError_t e = cudaMemsetAsync(ctx->attn_part, 0, ctx->attn_part_cap, stream);
+            if (e != cudaSuccess) return cuda_fail(ctx, e, "sparse_attn: counters");
+        }
     }
     const float scale_log2 = scale * 1.4426950408889634f;
     {
@@ -377,16 +392,9 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
             static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
             static_cast<const __nv_bfloat16*>(V), idx, Hq, k, rows_per_seq,
             static_cast<long long>(kv_seq_stride), kv_len, scale_log2, nsplit, kps,
-            static_cast<__nv_bfloat16*>(out), part, ctx->dev_err);
+            static_cast<__nv_bfloat16*>(out), part, row_done, ctx->dev_err);
         cudaError_t e = ls.done();
         if (e != cudaSuccess) return cuda_fail(ctx, e, "sparse_attn launch");
-    }
-    if (nsplit > 1) {
-        LaunchScope ls(ctx, IC_K_ATTN_COMBINE, stream);
-        k_attn_combine<D><<<rows, 256, 0, stream>>>(part, Hq, nsplit,
-                                                    static_cast<__nv_bfloat16*>(out));
-        cudaError_t e = ls.done();
-        if (e != cudaSuccess) return cuda_fail(ctx, e, "attn_combine launch");
     }
     return IC_OK;
 }

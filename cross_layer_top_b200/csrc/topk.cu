@@ -36,6 +36,10 @@ __device__ __forceinline__ uint32_t order_key(float x) {
     if ((b & 0x7fffffffu) == 0) b = 0;  // -0.0 == +0.0
     return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
 }
+// inverse of order_key (up to the sign of zero)
+__device__ __forceinline__ float key_float(uint32_t u) {
+    return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
+}
 
 struct TopkShared {
     uint32_t hist[2048];
@@ -51,13 +55,13 @@ struct TopkShared {
 // each) such that count(bins > b) < krem <= count(bins >= b).  Writes the
 // bin and count(bins > b) to S.bin / S.above.  Must be called by all threads.
 template <int NB>
-__device__ __forceinline__ void find_bin(TopkShared& S, uint32_t krem) {
+__device__ __forceinline__ void find_bin(TopkShared& S, uint32_t krem, const uint32_t* hist) {
     constexpr int PER = NB / kTopkThreads;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint32_t c[PER], tot = 0;
 #pragma unroll
     for (int b = 0; b < PER; ++b) {
-        c[b] = S.hist[tid * PER + b];
+        c[b] = hist[tid * PER + b];
         tot += c[b];
     }
     // inclusive suffix sum within the warp (higher lanes hold higher bins)
@@ -88,6 +92,10 @@ __device__ __forceinline__ void find_bin(TopkShared& S, uint32_t krem) {
         }
     }
     __syncthreads();
+}
+template <int NB>
+__device__ __forceinline__ void find_bin(TopkShared& S, uint32_t krem) {
+    find_bin<NB>(S, krem, S.hist);
 }
 
 template <bool IN_SMEM>
@@ -218,10 +226,289 @@ __global__ void __launch_bounds__(kTopkThreads)
     // n > k here, so exactly k positions were written; nothing to pad.
 }
 
+// ------------------------------------------------------------------------
+// Cluster variant for few long rows (the decode step: B rows of up to
+// ~200K candidates).  One thread-block cluster of kClusterCtas CTAs per row;
+// its first-level histogram has 2048 bins uniform in VALUE between the
+// row's min and max (a monotone function of the score, so every key in a
+// higher bin is larger), which narrows bin b1 to a short candidate list;
+// CTA `rank` stages the row segment [rank*seg, (rank+1)*seg) in its shared
+// memory.  The row-wide quantities (min/max, histograms, candidate lists,
+// per-segment counts) are exchanged through distributed shared memory
+// (mapa + ld.shared::cluster) between cluster barriers; every CTA then takes
+// the same decisions, and each writes the selected positions of its own
+// segment at the offsets of the segments before it.  Same output contract
+// as k_topk.
+constexpr int kClusterCtas = 8;
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile(
+        "barrier.cluster.arrive.release.aligned;\n\t"
+        "barrier.cluster.wait.acquire.aligned;" ::
+            : "memory");
+}
+__device__ __forceinline__ uint32_t dsmem_addr(const void* local, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
+    return r;
+}
+__device__ __forceinline__ uint32_t dsmem_ld(uint32_t addr) {
+    uint32_t v;
+    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+struct TopkClusterShared {
+    TopkShared S;
+    uint32_t hist_all[2048];
+    uint32_t seg_kmin, seg_kmax, seg_cg, seg_ce;
+};
+
+__global__ void __launch_bounds__(kTopkThreads)
+    k_topk_cluster(const float* __restrict__ scores, long long ld, int k,
+                   const int32_t* __restrict__ row_len, int causal_base,
+                   int32_t* __restrict__ out, long long ld_out, int seg_cap) {
+    // dynamic shared memory: the staged segment, then the merged candidates
+    extern __shared__ uint32_t srow[];
+    uint32_t* cand_all = srow + seg_cap;
+    __shared__ TopkClusterShared CS;
+    TopkShared& S = CS.S;
+    const int r = blockIdx.y;
+    const uint32_t rank = cluster_rank();
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n = row_len ? row_len[r] : causal_base + r + 1;
+    int32_t* o = out + static_cast<long long>(r) * ld_out;
+    if (n <= k) {  // the same for every CTA of the cluster: no cluster barrier is reached
+        if (rank == 0)
+            for (int i = tid; i < k; i += kTopkThreads) o[i] = i < n ? i : -1;
+        return;
+    }
+    const int seg = ((n + kClusterCtas - 1) / kClusterCtas + 3) / 4 * 4;
+    const int s0 = min(n, static_cast<int>(rank) * seg), s1 = min(n, s0 + seg);
+    const int m = s1 - s0;  // this CTA's segment length
+    const float* row = scores + static_cast<long long>(r) * ld + s0;
+
+    // ---- A: stage the segment, cluster-wide key range
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    {
+        const int m4 = m >> 2;
+        const float4* row4 = reinterpret_cast<const float4*>(row);
+        for (int i = tid; i < m4; i += kTopkThreads) {
+            const float4 v = __ldg(row4 + i);
+            const uint32_t u0 = order_key(v.x), u1 = order_key(v.y);
+            const uint32_t u2 = order_key(v.z), u3 = order_key(v.w);
+            *reinterpret_cast<uint4*>(srow + 4 * i) = make_uint4(u0, u1, u2, u3);
+            kmin = min(kmin, min(min(u0, u1), min(u2, u3)));
+            kmax = max(kmax, max(max(u0, u1), max(u2, u3)));
+        }
+        for (int i = 4 * m4 + tid; i < m; i += kTopkThreads) {
+            const uint32_t u = order_key(__ldg(row + i));
+            srow[i] = u;
+            kmin = min(kmin, u);
+            kmax = max(kmax, u);
+        }
+    }
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    if (lane == 0) {
+        S.wcnt[0][warp] = kmin;
+        S.wcnt[1][warp] = kmax;
+    }
+    for (int i = tid; i < 2048; i += kTopkThreads) S.hist[i] = 0;
+    if (tid == 0) S.ncand = 0;
+    __syncthreads();
+    if (tid == 0) {
+        uint32_t a = 0xFFFFFFFFu, b = 0u;
+        for (int w = 0; w < kTopkWarps; ++w) {
+            a = min(a, S.wcnt[0][w]);
+            b = max(b, S.wcnt[1][w]);
+        }
+        CS.seg_kmin = a;
+        CS.seg_kmax = b;
+    }
+    cluster_sync_all();
+    kmin = 0xFFFFFFFFu;
+    kmax = 0u;
+    for (uint32_t q = 0; q < kClusterCtas; ++q) {
+        kmin = min(kmin, dsmem_ld(dsmem_addr(&CS.seg_kmin, q)));
+        kmax = max(kmax, dsmem_ld(dsmem_addr(&CS.seg_kmax, q)));
+    }
+    const float xmin = key_float(kmin), xmax = key_float(kmax);
+    const float span = xmax - xmin;
+    const float inv = 2047.0f / span;
+    const bool by_value = span > 0.f && isfinite(span) && isfinite(inv) && inv > 0.f;
+    auto bin_of = [&](uint32_t u) -> uint32_t {
+        if (!by_value) return u >> 21;
+        return static_cast<uint32_t>(fminf((key_float(u) - xmin) * inv, 2047.0f));
+    };
+    // cluster-wide histogram: local counts, then every CTA sums all of them
+    auto cluster_hist = [&]() {
+        cluster_sync_all();  // every segment histogram is complete
+        for (int bb = tid; bb < 2048; bb += kTopkThreads) {
+            uint32_t t = 0;
+            for (uint32_t q = 0; q < kClusterCtas; ++q) t += dsmem_ld(dsmem_addr(&S.hist[bb], q));
+            CS.hist_all[bb] = t;
+        }
+        cluster_sync_all();  // nobody rewrites a histogram another CTA still reads
+    };
+    for (int i = tid; i < m; i += kTopkThreads) atomicAdd(&S.hist[bin_of(srow[i])], 1u);
+    cluster_hist();
+    find_bin<2048>(S, static_cast<uint32_t>(k), CS.hist_all);
+    const uint32_t b1 = S.bin;
+    uint32_t krem = static_cast<uint32_t>(k) - S.above;
+    const uint32_t in_bin = CS.hist_all[b1];
+    __syncthreads();
+
+    // ---- B: candidates of bin b1 from every segment, or (massive ties)
+    // cluster-wide radix passes over the bin's keys
+    const bool use_cand = in_bin <= static_cast<uint32_t>(kCandCap);
+    int ncand = 0;
+    if (use_cand) {
+        for (int i = tid; i < m; i += kTopkThreads) {
+            const uint32_t u = srow[i];
+            if (bin_of(u) == b1) S.cand[atomicAdd(&S.ncand, 1u)] = u;
+        }
+        cluster_sync_all();
+        for (uint32_t q = 0; q < kClusterCtas; ++q) {
+            const int nq = static_cast<int>(dsmem_ld(dsmem_addr(&S.ncand, q)));
+            for (int i = tid; i < nq; i += kTopkThreads)
+                cand_all[ncand + i] = dsmem_ld(dsmem_addr(&S.cand[i], q));
+            ncand += nq;
+        }
+        cluster_sync_all();
+    }
+    uint32_t prefix = 0, mask = 0;
+#pragma unroll 1
+    for (int pass = 0; pass < 3; ++pass) {
+        const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
+        const uint32_t dmask = pass == 2 ? 0x3FFu : 0x7FFu;
+        for (int i = tid; i < 2048; i += kTopkThreads) S.hist[i] = 0;
+        __syncthreads();
+        if (use_cand) {
+            for (int i = tid; i < ncand; i += kTopkThreads) {
+                const uint32_t u = cand_all[i];
+                if ((u & mask) == prefix) atomicAdd(&S.hist[(u >> shift) & dmask], 1u);
+            }
+            __syncthreads();
+        } else {
+            for (int i = tid; i < m; i += kTopkThreads) {
+                const uint32_t u = srow[i];
+                if ((u & mask) == prefix && bin_of(u) == b1)
+                    atomicAdd(&S.hist[(u >> shift) & dmask], 1u);
+            }
+            cluster_hist();
+        }
+        const uint32_t* h = use_cand ? S.hist : CS.hist_all;
+        if (pass < 2)
+            find_bin<2048>(S, krem, h);
+        else
+            find_bin<1024>(S, krem, h);
+        prefix |= S.bin << shift;
+        mask |= dmask << shift;
+        krem -= S.above;
+        __syncthreads();
+    }
+    const uint32_t T = prefix;
+
+    // ---- C: counts of this segment, offsets from the segments before it
+    const int wseg = ((m + kTopkWarps - 1) / kTopkWarps + 31) / 32 * 32;
+    const int sb = warp * wseg, se = min(m, sb + wseg);
+    uint32_t cg = 0, ce = 0;
+    for (int base = sb; base < se; base += 32) {
+        const int i = base + lane;
+        const bool in = i < se;
+        const uint32_t u = in ? srow[i] : 0u;
+        cg += __popc(__ballot_sync(0xffffffffu, in && u > T));
+        ce += __popc(__ballot_sync(0xffffffffu, in && u == T));
+    }
+    if (lane == 0) {
+        S.wcnt[0][warp] = cg;
+        S.wcnt[1][warp] = ce;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        uint32_t a = 0, b = 0;
+        for (int w = 0; w < kTopkWarps; ++w) {
+            a += S.wcnt[0][w];
+            b += S.wcnt[1][w];
+        }
+        CS.seg_cg = a;
+        CS.seg_ce = b;
+    }
+    cluster_sync_all();
+    uint32_t G = 0, E = 0;
+    for (uint32_t q = 0; q < rank; ++q) {
+        G += dsmem_ld(dsmem_addr(&CS.seg_cg, q));
+        E += dsmem_ld(dsmem_addr(&CS.seg_ce, q));
+    }
+#pragma unroll
+    for (int w = 0; w < kTopkWarps; ++w)
+        if (w < warp) {
+            G += S.wcnt[0][w];
+            E += S.wcnt[1][w];
+        }
+    const unsigned lt = (1u << lane) - 1u;
+    for (int base = sb; base < se; base += 32) {
+        const int i = base + lane;
+        const bool in = i < se;
+        const uint32_t u = in ? srow[i] : 0u;
+        const bool gt = in && u > T, eq = in && u == T;
+        const unsigned bg = __ballot_sync(0xffffffffu, gt);
+        const unsigned be = __ballot_sync(0xffffffffu, eq);
+        const uint32_t g_before = G + __popc(bg & lt);
+        const uint32_t e_before = E + __popc(be & lt);
+        if (gt)
+            o[g_before + (e_before < krem ? e_before : krem)] = s0 + i;
+        else if (eq && e_before < krem)
+            o[g_before + e_before] = s0 + i;
+        G += __popc(bg);
+        E += __popc(be);
+    }
+    cluster_sync_all();  // no CTA leaves while another may still read its shared memory
+}
+
+static int launch_topk_cluster(ic_ctx* ctx, const float* scores, int64_t ld, int rows, int k,
+                               int causal_base, const int32_t* row_len, int max_len,
+                               int32_t* idx_out, int64_t ld_out, cudaStream_t stream) {
+    const int seg_cap = ((max_len + kClusterCtas - 1) / kClusterCtas + 3) / 4 * 4;
+    const int smem = (seg_cap + kCandCap) * 4;
+    cudaError_t e = cudaFuncSetAttribute(k_topk_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         smem);
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaFuncSetAttribute(topk_cluster)");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(kClusterCtas, rows, 1);
+    cfg.blockDim = dim3(kTopkThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = kClusterCtas;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    LaunchScope ls(ctx, IC_K_TOPK, stream);
+    cudaLaunchKernelEx(&cfg, k_topk_cluster, scores, static_cast<long long>(ld), k, row_len,
+                       causal_base, idx_out, static_cast<long long>(ld_out), seg_cap);
+    e = ls.done();
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "topk_cluster launch");
+    return IC_OK;
+}
+
 int launch_topk(ic_ctx* ctx, const float* scores, int64_t ld, int rows, int k, int causal_base,
                 const int32_t* row_len, int max_len, int32_t* idx_out, int64_t ld_out,
                 cudaStream_t stream) {
     if (rows <= 0) return IC_OK;
+    // Few long rows (decode): a cluster of CTAs per row keeps many SMs busy.
+    if (row_len != nullptr && static_cast<long long>(rows) * kClusterCtas <= 4LL * ctx->num_sms &&
+        max_len > 16384 && max_len <= kClusterCtas * 45000)
+        return launch_topk_cluster(ctx, scores, ld, rows, k, causal_base, row_len, max_len, idx_out,
+                                   ld_out, stream);
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e = cudaFuncSetAttribute(k_topk<true>,

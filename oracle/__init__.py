@@ -42,6 +42,9 @@ def lib():
         L.oracle_pattern_uniform.argtypes = [ctypes.c_int, ctypes.c_int, ctypes.c_char_p]
         L.oracle_index_scores.argtypes = [_f32p, _f32p, _f32p, ctypes.c_int, ctypes.c_int,
                                           ctypes.c_int, _i32p, ctypes.c_int, _f64p, ctypes.c_int64]
+        L.oracle_index_scores_at.argtypes = [_f32p, _f32p, _f32p, ctypes.c_int, ctypes.c_int,
+                                             ctypes.c_int, _i32p, ctypes.c_int, _f64p,
+                                             ctypes.c_int64]
         L.oracle_e4m3_to_double.argtypes = [ctypes.c_uint8]
         L.oracle_e4m3_to_double.restype = ctypes.c_double
         L.oracle_decode_scores.argtypes = [_f32p, _f32p, _u8p, _f32p, ctypes.c_int, ctypes.c_int,
@@ -114,6 +117,23 @@ def index_scores(q, k, w, rows=None):
     return out
 
 
+def index_scores_at(q_rows, w_rows, k, positions):
+    """Scores of sampled rows given compactly: q_rows [R, H, d] and w_rows
+    [R, H] belong to query positions `positions` [R]; k is [L, d].  Returns
+    float64 [R, max(positions)+1] with NaN where s > t."""
+    q_rows = _c(q_rows, np.float32)
+    w_rows = _c(w_rows, np.float32)
+    k = _c(k, np.float32)
+    pos = _c(positions, np.int32)
+    R, H, d = q_rows.shape
+    L = k.shape[0]
+    width = int(pos.max()) + 1 if len(pos) else 0
+    out = np.full((R, width), np.nan, dtype=np.float64)
+    lib().oracle_index_scores_at(_p(q_rows, _f32p), _p(w_rows, _f32p), _p(k, _f32p), L, H, d,
+                                 _p(pos, _i32p), R, _p(out, _f64p), width)
+    return out
+
+
 def e4m3_to_float64(b: np.ndarray) -> np.ndarray:
     b = np.asarray(b, dtype=np.uint8)
     f = lib().oracle_e4m3_to_double
@@ -165,10 +185,22 @@ def index_topk(q, k, w, topk: int, rows=None) -> np.ndarray:
 # --------------------------------------------------------------------------
 # Sparse attention (reading-notes page §3)
 # --------------------------------------------------------------------------
-def sparse_attn(Q, K, V, idx, rows=None, scale=None, rows_per_seq=0):
+def sparse_attn(Q, K, V, idx, rows=None, scale=None, rows_per_seq=0, q_is_rows=False):
     """o[r, h] for the requested rows.  Q: [R, Hq, d] (indexed by row id),
     K, V: [S, d] (one sequence) or [B, S, d] with rows_per_seq rows per
-    sequence; idx: [nrows, k] index rows matching ``rows``.  float64 out."""
+    sequence; idx: [nrows, k] index rows matching ``rows``.  With
+    q_is_rows, Q holds only the requested rows, in order.  float64 out."""
+    if q_is_rows:
+        # attention of row r depends on its own query only: evaluate each
+        # requested row as row 0 of a one-row problem over the same K/V
+        Q = _c(Q, np.float32)
+        out = np.empty((Q.shape[0],) + Q.shape[1:], dtype=np.float64)
+        seqs = np.zeros(len(rows), np.int64) if rows_per_seq <= 0 else np.asarray(rows) // rows_per_seq
+        for r in range(Q.shape[0]):
+            Kr = K if K.ndim == 2 else K[seqs[r]]
+            Vr = V if V.ndim == 2 else V[seqs[r]]
+            out[r] = sparse_attn(Q[r:r + 1], Kr, Vr, np.asarray(idx)[r:r + 1], scale=scale)[0]
+        return out
     Q = _c(Q, np.float32)
     K = _c(K, np.float32)
     V = _c(V, np.float32)

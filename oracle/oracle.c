@@ -111,6 +111,24 @@ void oracle_index_scores(const float *q, const float *k, const float *w, int L, 
     }
 }
 
+/* Same scores for sampled rows whose query tensors are passed compactly:
+ * row r has position pos[r], query q_rows[r] ([H, d]) and weights
+ * w_rows[r] ([H]); keys k are the whole [L, d] tensor. */
+void oracle_index_scores_at(const float *q_rows, const float *w_rows, const float *k, int L, int H,
+                            int d, const int32_t *pos, int nrows, double *out, int64_t ld)
+{
+    int r;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (r = 0; r < nrows; ++r) {
+        int t = pos[r];
+        if (t < 0 || t >= L)
+            continue;
+        for (int s = 0; s <= t; ++s)
+            out[(size_t)r * ld + s] =
+                score_one(q_rows + (size_t)r * H * d, k + (size_t)s * d, w_rows + (size_t)r * H, H, d);
+    }
+}
+
 /* ------------------------------------------------------------------------
  * OCP FP8 E4M3 decode (1 sign, 4 exponent bits with bias 7, 3 mantissa
  * bits; exponent 0 is subnormal; S.1111.111 is NaN; no infinities).

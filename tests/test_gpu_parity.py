@@ -320,3 +320,24 @@ def test_argument_errors(ic, ctx):
         ic.ic_index_fp(ctx, q3, k, w3, 16, idx)
     assert e.value.code == ic.IC_ERR_UNSUPPORTED
     ctx.sync_status()
+
+
+@pytest.mark.parametrize("integer", [True, False])
+def test_topk_cluster_rows(ic, ctx, integer):
+    """Few long rows with explicit lengths take the cluster kernel (8 CTAs
+    per row sharing histograms and candidates through distributed shared
+    memory); integer scores force the massive-tie fallback."""
+    gen = torch.Generator().manual_seed(11 + integer)
+    B, ld = 5, 100032
+    if integer:
+        sc = torch.randint(-4, 5, (B, ld), generator=gen).float() * 0.5
+    else:
+        sc = torch.randn((B, ld), generator=gen)
+    lens = torch.tensor([100000, 16385, 2049, 99999, 77777], dtype=torch.int32)
+    idx = torch.empty((B, 2048), dtype=torch.int32, device="cuda")
+    ic.ic_topk(ctx, sc.cuda(), 2048, idx, row_len=lens.cuda(), ld=ld)
+    ctx.sync_status()
+    got = idx.cpu().numpy()
+    for b in range(B):
+        n = int(lens[b])
+        assert got[b].tolist() == oracle.topk_row(sc[b, :n].numpy().astype(np.float64), 2048).tolist(), b
