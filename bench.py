@@ -203,16 +203,30 @@ def run_ours(args, rank, world, local_rank):
                                "flop_per_launch": 2 * cfg.H_I * cfg.d_I * pairs_launch}
     if att_k["launches"]:
         avg_ms = att_k["ms"] / att_k["launches"]
-        # algorithmic bytes per launch: the k gathered K and V rows per query
-        # row plus the Q row read and the output row written
-        bytes_launch = L * (k * 2 * cfg.d * 2 + 2 * cfg.Hq * cfg.d * 2)
+        # algorithmic bytes per launch: the min(t+1, k) gathered K and V rows
+        # of each query row t, plus its Q row read and output row written
+        keys = sum(min(t + 1, k) for t in range(L))
+        bytes_launch = keys * 2 * cfg.d * 2 + L * 2 * cfg.Hq * cfg.d * 2
         gbs = bytes_launch / (avg_ms / 1e3) / 1e9
         roof["sparse_attn"] = {"bound": "hbm", "achieved": round(gbs, 1),
                                "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                               "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                               "frac": round(gbs / peaks["hbm_gbs"], 4),
+                               "traffic": ATTN_PREFILL_DRAM_BYTES,
                                "peak_kind": "HBM copy, " + peak_src,
                                "avg_launch_ms": round(avg_ms, 4), "bytes_per_launch": bytes_launch,
-                               "note": "gathered rows mostly hit L2 (8 MB K/V per layer)"}
+                               "note": "the layer's K/V (8 MB) stays in L2: the gathered rows are "
+                                       "served from L2, so the bound is the L2 random-row gather "
+                                       "rate (see l2_gather_ceiling), not HBM"}
+        ceiling = measure_gather_ceiling(cache, layers[-1], L, k, stream)
+        if ceiling:
+            roof["sparse_attn"]["l2_gather_ceiling_gbs"] = ceiling["achieved_gbs"]
+            roof["sparse_attn"]["frac_of_l2_gather_ceiling"] = round(
+                gbs / ceiling["achieved_gbs"], 4)
+            extra_ceiling = ceiling
+        else:
+            extra_ceiling = None
+    else:
+        extra_ceiling = None
     dominant = max(("index_score", "sparse_attn"), key=lambda n: ktimes[n]["ms"])
     roofline = dict(roof.get(dominant, {}))
     roofline["kernel"] = dominant
@@ -225,6 +239,7 @@ def run_ours(args, rank, world, local_rank):
         "stack_prefill_ms": round(ms_per_step, 4),
         "step_ms": [round(x, 4) for x in step_ms],
         "roofline_all": roof,
+        "l2_gather_ceiling": extra_ceiling,
     }
 
     # ------------------------------------------------ e2e through the C ABI with host buffers
@@ -272,6 +287,37 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0:
         print(json.dumps(line), flush=True)
     ctx.close()
+
+
+# DRAM traffic per launch of the prefill attention kernel from its ncu
+# capture (profiles/sparse_attn_prefill_L16384.md); None until measured for
+# the current kernel.
+ATTN_PREFILL_DRAM_BYTES = 209978624 + 51622912
+
+
+def measure_gather_ceiling(cache, lay, L, k, stream):
+    """Time the library's gather probe (the attention's K/V row gather alone,
+    no compute) over the fully populated index rows t >= k of this step's
+    cache: the random-row gather ceiling that bounds attention when K/V sit
+    in L2.  Best of 3, after one warm-up."""
+    from cross_layer_top_b200 import indexcache as ic
+    if L <= k:
+        return None
+    idx = cache[k:]
+    best = None
+    for ctas in (2, 3):
+        ic.ic_probe_gather(lay["K"], lay["V"], idx, ctas_per_sm=ctas)
+        for _ in range(3):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            ic.ic_probe_gather(lay["K"], lay["V"], idx, ctas_per_sm=ctas)
+            b.record(stream)
+            b.synchronize()
+            ms = a.elapsed_time(b)
+            best = ms if best is None else min(best, ms)
+    nbytes = (L - k) * k * 2 * lay["K"].shape[-1] * 2
+    return {"achieved_gbs": round(nbytes / (best / 1e3) / 1e9, 1), "ms": best, "bytes": nbytes,
+            "what": "cp.async gather of the same K/V rows (index rows t >= k), no compute"}
 
 
 def run_e2e(args, ctx, pat, dims, cfg, layers, cache, world, pairs_step, stream):

@@ -35,7 +35,7 @@ def sources():
 
 def headers():
     hs = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".h", ".cuh"))]
-    return hs + [os.path.join(INCLUDE, "indexcache.h")]
+    return hs + [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
 
 
 def _compile(src: str, verbose_ptxas: bool) -> str:

@@ -1,0 +1,75 @@
+// Measurement aid (include/indexcache_probe.h): the K/V row gather of the
+// sparse-attention kernel alone, to measure the random-row gather ceiling
+// that bounds attention when K/V sit in L2.  Not part of the method.
+#include "../../include/indexcache_probe.h"
+#include "ic_device.cuh"
+#include "ic_internal.h"
+
+namespace ic {
+
+constexpr int kProbeWarps = 4;
+constexpr int kProbeStages = 2;
+constexpr int kProbeChunk = 16 * 256 * 2;  // 16 rows of K and of V (d = 128)
+
+__global__ void __launch_bounds__(kProbeWarps * 32)
+    k_probe_gather(const __nv_bfloat16* __restrict__ K, const __nv_bfloat16* __restrict__ V,
+                   const int32_t* __restrict__ idx, int rows, int k, unsigned* __restrict__ sink) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const uint32_t base = smem_u32(smem) + warp * kProbeStages * kProbeChunk;
+    const int piece = lane & 15, prow = lane >> 4;
+    const int nch = k / (16 * kProbeWarps);  // chunks per warp per row
+    unsigned acc = 0;
+    for (int r = blockIdx.x; r < rows; r += gridDim.x) {
+        const int32_t* ir = idx + static_cast<long long>(r) * k;
+        auto issue = [&](int j) {
+            if (j < nch) {
+                const int c0 = (warp + j * kProbeWarps) * 16;
+                const uint32_t st = base + (j % kProbeStages) * kProbeChunk;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const int row = prow + 2 * i;
+                    const int s = __ldg(ir + c0 + row);
+                    const uint32_t off = static_cast<uint32_t>(row * 256 + ((piece ^ (row & 7)) << 4));
+                    cp_async16(st + off, K + static_cast<long long>(s) * 128 + piece * 8, true);
+                    cp_async16(st + 4096 + off, V + static_cast<long long>(s) * 128 + piece * 8, true);
+                }
+            }
+            cp_async_commit();
+        };
+        issue(0);
+        for (int j = 0; j < nch; ++j) {
+            cp_async_wait<0>();
+            __syncwarp();
+            acc += *reinterpret_cast<const volatile unsigned*>(
+                smem + warp * kProbeStages * kProbeChunk + (j % kProbeStages) * kProbeChunk + lane * 4);
+            __syncwarp();
+            issue(j + 1);
+        }
+        cp_async_wait<0>();
+    }
+    if (acc == 0x9e3779b9u) sink[0] = acc;  // keeps the loads observable
+}
+
+}  // namespace ic
+
+extern "C" int ic_probe_gather(const void* K, const void* V, const int32_t* idx, int rows, int k,
+                               int d, int ctas_per_sm, void* stream) {
+    if (!K || !V || !idx) return ic::fail(nullptr, IC_ERR_INVALID_ARG, "probe_gather: NULL");
+    if (d != 128 || k <= 0 || k % 64 != 0 || rows <= 0 || ctas_per_sm < 1 || ctas_per_sm > 3)
+        return ic::fail(nullptr, IC_ERR_UNSUPPORTED, "probe_gather: d=%d k=%d rows=%d", d, k, rows);
+    int dev = 0, sms = 148;
+    cudaGetDevice(&dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const int smem = ic::kProbeWarps * ic::kProbeStages * ic::kProbeChunk;
+    cudaError_t e = cudaFuncSetAttribute(ic::k_probe_gather,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return ic::cuda_fail(nullptr, e, "probe_gather attribute");
+    const int grid = sms * ctas_per_sm < rows ? sms * ctas_per_sm : rows;
+    ic::k_probe_gather<<<grid, ic::kProbeWarps * 32, smem, reinterpret_cast<cudaStream_t>(stream)>>>(
+        static_cast<const __nv_bfloat16*>(K), static_cast<const __nv_bfloat16*>(V), idx, rows, k,
+        nullptr);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return ic::cuda_fail(nullptr, e, "probe_gather launch");
+    return IC_OK;
+}

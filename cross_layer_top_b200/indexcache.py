@@ -79,6 +79,7 @@ _SIGS = {
     "ic_index_score_decode": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _i64, _vp], _i),
     "ic_index_fp_decode": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp], _i),
     "ic_index_fp_decode_noalloc": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp], _i),
+    "ic_probe_gather": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp], _i),
     "ic_sparse_attn": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64, _i, _f, _vp, _vp], _i),
     "ic_run_stack": ([_vp, _vp, ctypes.POINTER(ic_layer_io), ctypes.POINTER(ic_stack_dims), _vp,
                       _vp], _i),
@@ -293,6 +294,13 @@ def ic_sparse_attn(ctx: Context, Q, K, V, idx, out, rows_per_seq: int = 0, kv_se
     _check(_lib.ic_sparse_attn(ctx.handle, _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), rows, Hq, d, k,
                                rows_per_seq, kv_seq_stride, kv_len, scale, _ptr(out),
                                _stream(stream)), ctx)
+
+
+def ic_probe_gather(K, V, idx, ctas_per_sm: int = 2, stream=None):
+    """Measurement aid: the attention's K/V row gather alone (no compute)."""
+    rows, k = idx.shape
+    _check(_lib.ic_probe_gather(_ptr(K), _ptr(V), _ptr(idx), rows, k, K.shape[-1], ctas_per_sm,
+                                _stream(stream)))
 
 
 def make_stack_layers(layers, mode=IC_PREFILL):
