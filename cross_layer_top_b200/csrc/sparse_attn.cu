@@ -158,13 +158,14 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
     // rows g = lane/4 and g + 8
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
 
+    // every stage starts filled; the stage of chunk j is refilled (chunk
+    // j + STAGES) as soon as chunk j has been consumed
 #pragma unroll
-    for (int j = 0; j < S::STAGES - 1; ++j) issue(j);
+    for (int j = 0; j < S::STAGES; ++j) issue(j);
     for (int j = 0; j < my_n; ++j) {
         const int st = j % S::STAGES;
-        cp_async_wait<S::STAGES - 2>();  // chunk j has landed
+        cp_async_wait<S::STAGES - 1>();  // chunk j has landed
         __syncwarp();
-        issue(j + S::STAGES - 1);  // into the stage of chunk j-1, whose reads are done
         const uint32_t kb = wst + st * S::STAGE_BYTES;
         const uint32_t vb = kb + S::CH * S::ROWP;
         const int c0 = (warp + j * S::WARPS) * S::CH;
@@ -246,6 +247,8 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
             mma_bf16_16816(o[2 * dn], pa, b0, b1);
             mma_bf16_16816(o[2 * dn + 1], pa, b2, b3);
         }
+        __syncwarp();              // every lane is done reading stage st
+        issue(j + S::STAGES);      // refill it
     }
     cp_async_wait<0>();
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
@@ -313,27 +316,44 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
     if (!*s_flag) return;
     __threadfence();
     const float* part_row = part + static_cast<long long>(r) * nsplit * (16 * D + 32);
-    float* sf = mO;                // [nsplit][16] factors (merge buffer is free again)
-    float* sinv = mO + 64 * 16;    // [16]
+    constexpr int PSTRIDE = 16 * D + 32;
+    float* sML = mO;                 // [nsplit][32]: m[16], l[16] of every split
+    float* sf = mO + 64 * 32;        // [nsplit][16] merge factors
+    float* sinv = sf + 64 * 16;      // [16]
+    // one parallel round trip for every split's (m, l)
+    for (int i = tid; i < nsplit * 32; i += S::THREADS)
+        sML[i] = __ldcg(part_row + (i >> 5) * PSTRIDE + 16 * D + (i & 31));
+    __syncthreads();
     if (tid < 16) {
         const int h = tid;
         float M = -INFINITY;
-        for (int q = 0; q < nsplit; ++q) M = fmaxf(M, __ldcg(part_row + q * (16 * D + 32) + 16 * D + h));
+        for (int q = 0; q < nsplit; ++q) M = fmaxf(M, sML[q * 32 + h]);
         float L = 0.f;
         for (int q = 0; q < nsplit; ++q) {
-            const float* ps = part_row + q * (16 * D + 32);
-            const float f = M == -INFINITY ? 0.f : ex2_approx(__ldcg(ps + 16 * D + h) - M);
+            const float f = M == -INFINITY ? 0.f : ex2_approx(sML[q * 32 + h] - M);
             sf[q * 16 + h] = f;
-            L += __ldcg(ps + 16 * D + 16 + h) * f;
+            L += sML[q * 32 + 16 + h] * f;
         }
         sinv[h] = L > 0.f ? 1.f / L : 0.f;
     }
     __syncthreads();
-    for (int e = tid; e < Hq * D; e += S::THREADS) {
-        const int h = e / D, dd = e % D;
-        float acc = 0.f;
-        for (int q = 0; q < nsplit; ++q) acc += __ldcg(part_row + q * (16 * D + 32) + h * D + dd) * sf[q * 16 + h];
-        out[(static_cast<long long>(r) * Hq + h) * D + dd] = __float2bfloat16_rn(acc * sinv[h]);
+    // O: float4 columns, the split loop unrolled so its loads overlap
+    for (int e = tid; e < Hq * (D / 4); e += S::THREADS) {
+        const int h = e / (D / 4), d4 = (e % (D / 4)) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int q = 0; q < nsplit; ++q) {
+            const float4 v = __ldcg(reinterpret_cast<const float4*>(part_row + q * PSTRIDE + h * D + d4));
+            const float f = sf[q * 16 + h];
+            acc.x = fmaf(v.x, f, acc.x);
+            acc.y = fmaf(v.y, f, acc.y);
+            acc.z = fmaf(v.z, f, acc.z);
+            acc.w = fmaf(v.w, f, acc.w);
+        }
+        const float iv = sinv[h];
+        __nv_bfloat16* op = out + (static_cast<long long>(r) * Hq + h) * D + d4;
+        *reinterpret_cast<uint2*>(op) = make_uint2(pack_bf16x2(acc.x * iv, acc.y * iv),
+                                                   pack_bf16x2(acc.z * iv, acc.w * iv));
     }
     if (tid == 0) row_done[r] = 0;
 }
