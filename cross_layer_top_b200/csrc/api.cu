@@ -108,7 +108,7 @@ int make_tmap_bf16_2d(ic_ctx* ctx, CUtensorMap* map, const void* base, uint64_t 
 }
 
 int make_tmap_u8_2d(ic_ctx* ctx, CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                    uint32_t box_cols, uint32_t box_rows) {
+                    uint32_t box_cols, uint32_t box_rows, bool swizzle128) {
     EncodeTiledFn fn = encode_tiled_fn();
     if (!fn) return fail(ctx, IC_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
     const cuuint64_t gdim[2] = {cols, rows};
@@ -116,7 +116,8 @@ int make_tmap_u8_2d(ic_ctx* ctx, CUtensorMap* map, const void* base, uint64_t ro
     const cuuint32_t box[2] = {box_cols, box_rows};
     const cuuint32_t estride[2] = {1, 1};
     CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<void*>(base), gdim, gstride,
-                    box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                    box, estride, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                    swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                     CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS)
         return fail(ctx, IC_ERR_CUDA, "cuTensorMapEncodeTiled(u8 %llux%llu) failed: %d",

@@ -67,9 +67,10 @@ EncodeTiledFn encode_tiled_fn();
 // box of {64 columns, box_rows rows} and the 128-byte swizzle.
 int make_tmap_bf16_2d(ic_ctx* ctx, CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
                       uint32_t box_rows);
-// Same for an 8-bit tensor, box {128 columns, box_rows rows}, no swizzle.
+// Same for an 8-bit tensor, box {box_cols columns, box_rows rows}, with the
+// 128-byte swizzle (box_cols = 128) or none.
 int make_tmap_u8_2d(ic_ctx* ctx, CUtensorMap* map, const void* base, uint64_t rows, uint64_t cols,
-                    uint32_t box_cols, uint32_t box_rows);
+                    uint32_t box_cols, uint32_t box_rows, bool swizzle128);
 
 // ----------------------------------------------------------------- launchers
 int launch_index_score_prefill(ic_ctx* ctx, const void* qI, const void* kI, const void* w, int L,

@@ -8,21 +8,32 @@
 // cache ("IndexCache：…", §10.1); the indexer runs in FP8 ("IndexCache:
 // Accelerating Sparse Attention via Cross-Layer Index Reuse", §2.1).
 //
-// Design (sm_100a), one persistent CTA per SM, HBM-bound by construction:
-//  * warp 0 (TMA): streams raw e4m3 key tiles (128 keys x 128 B, one
-//    contiguous 16 KB block each, so one bulk copy) through a 5-deep ring,
-//    and the sequence's q rows (bf16, 128-byte swizzle, a tensor copy)
-//    when the sequence changes;
-//  * warps 4..11 (convert): widen each e4m3 tile to bf16 — exact, every e4m3
-//    value is a bf16 value — and write it in the K-major 128-byte-swizzle
-//    layout the tensor core reads, then fence the async proxy;
-//  * warp 1 (MMA): UMMA M=128 keys x N=H_I heads x K=128, fp32 in TMEM, four
-//    accumulators in flight;
-//  * warps 12..15 (epilogue): the thread owning TMEM lane s applies ReLU,
-//    the w weights, the head sum and the per-token scale, and stores I[b,s].
-// Each CTA scans a contiguous range of (sequence, key tile) pairs, so q is
-// reloaded only when its range crosses into the next sequence.  All waits
-// are bounded.
+// Design (sm_100a), one persistent CTA per SM, HBM-bound by construction.
+// The e4m3 key tile goes from HBM to the tensor core untouched: TMA writes
+// it in the 128-byte-swizzle K-major layout and UMMA kind::f8f6f4 reads it
+// as the A operand.  The bf16 query is carried exactly by two e4m3 terms:
+// with x = q * 2^s (2^s puts max|x| in [2^7, 2^8)), hi = e4m3(x) and
+// lo = e4m3(x - hi) give hi + lo = x exactly for every |x| >= 2^-2 (the
+// remainder x - hi is a multiple of x's bf16 ulp no larger than 8 ulps, so
+// it has at most four significant bits), and within 2^-10 (2^-17 of max|x|)
+// below that.  hi and lo are stacked as the 2 H_I rows of one B operand
+// (an M = 128 UMMA costs the same for any N <= 64, so N = 2 H_I is free):
+// D[s,j] = k_s . hi_j and D[s,H_I+j] = k_s . lo_j, added in the epilogue.
+//  * warp 0 (TMA): streams key tiles (256 keys x 128 B, one tensor copy)
+//    through a 5-deep ring; rows past the end of the cache read as zero and
+//    are never stored;
+//  * warps 4..7 (query): when the CTA's range enters a new sequence, read
+//    its q, find 2^s and write hi / lo (double-buffered, swizzled);
+//  * warp 1 (MMA): per tile, 4 UMMAs (M = 128 keys, N = 2 H_I, K = 32) for
+//    each 128-key half into its own accumulator, fp32 in TMEM; one commit
+//    per tile for the stage and one for the accumulator pair (the per-tile
+//    fixed costs are what bound the issuer, so tiles are 256 keys);
+//  * warps 8..15 (epilogue; warps 8..11 take the first half of each tile,
+//    12..15 the second): the thread owning TMEM lane s adds hi and lo,
+//    applies ReLU, the w weights, the head sum, 2^-s and the per-token
+//    scale, and stores I[b,s].
+// Each CTA scans a contiguous range of (sequence, key tile) pairs.  All
+// waits are bounded.
 #include "ic_device.cuh"
 #include "ic_internal.h"
 
@@ -30,78 +41,102 @@ namespace ic {
 
 template <int H_I>
 struct DecodeShape {
-    static constexpr int BM = 128;          // keys per tile
-    static constexpr int DI = 128;          // d_I
-    static constexpr int RAW = BM * DI;     // e4m3 tile bytes
-    static constexpr int RAW_ST = 5;
-    static constexpr int A_ATOM = BM * 128; // bf16 64-column slice
-    static constexpr int A_STAGE = 2 * A_ATOM;
-    static constexpr int A_ST = 3;
-    static constexpr int B_ATOM = H_I * 128;
-    static constexpr int B_BYTES = 2 * B_ATOM;
-    static constexpr int NACC = 4;
-    static constexpr int TMEM_COLS = NACC * H_I < 32 ? 32 : NACC * H_I;
-    static constexpr int W_BYTES = 4 * H_I * 4;  // per epilogue warp
-    static constexpr int SC_RING = 4;             // scale prefetch depth (tiles)
+    static constexpr int BM = 256;          // keys per tile (two UMMA halves of 128)
+    static constexpr int DI = 128;          // d_I (bytes per e4m3 key row)
+    static constexpr int A_BYTES = BM * DI; // one key tile
+    static constexpr int A_HALF = 128 * DI;
+    static constexpr int A_ST = 5;
+    static constexpr int B_HALF = H_I * DI; // hi or lo: H_I rows of 128 e4m3
+    static constexpr int B_BUF = 2 * B_HALF;
+    static constexpr int ACC_COLS = 2 * H_I;  // hi heads, then lo heads
+    static constexpr int TMEM_COLS = 512;
+    static constexpr int NACC = TMEM_COLS / (2 * ACC_COLS);  // accumulator pairs (one per tile)
+    // per-sequence ring (query warps -> epilogue): tag b, 2^-s, w[b,:] in fp32
+    static constexpr int SEQ_RING = 8;
+    static constexpr int SEQ_BYTES = 16 + 4 * H_I;
+    static constexpr int W_BYTES = SEQ_RING * SEQ_BYTES;
+    static constexpr int SC_RING = 8;       // scale prefetch depth (tiles)
     static constexpr int SC_BYTES = SC_RING * BM * 4;
-    static constexpr int BAR_BYTES = 256;
+    static constexpr int QRED_BYTES = 32;   // [2][4] warp maxima of |q|
+    static constexpr int BAR_BYTES = 512;
     static constexpr int OFF_A = 0;
-    static constexpr int OFF_B = OFF_A + A_ST * A_STAGE;
-    static constexpr int OFF_RAW = OFF_B + B_BYTES;
-    static constexpr int OFF_W = OFF_RAW + RAW_ST * RAW;
+    static constexpr int OFF_B = OFF_A + A_ST * A_BYTES;
+    static constexpr int OFF_W = OFF_B + 2 * B_BUF;
     static constexpr int OFF_SC = OFF_W + W_BYTES;
-    static constexpr int OFF_BAR = OFF_SC + SC_BYTES;
+    static constexpr int OFF_QRED = OFF_SC + SC_BYTES;
+    static constexpr int OFF_BAR = OFF_QRED + QRED_BYTES;
     static constexpr int SMEM = OFF_BAR + BAR_BYTES;
     static_assert(SMEM <= 232448, "shared memory budget");
+    static_assert(NACC >= 2, "TMEM allocation");
+    static_assert(OFF_B % 1024 == 0 && B_HALF % 1024 == 0, "swizzle atoms need 1024-B alignment");
 };
 
-// Two e4m3 bytes (low bytes of the two 16-bit lanes of y) -> bf16x2, exactly.
-// The e4m3 sign goes to bit 15 and its 7 exponent/mantissa bits to bits
-// 10..4, i.e. a bf16 whose exponent field is the e4m3 exponent field
-// unbiased: value * 2^-120 (for an e4m3 subnormal, the matching bf16
-// subnormal).  One bf16x2 multiply by 2^120 restores the value; it is exact
-// (a power-of-two scaling into the normal range).  The e4m3 NaN bytes
-// (0x7F, 0xFF) are not NaN afterwards (+-480); caches hold none.
-__device__ __forceinline__ uint32_t e4m3x2_lanes_to_bf16x2(uint32_t y) {
-    // (low 7 bits << 4) | (sign << 8) == (y << 4) + sign * (256 - 16)
-    const uint32_t bits = (y & 0x00800080u) * 240u + (y << 4);
-    const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162*>(&bits);
-    const __nv_bfloat162 s = __halves2bfloat162(__ushort_as_bfloat16(0x7B80),
-                                                __ushort_as_bfloat16(0x7B80));  // 2^120
-    const __nv_bfloat162 r = __hmul2(v, s);
-    return *reinterpret_cast<const uint32_t*>(&r);
+// e4m3 pair <-> float pair.  The low byte is the first element.
+__device__ __forceinline__ uint32_t e4m3x2_of(float first, float second) {
+    unsigned short r;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(second), "f"(first));
+    return r;
+}
+__device__ __forceinline__ float2 float2_of_e4m3x2(uint32_t pair16) {
+    uint32_t h;
+    asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(static_cast<unsigned short>(pair16)));
+    return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
 
-// 16 e4m3 values (one 16-byte chunk) -> 16 bf16 values, exactly.
-__device__ __forceinline__ void e4m3x16_to_bf16(const uint4 in, uint4& lo, uint4& hi) {
-    const uint32_t w[4] = {in.x, in.y, in.z, in.w};
-    uint32_t o[8];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        o[2 * i] = e4m3x2_lanes_to_bf16x2(__byte_perm(w[i], 0u, 0x4140));      // bytes 0, 1
-        o[2 * i + 1] = e4m3x2_lanes_to_bf16x2(__byte_perm(w[i], 0u, 0x4342));  // bytes 2, 3
-    }
-    lo = make_uint4(o[0], o[1], o[2], o[3]);
-    hi = make_uint4(o[4], o[5], o[6], o[7]);
+// Packed fp32 pairs (two lanes of one 64-bit register): one add / fma
+// instruction for two heads.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+    uint64_t r;
+    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+    return r;
+}
+__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
+    float2 r;
+    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
+    return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+    uint64_t d;
+    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+    return d;
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+    uint64_t d;
+    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+    return d;
 }
 
+// The power of two 2^s that brings the largest |q| of a sequence (bf16 bit
+// pattern M of its magnitude) into [2^7, 2^8), clamped to normal floats.
+__device__ __forceinline__ int q_shift_of_max(uint32_t M) {
+    const int e = static_cast<int>((M >> 7) & 0xFF) - 127;
+    const int sh = M == 0 ? 0 : 7 - e;
+    return sh > 126 ? 126 : (sh < -126 ? -126 : sh);
+}
 // Walks a CTA's contiguous range of (sequence b, key tile j) pairs in order,
 // visiting only tiles that hold candidates (j * BM < seq_len[b]) and
 // skipping a sequence's empty tail in one step.  One division at the start,
-// none afterwards.
+// none afterwards; next() past the end stays done and reads nothing.  A
+// length above S_max counts as S_max.
 template <int BM>
 struct TileWalk {
     long long g, g_end;
-    int b, j, n, tps;
+    int b, j, n, tps, s_max;
     const int32_t* seq_len;
-    __device__ __forceinline__ void init(long long g0, long long ge, int tps_, const int32_t* sl) {
+    __device__ __forceinline__ int len(int bb) const {
+        const int v = seq_len[bb];
+        return v < s_max ? v : s_max;
+    }
+    __device__ __forceinline__ void init(long long g0, long long ge, int tps_, const int32_t* sl,
+                                         int s_max_) {
         g = g0;
         g_end = ge;
         tps = tps_;
+        s_max = s_max_;
         seq_len = sl;
         b = static_cast<int>(g0 / tps_);
         j = static_cast<int>(g0 - static_cast<long long>(b) * tps_);
-        n = g < g_end ? seq_len[b] : 0;
+        n = g < g_end ? len(b) : 0;
         settle();
     }
     __device__ __forceinline__ void settle() {
@@ -109,7 +144,7 @@ struct TileWalk {
             g += tps - j;
             ++b;
             j = 0;
-            if (g < g_end) n = seq_len[b];
+            if (g < g_end) n = len(b);
         }
     }
     __device__ __forceinline__ bool done() const { return g >= g_end; }
@@ -118,7 +153,7 @@ struct TileWalk {
         if (++j == tps) {
             j = 0;
             ++b;
-            if (g < g_end) n = seq_len[b];
+            if (g < g_end) n = len(b);
         }
         settle();
     }
@@ -126,27 +161,26 @@ struct TileWalk {
 
 template <int H_I>
 __global__ void __launch_bounds__(512, 1)
-    k_index_score_decode(const __grid_constant__ CUtensorMap tm_q,
-                         const uint8_t* __restrict__ k8,
-                         const __nv_bfloat16* __restrict__ w, const float* __restrict__ kscale,
-                         const int32_t* __restrict__ seq_len, int B, int S_max, int tps,
-                         float* __restrict__ scores, long long ld, int* __restrict__ err) {
+    k_index_score_decode(const __grid_constant__ CUtensorMap tm_k,
+                         const __nv_bfloat16* __restrict__ qg, const __nv_bfloat16* __restrict__ w,
+                         const float* __restrict__ kscale, const int32_t* __restrict__ seq_len,
+                         int B, int S_max, int tps, float* __restrict__ scores, long long ld,
+                         int* __restrict__ err) {
     using S = DecodeShape<H_I>;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t* sA = smem + S::OFF_A;
     uint8_t* sB = smem + S::OFF_B;
-    uint8_t* sRaw = smem + S::OFF_RAW;
-    float* sW = reinterpret_cast<float*>(smem + S::OFF_W);
     uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::OFF_BAR);
-    uint64_t* raw_full = bars;                  // [RAW_ST]
-    uint64_t* raw_empty = raw_full + S::RAW_ST; // [RAW_ST]
-    uint64_t* a_full = raw_empty + S::RAW_ST;   // [A_ST]
-    uint64_t* a_empty = a_full + S::A_ST;       // [A_ST]
+    uint64_t* a_full = bars;                    // [A_ST] key tile landed (TMA tx)
+    uint64_t* a_empty = a_full + S::A_ST;       // [A_ST] key tile consumed (MMA commit)
     uint64_t* acc_full = a_empty + S::A_ST;     // [NACC]
     uint64_t* acc_empty = acc_full + S::NACC;   // [NACC]
-    uint64_t* q_full = acc_empty + S::NACC;
-    uint64_t* q_empty = q_full + 1;
-    uint64_t* done_bar = q_full + 2;
+    uint64_t* q_full = acc_empty + S::NACC;     // [2] hi / lo written (query warps)
+    uint64_t* q_empty = q_full + 2;             // [2] hi / lo no longer read (MMA commit)
+    uint64_t* q_max = q_empty + 2;              // query warps' max|q| reduction
+    uint64_t* done_bar = q_max + 1;
+    uint32_t* qred = reinterpret_cast<uint32_t*>(smem + S::OFF_QRED);  // [2][4]
+    uint8_t* seq_ring = smem + S::OFF_W;
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -161,23 +195,24 @@ __global__ void __launch_bounds__(512, 1)
             *abort_flag = 1;
             atomicCAS(err, 0, kDevSmemMisaligned);
         }
-        for (int i = 0; i < S::RAW_ST; ++i) {
-            mbar_init(&raw_full[i], 1);
-            mbar_init(&raw_empty[i], 8);  // one arrival per converter warp
-        }
         for (int i = 0; i < S::A_ST; ++i) {
-            mbar_init(&a_full[i], 8);
+            mbar_init(&a_full[i], 1);
             mbar_init(&a_empty[i], 1);
         }
         for (int i = 0; i < S::NACC; ++i) {
             mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], 4);
+            mbar_init(&acc_empty[i], 8);  // every epilogue warp
         }
-        mbar_init(q_full, 1);
-        mbar_init(q_empty, 1);
+        for (int i = 0; i < 2; ++i) {
+            mbar_init(&q_full[i], 4);  // one arrival per query warp
+            mbar_init(&q_empty[i], 1);
+        }
+        mbar_init(q_max, 4);
         mbar_init(done_bar, 1);
+        for (int i = 0; i < S::SEQ_RING; ++i)
+            *reinterpret_cast<volatile int*>(seq_ring + i * S::SEQ_BYTES) = -1;
         fence_mbar_init();
-        tma_prefetch_desc(&tm_q);
+        tma_prefetch_desc(&tm_k);
     }
     if (warp == 2) {
         tmem_alloc(tmem_slot, S::TMEM_COLS);
@@ -191,150 +226,188 @@ __global__ void __launch_bounds__(512, 1)
 
     if (warp == 0 && lane == 0 && start_ok) {
         // ------------------------------------------------ TMA producer
-        int rs = 0;
-        uint32_t rph = 0, q_it = 0;
-        int last_ph[S::RAW_ST];
-#pragma unroll
-        for (int i = 0; i < S::RAW_ST; ++i) last_ph[i] = -1;
-        int q_last = -1, cur_b = -1;
+        int st = 0;
+        uint32_t ph = 0;
+        uint32_t used = 0, last_ph = 0;  // per stage: loaded at all, parity of the last load
         TileWalk<S::BM> tw;
-        for (tw.init(g_begin, g_end, tps, seq_len); !tw.done(); tw.next()) {
-            const int b = tw.b, j = tw.j;
-            if (b != cur_b) {
-                if (!mbar_wait(q_empty, (q_it & 1) ^ 1, abort_flag, err, kDevTimeoutProducer)) break;
-                mbar_arrive_expect_tx(q_full, S::B_BYTES);
-                tma_load_2d(sB, &tm_q, q_full, 0, b * H_I);
-                tma_load_2d(sB + S::B_ATOM, &tm_q, q_full, 64, b * H_I);
-                q_last = q_it & 1;
-                ++q_it;
-                cur_b = b;
-            }
-            if (!mbar_wait(&raw_empty[rs], rph ^ 1, abort_flag, err, kDevTimeoutProducer)) break;
-            // the tile's 128 key rows are one contiguous block: a single bulk
-            // copy, clamped at the end of the cache (rows past it stay stale
-            // and are never stored)
-            const long long row0 = static_cast<long long>(b) * S_max + j * S::BM;
-            const long long left = static_cast<long long>(B) * S_max - row0;
-            const uint32_t bytes = static_cast<uint32_t>(left < S::BM ? left : S::BM) * S::DI;
-            mbar_arrive_expect_tx(&raw_full[rs], bytes);
-            bulk_load(smem_u32(sRaw + rs * S::RAW), k8 + row0 * S::DI, bytes, &raw_full[rs]);
-            last_ph[rs] = static_cast<int>(rph);
-            if (++rs == S::RAW_ST) {
-                rs = 0;
-                rph ^= 1;
+        for (tw.init(g_begin, g_end, tps, seq_len, S_max); !tw.done(); tw.next()) {
+            if (!mbar_wait(&a_empty[st], ph ^ 1, abort_flag, err, kDevTimeoutProducer)) break;
+            // rows past the end of the cache are zero-filled by TMA, rows past
+            // seq_len[b] are read but never stored
+            const int row0 = tw.b * S_max + tw.j * S::BM;
+            mbar_arrive_expect_tx(&a_full[st], S::A_BYTES);
+            tma_load_2d(sA + st * S::A_BYTES, &tm_k, &a_full[st], 0, row0);
+            used |= 1u << st;
+            last_ph = (last_ph & ~(1u << st)) | (ph << st);
+            if (++st == S::A_ST) {
+                st = 0;
+                ph ^= 1;
             }
         }
-        for (int i = 0; i < S::RAW_ST; ++i)
-            if (last_ph[i] >= 0) mbar_wait_drain(&raw_full[i], static_cast<uint32_t>(last_ph[i]));
-        if (q_last >= 0) mbar_wait_drain(q_full, static_cast<uint32_t>(q_last));
+        for (int i = 0; i < S::A_ST; ++i)
+            if ((used >> i) & 1) mbar_wait_drain(&a_full[i], (last_ph >> i) & 1);
     } else if (warp == 1 && lane == 0 && start_ok) {
         // ------------------------------------------------ MMA issuer
-        constexpr uint32_t IDESC = idesc_bf16_f32(S::BM, H_I);
-        int as = 0, acc = 0;
-        uint32_t aph = 0, q_it = 0;
-        uint32_t acc_it[S::NACC] = {0, 0, 0, 0};
+        constexpr uint32_t IDESC = idesc_e4m3_f32(128, S::ACC_COLS);
+        int st = 0, acc = 0, qb = 0;
+        uint32_t ph = 0, q_it = 0;
+        uint32_t acc_ph = 0;  // bit a: parity of accumulator a's next use
         int cur_b = -1;
-        bool ok = true;
         TileWalk<S::BM> tw;
-        for (tw.init(g_begin, g_end, tps, seq_len); !tw.done() && ok; tw.next()) {
-            const int b = tw.b;
-            if (b != cur_b) {
-                if (cur_b >= 0) umma_commit(q_empty);  // previous q no longer read
-                if (!mbar_wait(q_full, q_it & 1, abort_flag, err, kDevTimeoutMma)) break;
+        for (tw.init(g_begin, g_end, tps, seq_len, S_max); !tw.done(); tw.next()) {
+            if (tw.b != cur_b) {
+                if (cur_b >= 0) umma_commit(&q_empty[qb]);  // previous hi / lo no longer read
+                qb = static_cast<int>(q_it & 1);
+                if (!mbar_wait(&q_full[qb], (q_it >> 1) & 1, abort_flag, err, kDevTimeoutMma)) break;
                 ++q_it;
-                cur_b = b;
+                cur_b = tw.b;
             }
-            if (!mbar_wait(&a_full[as], aph, abort_flag, err, kDevTimeoutMma)) break;
-            if (!mbar_wait(&acc_empty[acc], (acc_it[acc] & 1) ^ 1, abort_flag, err,
-                           kDevTimeoutMma)) {
-                ok = false;
+            if (!mbar_wait(&a_full[st], ph, abort_flag, err, kDevTimeoutMma)) break;
+            if (!mbar_wait(&acc_empty[acc], ((acc_ph >> acc) & 1) ^ 1, abort_flag, err,
+                           kDevTimeoutMma))
                 break;
-            }
             tc_fence_after();
-            const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * H_I);
+            const uint32_t d_tmem = tmem + static_cast<uint32_t>(acc * 2 * S::ACC_COLS);
+            const uint32_t a0 = smem_u32(sA + st * S::A_BYTES);
+            const uint32_t b0 = smem_u32(sB + qb * S::B_BUF);  // hi rows, then lo rows
 #pragma unroll
-            for (int k = 0; k < 2; ++k)
+            for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t ad =
-                        sdesc_k_sw128(smem_u32(sA + as * S::A_STAGE + k * S::A_ATOM + kk * 32));
-                    const uint64_t bd = sdesc_k_sw128(smem_u32(sB + k * S::B_ATOM + kk * 32));
-                    umma_bf16(d_tmem, ad, bd, IDESC, (k | kk) != 0 ? 1u : 0u);
-                }
+                for (int kk = 0; kk < 4; ++kk)
+                    umma_f8(d_tmem + hf * S::ACC_COLS, sdesc_k_sw128(a0 + hf * S::A_HALF + kk * 32),
+                            sdesc_k_sw128(b0 + kk * 32), IDESC, kk != 0 ? 1u : 0u);
             umma_commit(&acc_full[acc]);
-            umma_commit(&a_empty[as]);
-            ++acc_it[acc];
+            umma_commit(&a_empty[st]);
+            acc_ph ^= 1u << acc;
             if (++acc == S::NACC) acc = 0;
-            if (++as == S::A_ST) {
-                as = 0;
-                aph ^= 1;
+            if (++st == S::A_ST) {
+                st = 0;
+                ph ^= 1;
             }
         }
         umma_commit(done_bar);
         if (!mbar_wait_drain(done_bar, 0)) atomicCAS(err, 0, kDevTimeoutDrain);
-    } else if (warp >= 4 && warp < 12 && start_ok) {
-        // ------------------------------------------------ e4m3 -> bf16
-        const int t = threadIdx.x - 128;  // 0..255
-        int rs = 0, as = 0;
-        uint32_t rph = 0, aph = 0;
-        bool ok = true;
+    } else if (warp >= 4 && warp < 8 && start_ok) {
+        // ------------------------------------------------ query hi / lo
+        const int t = threadIdx.x - 128;  // 0..127
+        const int qw = t >> 5;
+        constexpr int NCH = H_I * 8 / 128;  // 16-element chunks per thread
+        uint32_t q_it = 0;
+        int cur_b = -1;
         TileWalk<S::BM> tw;
-        for (tw.init(g_begin, g_end, tps, seq_len); !tw.done() && ok; tw.next()) {
-            bool got = mbar_wait(&raw_full[rs], rph, abort_flag, err, kDevTimeoutEpilogue);
-            got = got && mbar_wait(&a_empty[as], aph ^ 1, abort_flag, err, kDevTimeoutEpilogue);
-            got = __all_sync(0xffffffffu, got);
-            if (!got) {
-                ok = false;
-                break;
-            }
-            const uint8_t* raw = sRaw + rs * S::RAW;
-            uint8_t* dst = sA + as * S::A_STAGE;
+        for (tw.init(g_begin, g_end, tps, seq_len, S_max); !tw.done(); tw.next()) {
+            if (tw.b == cur_b) continue;
+            cur_b = tw.b;
+            const int qb = static_cast<int>(q_it & 1);
+            const uint32_t par = q_it & 1;
+            bool ok = mbar_wait(&q_empty[qb], ((q_it >> 1) & 1) ^ 1, abort_flag, err,
+                                kDevTimeoutEpilogue);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            // chunk c = t + 128 i: head h = c >> 3, elements 16 (c & 7) .. +15
+            const uint4* qv = reinterpret_cast<const uint4*>(qg + static_cast<size_t>(cur_b) * H_I * 128);
+            uint4 v[NCH][2];
+            uint32_t mx = 0;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int c = i * 256 + t;       // 16-byte chunk id in the raw tile
-                const int row = c >> 3, c8 = c & 7;
-                const uint4 v = *reinterpret_cast<const uint4*>(raw + c * 16);
-                uint4 lo, hi;
-                e4m3x16_to_bf16(v, lo, hi);
-                uint8_t* atom = dst + (c8 >> 2) * S::A_ATOM + row * 128;
-                const int ch = 2 * (c8 & 3);
-                *reinterpret_cast<uint4*>(atom + ((ch ^ (row & 7)) << 4)) = lo;
-                *reinterpret_cast<uint4*>(atom + (((ch + 1) ^ (row & 7)) << 4)) = hi;
+            for (int i = 0; i < NCH; ++i) {
+                const int c = t + 128 * i;
+                v[i][0] = __ldg(qv + 2 * c);
+                v[i][1] = __ldg(qv + 2 * c + 1);
             }
-            // generic-proxy writes must be visible to the tensor core; one
-            // arrival per warp keeps the barriers' arrival traffic small
+            // warp 0 also fetches w[b,:] now, so its latency overlaps q's
+            float wv[(H_I + 31) / 32];
+            if (qw == 0)
+#pragma unroll
+                for (int r = 0; r < (H_I + 31) / 32; ++r)
+                    wv[r] = __bfloat162float(w[static_cast<size_t>(cur_b) * H_I + r * 32 + lane]);
+#pragma unroll
+            for (int i = 0; i < NCH; ++i)
+#pragma unroll
+                for (int u = 0; u < 2; ++u) {
+                    const uint32_t w4[4] = {v[i][u].x, v[i][u].y, v[i][u].z, v[i][u].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        mx = max(mx, max(w4[e] & 0x7FFFu, (w4[e] >> 16) & 0x7FFFu));
+                }
+            mx = __reduce_max_sync(0xffffffffu, mx);
+            if (lane == 0) {
+                qred[par * 4 + qw] = mx;
+                mbar_arrive(q_max);
+            }
+            ok = mbar_wait(q_max, par, abort_flag, err, kDevTimeoutEpilogue);
+            if (!__all_sync(0xffffffffu, ok)) break;
+            uint32_t M = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) M = max(M, qred[par * 4 + i]);
+            const int sh = q_shift_of_max(M);
+            const float up = __int_as_float((127 + sh) << 23);
+            uint8_t* hi_base = sB + qb * S::B_BUF;
+#pragma unroll
+            for (int i = 0; i < NCH; ++i) {
+                const int c = t + 128 * i, h = c >> 3, c16 = c & 7;
+                const uint32_t* w8 = reinterpret_cast<const uint32_t*>(&v[i][0]);
+                uint32_t hi4[4], lo4[4];
+#pragma unroll
+                for (int p = 0; p < 4; ++p) {  // 4 elements per output word
+                    uint32_t hw = 0, lw = 0;
+#pragma unroll
+                    for (int e2 = 0; e2 < 2; ++e2) {
+                        const uint32_t bb = w8[2 * p + e2];
+                        const float x0 = __uint_as_float(bb << 16) * up;
+                        const float x1 = __uint_as_float(bb & 0xFFFF0000u) * up;
+                        const uint32_t hp = e4m3x2_of(x0, x1);
+                        const float2 hf = float2_of_e4m3x2(hp);
+                        const uint32_t lp = e4m3x2_of(x0 - hf.x, x1 - hf.y);
+                        hw |= hp << (16 * e2);
+                        lw |= lp << (16 * e2);
+                    }
+                    hi4[p] = hw;
+                    lo4[p] = lw;
+                }
+                const int off = h * 128 + ((c16 ^ (h & 7)) << 4);
+                *reinterpret_cast<uint4*>(hi_base + off) = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
+                *reinterpret_cast<uint4*>(hi_base + S::B_HALF + off) =
+                    make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
+            }
+            // generic-proxy writes must be visible to the tensor core
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
-            if ((threadIdx.x & 31) == 0) {
-                mbar_arrive(&a_full[as]);
-                mbar_arrive(&raw_empty[rs]);
+            if (lane == 0) mbar_arrive(&q_full[qb]);
+            if (qw == 0) {
+                // publish w[b,:] and 2^-s for the epilogue: payload first, tag b
+                // last (the epilogue reaches this sequence only after the MMA
+                // consumed its q)
+                uint8_t* ent = seq_ring + (q_it % S::SEQ_RING) * S::SEQ_BYTES;
+                float* wr = reinterpret_cast<float*>(ent + 16);
+#pragma unroll
+                for (int r = 0; r < (H_I + 31) / 32; ++r) wr[r * 32 + lane] = wv[r];
+                if (lane == 0) reinterpret_cast<float*>(ent)[1] = __int_as_float((127 - sh) << 23);
+                __threadfence_block();
+                __syncwarp();
+                if (lane == 0) *reinterpret_cast<volatile int*>(ent) = cur_b;
             }
-            if (++rs == S::RAW_ST) {
-                rs = 0;
-                rph ^= 1;
-            }
-            if (++as == S::A_ST) {
-                as = 0;
-                aph ^= 1;
-            }
+            ++q_it;
         }
-    } else if (warp >= 12 && start_ok) {
+    } else if (warp >= 8 && start_ok) {
         // ------------------------------------------------ epilogue
-        const int lq = warp & 3;
-        float* wW = sW + lq * H_I;
+        const int hf = (warp - 8) >> 2;  // which 128-key half of every tile
+        const int lq = warp & 3;         // TMEM lanes 32 lq .. 32 lq + 31
+        const int key = hf * 128 + lq * 32 + lane;  // this thread's key within a tile
+        const float* wW = nullptr;  // w[b,:] of the current sequence, in the ring
+        uint32_t e_it = 0;          // sequences entered so far
         int acc = 0;
-        uint32_t acc_it[S::NACC] = {0, 0, 0, 0};
+        uint32_t acc_ph = 0;  // bit a: parity of accumulator a's next use
         int cur_b = -1;
+        float q_unscale = 1.f;  // 2^-s of the current sequence's q
         // this thread's per-token scales are prefetched SC_RING-1 tiles ahead
         // (walker `tp`) with cp.async into a per-thread shared-memory ring
-        // (zero past the sequence end), so no register waits on a global load
-        const uint32_t sc_ring = smem_u32(smem + S::OFF_SC) + (lq * 32 + lane) * 4;
+        // (zero past the sequence end)
+        const uint32_t sc_ring = smem_u32(smem + S::OFF_SC) + key * 4;
         TileWalk<S::BM> tw, tp;
-        tw.init(g_begin, g_end, tps, seq_len);
-        tp.init(g_begin, g_end, tps, seq_len);
+        tw.init(g_begin, g_end, tps, seq_len, S_max);
+        tp.init(g_begin, g_end, tps, seq_len, S_max);
         auto prefetch_scale = [&](int slot) {
             if (!tp.done()) {
-                const int s = tp.j * S::BM + lq * 32 + lane;
+                const int s = tp.j * S::BM + key;
                 const bool ok = s < tp.n;
                 const float* src = kscale + static_cast<long long>(tp.b) * S_max + (ok ? s : 0);
                 asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(
@@ -349,44 +422,73 @@ __global__ void __launch_bounds__(512, 1)
         for (int p = 0; p < S::SC_RING - 1; ++p) prefetch_scale(p);
         for (; !tw.done(); tw.next()) {
             prefetch_scale((it + S::SC_RING - 1) % S::SC_RING);
-            const int b = tw.b, j = tw.j, n = tw.n;
+            const int b = tw.b, n = tw.n;
+            const int s = tw.j * S::BM + key;
             if (b != cur_b) {
-                __syncwarp();
-                for (int h = lane; h < H_I; h += 32)
-                    wW[h] = __bfloat162float(w[static_cast<size_t>(b) * H_I + h]);
-                __syncwarp();
+                // the query warps published this sequence's entry before its q
+                // reached the tensor core; the tag makes the read self-checking
+                const uint8_t* ent = seq_ring + (e_it % S::SEQ_RING) * S::SEQ_BYTES;
+                bool seen = *reinterpret_cast<const volatile int*>(ent) == b;
+                if (!seen) {  // bounded: gives up on the CTA's abort flag or after the limit
+                    const long long t0 = clock64();
+                    while (!(seen = *reinterpret_cast<const volatile int*>(ent) == b)) {
+                        if (*abort_flag) break;
+                        if (clock64() - t0 > kWaitLimitCycles) {
+                            *abort_flag = 1;
+                            atomicCAS(err, 0, kDevTimeoutEpilogue);
+                            break;
+                        }
+                        __nanosleep(64);
+                    }
+                }
+                if (!__all_sync(0xffffffffu, seen)) break;
+                __threadfence_block();
+                q_unscale = reinterpret_cast<const volatile float*>(ent)[1];
+                wW = reinterpret_cast<const float*>(ent + 16);
+                ++e_it;
                 cur_b = b;
             }
-            const int s = j * S::BM + lq * 32 + lane;
-            bool got = mbar_wait(&acc_full[acc], acc_it[acc] & 1, abort_flag, err,
+            bool got = mbar_wait(&acc_full[acc], (acc_ph >> acc) & 1, abort_flag, err,
                                  kDevTimeoutEpilogue);
-            got = __all_sync(0xffffffffu, got);
-            if (!got) break;
+            if (!__all_sync(0xffffffffu, got)) break;
             tc_fence_after();
-            const uint32_t taddr =
-                tmem + (static_cast<uint32_t>(lq * 32) << 16) + static_cast<uint32_t>(acc * H_I);
-            uint32_t va[32], vb[32];
-            tmem_ld32(taddr, va);
-            if (H_I == 64) tmem_ld32(taddr + 32, vb);
-            tmem_ld_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[acc]);
-            float p[4] = {0.f, 0.f, 0.f, 0.f};
+            const uint32_t taddr = tmem + (static_cast<uint32_t>(lq * 32) << 16) +
+                                   static_cast<uint32_t>((2 * acc + hf) * S::ACC_COLS);
+            uint64_t p2[2] = {0, 0};  // two packed partial sums (heads h = 0, 1 mod 4; 2, 3 mod 4)
 #pragma unroll
-            for (int h = 0; h < H_I; h += 4) {
-                const float4 wv = *reinterpret_cast<const float4*>(wW + h);
-                const uint32_t* src = h < 32 ? va : vb;
-                p[0] = fmaf(wv.x, fmaxf(__uint_as_float(src[(h + 0) & 31]), 0.f), p[0]);
-                p[1] = fmaf(wv.y, fmaxf(__uint_as_float(src[(h + 1) & 31]), 0.f), p[1]);
-                p[2] = fmaf(wv.z, fmaxf(__uint_as_float(src[(h + 2) & 31]), 0.f), p[2]);
-                p[3] = fmaf(wv.w, fmaxf(__uint_as_float(src[(h + 3) & 31]), 0.f), p[3]);
+            for (int h0 = 0; h0 < H_I; h0 += 32) {  // 32 heads: their hi and lo columns
+                uint32_t vh[32], vl[32];
+                tmem_ld32(taddr + h0, vh);
+                tmem_ld32(taddr + H_I + h0, vl);
+                tmem_ld_wait();
+                if (h0 + 32 == H_I) {
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(&acc_empty[acc]);
+                }
+#pragma unroll
+                for (int h = 0; h < 32; h += 4) {
+                    const ulonglong2 w2 = *reinterpret_cast<const ulonglong2*>(wW + h0 + h);
+#pragma unroll
+                    for (int u = 0; u < 2; ++u) {
+                        const float2 x = f2_unpack(
+                            f2_add(f2_pack(__uint_as_float(vh[h + 2 * u]), __uint_as_float(vh[h + 2 * u + 1])),
+                                   f2_pack(__uint_as_float(vl[h + 2 * u]), __uint_as_float(vl[h + 2 * u + 1]))));
+                        p2[u] = f2_fma(u ? w2.y : w2.x, f2_pack(fmaxf(x.x, 0.f), fmaxf(x.y, 0.f)), p2[u]);
+                    }
+                }
             }
+            const float2 pa = f2_unpack(p2[0]), pb = f2_unpack(p2[1]);
+            const float p[4] = {pa.x, pa.y, pb.x, pb.y};
             cp_async_wait<S::SC_RING - 1>();  // this tile's scale has landed
             float sc;
-            asm volatile("ld.shared.f32 %0, [%1];" : "=f"(sc) : "r"(sc_ring + (it % S::SC_RING) * S::BM * 4));
-            if (s < n) scores[static_cast<long long>(b) * ld + s] = sc * ((p[0] + p[1]) + (p[2] + p[3]));
-            ++acc_it[acc];
+            asm volatile("ld.shared.f32 %0, [%1];"
+                         : "=f"(sc)
+                         : "r"(sc_ring + (it % S::SC_RING) * S::BM * 4));
+            if (s < n)
+                scores[static_cast<long long>(b) * ld + s] =
+                    (sc * q_unscale) * ((p[0] + p[1]) + (p[2] + p[3]));
+            acc_ph ^= 1u << acc;
             if (++acc == S::NACC) acc = 0;
             ++it;
         }
@@ -413,16 +515,21 @@ static int launch_decode_t(ic_ctx* ctx, const void* q, const void* w, const uint
         if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaFuncSetAttribute(index_decode)");
         attr_set = true;
     }
-    CUtensorMap tm_q;
-    int rc = make_tmap_bf16_2d(ctx, &tm_q, q, static_cast<uint64_t>(B) * H_I, 128, H_I);
+    // tile row coordinates are 32-bit
+    if (static_cast<long long>(B) * S_max + S::BM > 0x7FFFFFFFll)
+        return fail(ctx, IC_ERR_SHAPE, "decode index: B*S_max=%lld too large",
+                    static_cast<long long>(B) * S_max);
+    CUtensorMap tm_k;
+    int rc = make_tmap_u8_2d(ctx, &tm_k, kI8, static_cast<uint64_t>(B) * S_max, 128, 128, S::BM,
+                             true);
     if (rc) return rc;
     const int tps = (S_max + S::BM - 1) / S::BM;
     const long long total = static_cast<long long>(B) * tps;
     const int grid = total < ctx->num_sms ? static_cast<int>(total) : ctx->num_sms;
     LaunchScope ls(ctx, IC_K_INDEX_SCORE_DECODE, stream);
     k_index_score_decode<H_I><<<grid, 512, S::SMEM, stream>>>(
-        tm_q, kI8, static_cast<const __nv_bfloat16*>(w), kI_scale, seq_len, B, S_max, tps,
-        scores, static_cast<long long>(ld), ctx->dev_err);
+        tm_k, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(w), kI_scale,
+        seq_len, B, S_max, tps, scores, static_cast<long long>(ld), ctx->dev_err);
     cudaError_t e = ls.done();
     if (e != cudaSuccess) return cuda_fail(ctx, e, "index_score_decode launch");
     return IC_OK;

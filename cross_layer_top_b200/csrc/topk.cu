@@ -101,13 +101,15 @@ __device__ __forceinline__ void find_bin(TopkShared& S, uint32_t krem) {
 template <bool IN_SMEM>
 __global__ void __launch_bounds__(kTopkThreads)
     k_topk(const float* __restrict__ scores, long long ld, int row0, int k, int causal_base,
-           const int32_t* __restrict__ row_len, int32_t* __restrict__ out, long long ld_out) {
+           const int32_t* __restrict__ row_len, int max_len, int32_t* __restrict__ out,
+           long long ld_out) {
     extern __shared__ uint32_t srow[];
     __shared__ TopkShared S;
 
     const int r = row0 + blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int n = row_len ? row_len[r] : causal_base + r + 1;
+    // a given length above max_len (what shared memory was sized for) counts as max_len
+    const int n = row_len ? min(row_len[r], max_len) : causal_base + r + 1;
     int32_t* o = out + static_cast<long long>(r) * ld_out;
     if (n <= k) {
         for (int i = tid; i < k; i += kTopkThreads) o[i] = i < n ? i : -1;
@@ -271,7 +273,7 @@ struct TopkClusterShared {
 
 __global__ void __launch_bounds__(kTopkThreads)
     k_topk_cluster(const float* __restrict__ scores, long long ld, int k,
-                   const int32_t* __restrict__ row_len, int causal_base,
+                   const int32_t* __restrict__ row_len, int max_len, int causal_base,
                    int32_t* __restrict__ out, long long ld_out, int seg_cap) {
     // dynamic shared memory: the staged segment, then the merged candidates
     extern __shared__ uint32_t srow[];
@@ -281,7 +283,7 @@ __global__ void __launch_bounds__(kTopkThreads)
     const int r = blockIdx.y;
     const uint32_t rank = cluster_rank();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int n = row_len ? row_len[r] : causal_base + r + 1;
+    const int n = row_len ? min(row_len[r], max_len) : causal_base + r + 1;
     int32_t* o = out + static_cast<long long>(r) * ld_out;
     if (n <= k) {  // the same for every CTA of the cluster: no cluster barrier is reached
         if (rank == 0)
@@ -494,7 +496,7 @@ static int launch_topk_cluster(ic_ctx* ctx, const float* scores, int64_t ld, int
     cfg.numAttrs = 1;
     LaunchScope ls(ctx, IC_K_TOPK, stream);
     cudaLaunchKernelEx(&cfg, k_topk_cluster, scores, static_cast<long long>(ld), k, row_len,
-                       causal_base, idx_out, static_cast<long long>(ld_out), seg_cap);
+                       max_len, causal_base, idx_out, static_cast<long long>(ld_out), seg_cap);
     e = ls.done();
     if (e != cudaSuccess) return cuda_fail(ctx, e, "topk_cluster launch");
     return IC_OK;
@@ -531,14 +533,14 @@ int launch_topk(ic_ctx* ctx, const float* scores, int64_t ld, int rows, int k, i
         const int smem = ((nmax < kTopkSmemCap ? nmax : kTopkSmemCap) + 3) / 4 * 16;
         LaunchScope ls(ctx, IC_K_TOPK, stream);
         k_topk<true><<<split, kTopkThreads, smem, stream>>>(scores, ld, 0, k, causal_base, row_len,
-                                                             idx_out, ld_out);
+                                                             max_len, idx_out, ld_out);
         cudaError_t e = ls.done();
         if (e != cudaSuccess) return cuda_fail(ctx, e, "topk launch");
     }
     if (split < rows) {
         LaunchScope ls(ctx, IC_K_TOPK, stream);
         k_topk<false><<<rows - split, kTopkThreads, 0, stream>>>(scores, ld, split, k, causal_base,
-                                                                 row_len, idx_out, ld_out);
+                                                                 row_len, max_len, idx_out, ld_out);
         cudaError_t e = ls.done();
         if (e != cudaSuccess) return cuda_fail(ctx, e, "topk launch");
     }

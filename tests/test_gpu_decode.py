@@ -64,6 +64,48 @@ def test_decode_scores_integer_bit_exact(ic, ctx, H_I):
         assert np.all(np.isnan(got[b, n:]))
 
 
+def _e4m3_byte_of_int(v):
+    """e4m3 encoding of an integer with |v| <= 16 (1 sign, 4 exponent bits
+    with bias 7, 3 mantissa bits)."""
+    if v == 0:
+        return 0
+    a = abs(v)
+    e = a.bit_length() - 1
+    m = (a - (1 << e)) * 8 >> e
+    assert (((1 << e) + (m << e >> 3)) == a), v
+    return (0x80 if v < 0 else 0) | ((e + 7) << 3) | m
+
+
+@pytest.mark.parametrize("H_I", [64, 32])
+def test_decode_scores_wide_integer_exact(ic, ctx, H_I):
+    """Integer q in [-31, 31] and integer keys in [-16, 16]: a dot product
+    reaches 6.3e4 (well past 2^14) and every product, dot product and head
+    sum is an integer multiple of 0.5 small enough to be exact in fp32, so
+    the scores must equal the oracle's bit for bit.  This pins the split of
+    q into two e4m3 terms and full fp32 accumulation in the tensor core."""
+    B, S_max = 2, 777
+    gen = torch.Generator().manual_seed(11)
+    q = torch.randint(-31, 32, (B, H_I, 128), generator=gen).float()
+    q[:, 0, 0] = 31.0  # fixes max|q|, hence the power-of-two rescaling
+    q[:, 1, :] = torch.where(q[:, 1, :] >= 0, 31.0, -31.0)  # a head with large dot products
+    table = torch.tensor([_e4m3_byte_of_int(v) for v in range(-16, 17)], dtype=torch.uint8)
+    k8 = table[torch.randint(0, 33, (B, S_max, 128), generator=gen)]
+    for b in range(B):  # rows 0..4: keys 16 sign(q[b,1,:]), so head 1's dot product is 31*16*128
+        k8[b, :5, :] = torch.where(q[b, 1, :] >= 0, table[32], table[0])
+    w = torch.tensor([-1.0, -0.5, 0.5, 1.0])[torch.randint(0, 4, (B, H_I), generator=gen)]
+    sc = torch.tensor([1.0, 0.5, 2.0, 0.25])[torch.randint(0, 4, (B, S_max), generator=gen)]
+    lens = torch.tensor([S_max, 300], dtype=torch.int32)
+    q, w = q.bfloat16(), w.bfloat16()
+    out = torch.full((B, 780), float("nan"), device="cuda")  # ld: a multiple of 4
+    ic.ic_index_score_decode(ctx, q.cuda(), w.cuda(), k8.cuda(), sc.float().cuda(), lens.cuda(), out)
+    ctx.sync_status()
+    got = out.cpu().numpy()
+    for b in range(B):
+        n = int(lens[b])
+        ref = oracle.decode_scores(f32(q[b]), f32(w[b]), k8[b].numpy(), sc[b].float().numpy(), S=n)
+        assert np.array_equal(got[b, :n].astype(np.float64), ref)
+
+
 def test_decode_scores_gaussian_close(ic, ctx):
     B, S_max = 4, 6000
     q, w, k8, sc, lens = _decode_inputs(B, S_max, 64, 2, lens=[6000, 5999, 4097, 3])
