@@ -152,10 +152,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
            (static_cast<uint32_t>(M >> 4) << 24);
 }
 
-// Instruction descriptor, kind::f16: D = F32, A = B = F16, both K-major.
-__host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
-    return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
-}
 
 // Instruction descriptor, kind::f8f6f4: D = F32, A = B = E4M3 (format 0),
 // both K-major.

@@ -253,6 +253,79 @@ def test_attention_random_indices(ic, ctx, d, Hq):
     attn_close(out.float().cpu().numpy(), ref)
 
 
+@pytest.mark.parametrize("Hq,k", [(16, 2048), (5, 1000)])
+def test_attention_many_rows(ic, ctx, Hq, k):
+    """Enough rows (400, over two per SM) for the tensor-core kernel: row
+    lengths from 0 to k (ragged tiles, empty rows), sorted, unsorted and
+    gapped index rows, k not a multiple of the 128-key tile."""
+    gen = torch.Generator().manual_seed(7 + Hq)
+    rows, S, d = 400, 5000, 128
+    Q = (torch.randn((rows, Hq, d), generator=gen) / math.sqrt(d)).bfloat16()
+    K = torch.randn((S, d), generator=gen).bfloat16()
+    V = torch.randn((S, d), generator=gen).bfloat16()
+    idx = torch.full((rows, k), -1, dtype=torch.int32)
+    lens = [0, 1, 17, 128, 129, 1500, k, 33, 255, 256, k - 1, 640]
+    for r in range(rows):
+        n = min(lens[r % len(lens)], k)
+        sel = torch.randperm(S, generator=gen)[:n].int()
+        kind = (r // len(lens)) % 3
+        if kind == 0:
+            idx[r, :n] = torch.sort(sel).values
+        elif kind == 1:
+            idx[r, :n] = sel  # unsorted
+        else:  # gaps: the selected slots scattered over the row
+            pos = torch.sort(torch.randperm(k, generator=gen)[:n]).values
+            idx[r, pos] = sel
+    out = torch.empty((rows, Hq, d), dtype=torch.bfloat16, device="cuda")
+    ic.ic_sparse_attn(ctx, Q.cuda(), K.cuda(), V.cuda(), idx.cuda(), out)
+    ctx.sync_status()
+    ref = oracle.sparse_attn(f32(Q), f32(K), f32(V), idx.numpy())
+    attn_close(out.float().cpu().numpy(), ref)
+
+
+def test_attention_many_rows_per_sequence(ic, ctx):
+    """Several sequences (rows_per_seq = 100, each with its own K/V block)
+    through the tensor-core kernel."""
+    gen = torch.Generator().manual_seed(21)
+    nseq, rps, S, Hq, d, k = 4, 100, 3000, 16, 128, 2048
+    rows = nseq * rps
+    Q = (torch.randn((rows, Hq, d), generator=gen) / math.sqrt(d)).bfloat16()
+    K = torch.randn((nseq, S, d), generator=gen).bfloat16()
+    V = torch.randn((nseq, S, d), generator=gen).bfloat16()
+    idx = torch.full((rows, k), -1, dtype=torch.int32)
+    for r in range(rows):
+        n = [2048, 700, 1, 1999][r % 4]
+        idx[r, :n] = torch.sort(torch.randperm(S, generator=gen)[:n]).values
+    out = torch.empty((rows, Hq, d), dtype=torch.bfloat16, device="cuda")
+    ic.ic_sparse_attn(ctx, Q.cuda(), K.cuda(), V.cuda(), idx.cuda(), out, rows_per_seq=rps,
+                      kv_seq_stride=S * d, kv_len=S)
+    ctx.sync_status()
+    ref = oracle.sparse_attn(f32(Q), f32(K), f32(V), idx.numpy(), rows_per_seq=rps)
+    attn_close(out.float().cpu().numpy(), ref)
+
+
+def test_attention_many_rows_bad_index_is_reported(ic, ctx):
+    gen = torch.Generator().manual_seed(5)
+    rows, S, Hq, d, k = 320, 100, 16, 128, 8
+    Q = torch.randn((rows, Hq, d), generator=gen).bfloat16()
+    K = torch.randn((S, d), generator=gen).bfloat16()
+    V = torch.randn((S, d), generator=gen).bfloat16()
+    idx = torch.randint(0, S, (rows, k), generator=gen, dtype=torch.int32)
+    idx[3, 2] = S        # past the end
+    idx[100, 0] = -7     # negative other than -1
+    out = torch.empty((rows, Hq, d), dtype=torch.bfloat16, device="cuda")
+    ic.ic_sparse_attn(ctx, Q.cuda(), K.cuda(), V.cuda(), idx.cuda(), out)
+    with pytest.raises(ic.ICError) as e:
+        ctx.sync_status()
+    assert e.value.code == ic.IC_ERR_DEVICE
+    ctx.sync_status()
+    clean = idx.clone()
+    clean[3, 2] = -1
+    clean[100, 0] = -1
+    ref = oracle.sparse_attn(f32(Q), f32(K), f32(V), clean.numpy())
+    attn_close(out.float().cpu().numpy(), ref)
+
+
 def test_attention_decode_split(ic, ctx):
     """rows_per_seq = 1 (decode): few rows, split across CTAs and combined."""
     gen = torch.Generator().manual_seed(3)
