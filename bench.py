@@ -227,6 +227,7 @@ def run_ours(args, rank, world, local_rank):
             extra_ceiling = None
     else:
         extra_ceiling = None
+    overlap = measure_overlap(ctx, layers, cfg, stream)
     dominant = max(("index_score", "sparse_attn"), key=lambda n: ktimes[n]["ms"])
     roofline = dict(roof.get(dominant, {}))
     roofline["kernel"] = dominant
@@ -240,6 +241,7 @@ def run_ours(args, rank, world, local_rank):
         "step_ms": [round(x, 4) for x in step_ms],
         "roofline_all": roof,
         "l2_gather_ceiling": extra_ceiling,
+        "cross_layer_overlap": overlap,
     }
 
     # ------------------------------------------------ e2e through the C ABI with host buffers
@@ -318,6 +320,37 @@ def measure_gather_ceiling(cache, lay, L, k, stream):
     nbytes = (L - k) * k * 2 * lay["K"].shape[-1] * 2
     return {"achieved_gbs": round(nbytes / (best / 1e3) / 1e9, 1), "ms": best, "bytes": nbytes,
             "what": "cp.async gather of the same K/V rows (index rows t >= k), no compute"}
+
+
+def measure_overlap(ctx, layers, cfg, stream):
+    """The cross-layer overlap diagnostic between the stack's two F layers
+    (0 and 4): their top-k sets recomputed, then |T_0 ∩ T_4| per row timed
+    over all L rows.  The synthetic layers are independent, so the overlap
+    is near that of random sets (about k / (t + 1)), not the 70-100% a
+    trained model shows between neighbouring layers."""
+    from cross_layer_top_b200 import indexcache as ic
+    f = [l for l, c in enumerate(cfg.pattern) if c == "F"]
+    if len(f) < 2:
+        return None
+    L, k = cfg.L, cfg.k
+    idx = [torch.empty((L, k), dtype=torch.int32, device=layers[0]["Q"].device) for _ in range(2)]
+    for t, l in zip(idx, f[:2]):
+        ic.ic_index_fp(ctx, layers[l]["qI"], layers[l]["kI"], layers[l]["w"], k, t)
+    hits = torch.empty(L, dtype=torch.int32, device=idx[0].device)
+    ic.ic_index_overlap(ctx, idx[0], idx[1], hits, L)
+    best = None
+    for _ in range(5):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        ic.ic_index_overlap(ctx, idx[0], idx[1], hits, L)
+        b.record(stream)
+        b.synchronize()
+        best = a.elapsed_time(b) if best is None else min(best, a.elapsed_time(b))
+    ctx.sync_status()
+    h = hits[k:].double()  # rows with a full k-set in both layers
+    return {"layers": f[:2], "mean_overlap_full_rows": round(float(h.mean()) / k, 5),
+            "kernel_ms": round(best, 4), "rows_per_s": L / (best / 1e3),
+            "bytes_per_launch": 2 * L * k * 4}
 
 
 def run_e2e(args, ctx, pat, dims, cfg, layers, cache, world, pairs_step, stream):
@@ -492,8 +525,9 @@ def run_long_prefill(args, ctx, peaks, local_rank):
 
 def run_decode_sweep(args, ctx, local_rank):
     """200K-context decode: 8 sequences x 200001 candidates, 47 layers, one
-    decode step at uniform retention 1/1, 1/2, 1/4, 1/8 (the same layer
-    tensors; S layers ignore their indexer inputs)."""
+    decode step at uniform retention 1/1, 1/2, 1/4, 1/8 and with the searched
+    patterns at 1/2, 1/4, 1/8 (the same layer tensors; S layers ignore their
+    indexer inputs)."""
     from cross_layer_top_b200 import indexcache as ic
     from cross_layer_top_b200 import synth
     cfg = synth.CONFIGS["decode_sweep_r1"]
@@ -520,6 +554,15 @@ def run_decode_sweep(args, ctx, local_rank):
         res["r%d" % r] = {"pattern_F_layers": str(pat).count("F"), "step_ms": ms,
                           "tokens_per_s": B / (ms / 1e3),
                           "kernels_ms": {n: round(v, 4) for n, v in kt.items()}}
+    # the searched patterns of the 47-layer model (same layer tensors)
+    for ret, c in synth.SEARCHED_PATTERNS_47.items():
+        pat = ic.ic_create_pattern(c)
+        for _ in range(2):
+            ic.ic_run_stack(ctx, pat, None, dims, cache, layer_array=arr)
+        ms, kt = _time_stack(ctx, pat, dims, cache, arr, 5, stream)
+        res["searched_" + ret.replace("/", "_")] = {
+            "pattern_F_layers": c.count("F"), "step_ms": ms, "tokens_per_s": B / (ms / 1e3),
+            "kernels_ms": {n: round(v, 4) for n, v in kt.items()}}
     res["speedup_r4_vs_r1"] = res["r1"]["step_ms"] / res["r4"]["step_ms"]
     del layers, arr, cache
     torch.cuda.empty_cache()

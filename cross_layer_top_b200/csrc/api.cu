@@ -450,6 +450,18 @@ extern "C" int ic_sparse_attn(ic_ctx* ctx, const void* Q, const void* K, const v
                               kv_len, scale, out, as_stream(stream));
 }
 
+// -------------------------------------------------- cross-layer overlap
+extern "C" int ic_index_overlap(ic_ctx* ctx, const int32_t* idx_a, const int32_t* idx_b, int rows,
+                                int k, int n_keys, int32_t* hits, void* stream) {
+    if (!ctx) return fail(nullptr, IC_ERR_INVALID_ARG, "context is NULL");
+    if (rows < 0 || k < 1 || n_keys < 1)
+        return fail(ctx, IC_ERR_SHAPE, "index_overlap: rows=%d k=%d n_keys=%d", rows, k, n_keys);
+    if (rows == 0) return IC_OK;
+    if (!idx_a || !idx_b || !hits) return fail(ctx, IC_ERR_INVALID_ARG, "index_overlap: NULL");
+    cudaSetDevice(ctx->device);
+    return launch_index_overlap(ctx, idx_a, idx_b, rows, k, n_keys, hits, as_stream(stream));
+}
+
 // ------------------------------------------------------------ layer stack
 extern "C" int ic_run_stack(ic_ctx* ctx, const ic_pattern* pattern, const ic_layer_io* layers,
                             const ic_stack_dims* dims, int32_t* idx_cache, void* stream) {

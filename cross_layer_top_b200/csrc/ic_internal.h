@@ -82,6 +82,8 @@ int launch_index_score_decode(ic_ctx* ctx, const void* q, const void* w, const u
 int launch_topk(ic_ctx* ctx, const float* scores, int64_t ld, int rows, int k, int causal_base,
                 const int32_t* row_len, int max_len, int32_t* idx_out, int64_t ld_out,
                 cudaStream_t stream);
+int launch_index_overlap(ic_ctx* ctx, const int32_t* a, const int32_t* b, int rows, int k,
+                         int n_keys, int32_t* hits, cudaStream_t stream);
 int launch_sparse_attn(ic_ctx* ctx, const void* Q, const void* K, const void* V,
                        const int32_t* idx, int rows, int Hq, int d, int k, int rows_per_seq,
                        int64_t kv_seq_stride, int kv_len, float scale, void* out,

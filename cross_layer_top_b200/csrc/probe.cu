@@ -73,3 +73,30 @@ extern "C" int ic_probe_gather(const void* K, const void* V, const int32_t* idx,
     if (e != cudaSuccess) return ic::cuda_fail(nullptr, e, "probe_gather launch");
     return IC_OK;
 }
+
+namespace ic {
+
+// One bounded wait on a barrier that nothing arrives at: the library's
+// bounded mbarrier wait gives up after its limit and latches the timeout code.
+__global__ void k_probe_wait_timeout(int* err) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_s;
+    if (threadIdx.x == 0) {
+        abort_s = 0;
+        mbar_init(&bar, 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) mbar_wait(&bar, 0, &abort_s, err, kDevTimeoutProducer);
+}
+
+}  // namespace ic
+
+extern "C" int ic_probe_wait_timeout(ic_ctx* ctx, void* stream) {
+    if (!ctx) return ic::fail(nullptr, IC_ERR_INVALID_ARG, "probe_wait_timeout: context is NULL");
+    cudaSetDevice(ctx->device);
+    ic::k_probe_wait_timeout<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(ctx->dev_err);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return ic::cuda_fail(ctx, e, "probe_wait_timeout launch");
+    return IC_OK;
+}

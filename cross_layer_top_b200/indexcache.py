@@ -36,9 +36,9 @@ IC_K_INDEX_SCORE = 0
 IC_K_INDEX_SCORE_DECODE = 1
 IC_K_TOPK = 2
 IC_K_ATTN = 3
-IC_K_ATTN_COMBINE = 4
+IC_K_OVERLAP = 4
 IC_K_COUNT = 5
-KERNEL_NAMES = ["index_score", "index_score_decode", "topk", "sparse_attn", "attn_combine"]
+KERNEL_NAMES = ["index_score", "index_score_decode", "topk", "sparse_attn", "index_overlap"]
 
 _vp = ctypes.c_void_p
 _i = ctypes.c_int
@@ -81,6 +81,8 @@ _SIGS = {
     "ic_index_fp_decode_noalloc": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp], _i),
     "ic_probe_gather": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp], _i),
     "ic_sparse_attn": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64, _i, _f, _vp, _vp], _i),
+    "ic_index_overlap": ([_vp, _vp, _vp, _i, _i, _i, _vp, _vp], _i),
+    "ic_probe_wait_timeout": ([_vp, _vp], _i),
     "ic_run_stack": ([_vp, _vp, ctypes.POINTER(ic_layer_io), ctypes.POINTER(ic_stack_dims), _vp,
                       _vp], _i),
 }
@@ -294,6 +296,22 @@ def ic_sparse_attn(ctx: Context, Q, K, V, idx, out, rows_per_seq: int = 0, kv_se
     _check(_lib.ic_sparse_attn(ctx.handle, _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), rows, Hq, d, k,
                                rows_per_seq, kv_seq_stride, kv_len, scale, _ptr(out),
                                _stream(stream)), ctx)
+
+
+def ic_index_overlap(ctx: Context, idx_a, idx_b, hits, n_keys: int, stream=None):
+    """hits[r] = |T_a[r] ∩ T_b[r]| for two [rows, k] int32 index tensors
+    (the overlap of row r is hits[r] / k)."""
+    rows, k = idx_a.shape
+    if tuple(idx_b.shape) != (rows, k):
+        raise ValueError("idx_a and idx_b must have the same shape")
+    _check(_lib.ic_index_overlap(ctx.handle, _ptr(idx_a), _ptr(idx_b), rows, k, n_keys, _ptr(hits),
+                                 _stream(stream)), ctx)
+
+
+def ic_probe_wait_timeout(ctx: Context, stream=None):
+    """Test aid: one bounded device wait that runs out (about a second); the
+    next ctx.sync_status() raises IC_ERR_TIMEOUT."""
+    _check(_lib.ic_probe_wait_timeout(ctx.handle, _stream(stream)), ctx)
 
 
 def ic_probe_gather(K, V, idx, ctas_per_sm: int = 2, stream=None):

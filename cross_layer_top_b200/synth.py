@@ -18,7 +18,8 @@ Distributions per workload (all tensors bf16 unless stated):
                 scale (amax/448 of the N(0,1) key); main K/V ~ N(0,1);
                 16 query heads, d=128, k=2048; seed 3
   decode_sweep  8 sequences x (200000 + 1) tokens, 47 layers, uniform
-                retention 1/r; otherwise as decode; seed 4
+                retention 1/r (or the searched patterns below); otherwise as
+                decode; seed 4
 """
 from __future__ import annotations
 
@@ -84,6 +85,16 @@ CONFIGS = {
 for _r in (1, 2, 4, 8):
     CONFIGS["decode_sweep_r%d" % _r] = DecodeConfig(
         "decode_sweep_r%d" % _r, 8, 200000, uniform_pattern(47, _r), 64, 128, 2048, 16, 128, 4)
+
+# The F/S patterns searched for the 47-layer model at retention 1/2, 1/4 and
+# 1/8 ("IndexCache: Accelerating Sparse Attention via Cross-Layer Index
+# Reuse", Appendix B): 24, 12 and 7 F layers.  Run on the 200K decode sweep's
+# layer tensors in place of the uniform patterns.
+SEARCHED_PATTERNS_47 = {
+    "1/2": "FSFSFSSSSFSFFFFSFFSSFFSFFFSSFFSSFSSSSFSFFFSFSSF",
+    "1/4": "FSFSFSSSSFSSSFSSFFSSFSSFSSSSFSSSFSSSSFSSSSSSSSS",
+    "1/8": "FSSSFSSSSSSSSFSSSFSSSSSFSSSSFSSSSSSSSFSSSSSSSSS",
+}
 
 
 def _gen(device, seed: int, layer: int, slot: int) -> torch.Generator:

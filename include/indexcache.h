@@ -63,7 +63,7 @@ extern "C" {
 #define IC_K_INDEX_SCORE_DECODE 1 /* decode FP8 indexer-key scan (tcgen05) */
 #define IC_K_TOPK 2               /* per-row top-k select */
 #define IC_K_ATTN 3               /* sparse MQA attention (gather + softmax) */
-#define IC_K_ATTN_COMBINE 4       /* split-attention combine */
+#define IC_K_OVERLAP 4            /* cross-layer index overlap (diagnostic) */
 #define IC_K_COUNT 5
 
 typedef struct ic_ctx ic_ctx;
@@ -203,6 +203,19 @@ int ic_index_fp_decode_noalloc(const void *q, const void *w, const uint8_t *kI8,
 int ic_sparse_attn(ic_ctx *ctx, const void *Q, const void *K, const void *V, const int32_t *idx,
                    int rows, int Hq, int d, int k, int rows_per_seq, int64_t kv_seq_stride,
                    int kv_len, float scale, void *out, void *stream);
+
+/* ------------------------------------------------ cross-layer overlap */
+
+/* [IC] Appendix A, [RN] §3.2: how far two layers' top-k sets agree, the
+ * quantity that makes reusing one layer's indices in the next workable.
+ *   hits[r] = |{x : idx_a[r,x] >= 0 and idx_a[r,x] occurs in idx_b[r,:]}|
+ * and the overlap of row r is hits[r] / k.  idx_a, idx_b: device int32
+ * [rows, k], contiguous, entries in [0, n_keys) or -1 (never counted), in any
+ * order; an entry of idx_a counts once per occurrence.  hits: device int32
+ * [rows], written by this call.  An entry outside [-1, n_keys) is skipped and
+ * latched as IC_ERR_DEVICE.  Supported: 1 <= n_keys <= 6553600, k >= 1. */
+int ic_index_overlap(ic_ctx *ctx, const int32_t *idx_a, const int32_t *idx_b, int rows, int k,
+                     int n_keys, int32_t *hits, void *stream);
 
 /* ------------------------------------------------------------ layer stack */
 

@@ -13,11 +13,21 @@
  *   in [0, kv_len).  d = 128, k a multiple of 64, 1 <= ctas_per_sm <= 3.
  * Returns IC_OK or IC_ERR_INVALID_ARG / IC_ERR_UNSUPPORTED / IC_ERR_CUDA;
  * asynchronous on `stream`; allocates nothing.
+ *
+ * ic_probe_wait_timeout is a test aid for failure detection: it enqueues one
+ * CTA that waits on a shared-memory barrier nothing ever arrives at, with the
+ * same bounded wait the library's pipelined kernels use.  The wait gives up
+ * after its limit (about one second), the kernel returns normally and the
+ * timeout is latched in ctx, so the next ic_sync_status(ctx, stream) returns
+ * IC_ERR_TIMEOUT and clears it; the context stays usable.  Nothing traps or
+ * faults.  Returns IC_OK, IC_ERR_INVALID_ARG (ctx NULL) or IC_ERR_CUDA.
  */
 #ifndef INDEXCACHE_PROBE_H
 #define INDEXCACHE_PROBE_H
 
 #include <stdint.h>
+
+#include "indexcache.h"
 
 #ifdef __cplusplus
 extern "C" {
@@ -25,6 +35,8 @@ extern "C" {
 
 int ic_probe_gather(const void *K, const void *V, const int32_t *idx, int rows, int k, int d,
                     int ctas_per_sm, void *stream);
+
+int ic_probe_wait_timeout(ic_ctx *ctx, void *stream);
 
 #ifdef __cplusplus
 }

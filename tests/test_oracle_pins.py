@@ -47,6 +47,15 @@ def test_appendix_b_patterns(golden):
             assert "F" not in c[src[l] + 1:l + 1] if ch == "S" else src[l] == l
 
 
+def test_searched_patterns_in_the_sweep_match_the_pages(golden):
+    """The decode sweep's searched patterns are the printed 47-layer ones."""
+    from cross_layer_top_b200 import synth
+    printed = {p["retention"]: p["c"] for p in golden["appendix_b_patterns"]["patterns"]
+               if p["layers"] == 47}
+    assert synth.SEARCHED_PATTERNS_47 == printed
+    assert [c.count("F") for c in synth.SEARCHED_PATTERNS_47.values()] == [24, 12, 7]
+
+
 @pytest.mark.parametrize("bad", ["", "SFFF", "FSXS", "fsss", "S"])
 def test_pattern_rejects(bad):
     with pytest.raises(ValueError):
@@ -324,6 +333,25 @@ def test_attention_batched_sequences():
 def test_overlap_page_toy(golden):
     g = golden["overlap_toy"]
     assert oracle.overlap(g["a"], g["b"]) == g["overlap"]
+
+
+def test_overlap_against_set_intersection():
+    """The pairwise search equals a hash-set intersection on rows without
+    repeats; a row against itself counts its selected entries, disjoint rows
+    count nothing."""
+    rng = np.random.default_rng(4)
+    k = 97
+    for _ in range(20):
+        na, nb = rng.integers(0, k + 1, 2)
+        pool = rng.permutation(150)
+        a = np.full(k, -1, np.int32)
+        b = np.full(k, -1, np.int32)
+        a[rng.permutation(k)[:na]] = pool[:na]
+        b[rng.permutation(k)[:nb]] = rng.permutation(pool[:120])[:nb]
+        expect = len(set(a[a >= 0].tolist()) & set(b[b >= 0].tolist()))
+        assert round(oracle.overlap(a, b) * k) == expect  # the ratio, scaled back to a count
+        assert round(oracle.overlap(a, a) * k) == na
+    assert oracle.overlap(np.arange(10), np.arange(10, 20)) == 0.0
 
 
 def test_stack_reuse_invariant():
