@@ -254,6 +254,7 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.empty_cache()
     if not args.no_decode:
         extra["decode"] = run_decode(args, ctx, peaks, peak_src, local_rank)
+    extra["fp8_indexer"] = run_fp8_indexer(args, ctx, peaks, peak_src, local_rank)
     if not args.no_extended:
         extra["long_prefill"] = run_long_prefill(args, ctx, peaks, local_rank)
         extra["decode_retention_sweep"] = run_decode_sweep(args, ctx, local_rank)
@@ -521,6 +522,49 @@ def run_long_prefill(args, ctx, peaks, local_rank):
     del layers, arr, cache
     torch.cuda.empty_cache()
     return res
+
+
+def run_fp8_indexer(args, ctx, peaks, peak_src, local_rank):
+    """The FP8 prefill indexer (e4m3 q_I / k_I, per-(token, head) and
+    per-token scales) on the prefill workload's F layer: one F layer (scores
+    + top-k) per step, 3 warm-up and 10 timed; the score kernel's roofline
+    against the fp8 tensor peak (the measured bf16 peak x 2, the nominal
+    fp8 / bf16 ratio)."""
+    from cross_layer_top_b200 import indexcache as ic
+    from cross_layer_top_b200 import synth
+    cfg = synth.CONFIGS["prefill"]
+    dev = torch.device("cuda", local_rank)
+    lay = synth.prefill_indexer_fp8(cfg, 0, dev)
+    L, k = cfg.L, cfg.k
+    idx = torch.empty((L, k), dtype=torch.int32, device=dev)
+    run = lambda: ic.ic_index_fp_fp8(ctx, lay["qI8"], lay["q_scale"], lay["kI8"], lay["k_scale"],
+                                     lay["w"], k, idx)
+    for _ in range(3):
+        run()
+    ctx.sync_status()
+    ctx.reset_timing()
+    ctx.set_timing(True)
+    n = 10
+    for _ in range(n):
+        run()
+    torch.cuda.synchronize()
+    ctx.set_timing(False)
+    ctx.sync_status()
+    ms, launches = ctx.get_timing(ic.IC_K_INDEX_SCORE)
+    tms, _ = ctx.get_timing(ic.IC_K_TOPK)
+    pairs = sum(t + 1 for t in range(k, L))  # rows t >= k are scored
+    flop = 2 * cfg.H_I * cfg.d_I * pairs
+    avg = ms / launches
+    tflops = flop / (avg / 1e3) / 1e12
+    peak = 2 * peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
+    del lay, idx
+    torch.cuda.empty_cache()
+    return {"workload": "prefill F layer, FP8 indexer inputs: L=16384, H_I=64, d_I=128, k=2048",
+            "score_ms": round(avg, 4), "topk_ms": round(tms / n, 4),
+            "roofline": {"bound": "tensor", "achieved": round(tflops, 1), "peak": round(peak, 1),
+                         "unit": "TFLOP/s", "frac": round(tflops / peak, 4), "traffic": None,
+                         "peak_kind": "2 x sustained bf16, " + peak_src},
+            "flop_per_launch": flop}
 
 
 def run_decode_sweep(args, ctx, local_rank):

@@ -337,6 +337,37 @@ extern "C" int ic_topk(ic_ctx* ctx, const float* scores, int64_t ld, int rows, i
                        as_stream(stream));
 }
 
+// F layer: rows t < k select {0..t} without scores; the other rows are
+// scored in chunks whose fp32 rows fit in the scratch limit, each chunk
+// followed by its top-k.  `score(rb, re, scores, ld)` scores rows [rb, re).
+template <class ScoreFn>
+static int index_fp_rows(ic_ctx* ctx, int L, int k, int32_t* idx_out, cudaStream_t s,
+                         ScoreFn score) {
+    const int first = k < L ? k : L;
+    if (first > 0) {
+        int rc = launch_topk(ctx, nullptr, 0, first, k, 0, nullptr, 0, idx_out, k, s);
+        if (rc) return rc;
+    }
+    if (first >= L) return IC_OK;
+    const int64_t ld = (static_cast<int64_t>(L) + 63) / 64 * 64;
+    int64_t chunk = static_cast<int64_t>(ctx->scratch_limit / (static_cast<size_t>(ld) * 4));
+    if (chunk < 1) return fail(ctx, IC_ERR_NOMEM, "index_fp: scratch too small for one row");
+    if (chunk > L - first) chunk = L - first;
+    int rc = ensure_buffer(ctx, reinterpret_cast<void**>(&ctx->scores), &ctx->scores_cap,
+                           static_cast<size_t>(chunk) * ld * 4);
+    if (rc) return rc;
+    for (int rb = first; rb < L; rb += static_cast<int>(chunk)) {
+        const int re = static_cast<int>(rb + chunk < L ? rb + chunk : L);
+        const int64_t ldc = (static_cast<int64_t>(re) + 63) / 64 * 64;
+        rc = score(rb, re, ctx->scores, ldc);
+        if (rc) return rc;
+        rc = launch_topk(ctx, ctx->scores, ldc, re - rb, k, rb,
+                         nullptr, 0, idx_out + static_cast<int64_t>(rb) * k, k, s);
+        if (rc) return rc;
+    }
+    return IC_OK;
+}
+
 extern "C" int ic_index_fp(ic_ctx* ctx, const void* qI, const void* kI, const void* w, int L,
                            int H_I, int d_I, int k, int32_t* idx_out, void* stream) {
     int rc = check_index_args(ctx, qI, kI, w, L, H_I, d_I);
@@ -345,31 +376,59 @@ extern "C" int ic_index_fp(ic_ctx* ctx, const void* qI, const void* kI, const vo
     if (k < 1 || k > 2048) return fail(ctx, IC_ERR_SHAPE, "index_fp: k=%d not in [1,2048]", k);
     cudaSetDevice(ctx->device);
     cudaStream_t s = as_stream(stream);
-    // rows t < k select {0..t} without scores
-    const int first = k < L ? k : L;
-    if (first > 0) {
-        rc = launch_topk(ctx, nullptr, 0, first, k, 0, nullptr, 0, idx_out, k, s);
-        if (rc) return rc;
-    }
-    if (first >= L) return IC_OK;
-    // chunks of rows whose fp32 score rows fit in the scratch limit
-    const int64_t ld = (static_cast<int64_t>(L) + 63) / 64 * 64;
-    int64_t chunk = static_cast<int64_t>(ctx->scratch_limit / (static_cast<size_t>(ld) * 4));
-    if (chunk < 1) return fail(ctx, IC_ERR_NOMEM, "index_fp: scratch too small for one row");
-    if (chunk > L - first) chunk = L - first;
-    rc = ensure_buffer(ctx, reinterpret_cast<void**>(&ctx->scores), &ctx->scores_cap,
-                       static_cast<size_t>(chunk) * ld * 4);
-    if (rc) return rc;
-    for (int rb = first; rb < L; rb += static_cast<int>(chunk)) {
-        const int re = static_cast<int>(rb + chunk < L ? rb + chunk : L);
-        const int64_t ldc = (static_cast<int64_t>(re) + 63) / 64 * 64;
-        rc = launch_index_score_prefill(ctx, qI, kI, w, L, H_I, d_I, rb, re, ctx->scores, ldc, s);
-        if (rc) return rc;
-        rc = launch_topk(ctx, ctx->scores, ldc, re - rb, k, rb,
-                         nullptr, 0, idx_out + static_cast<int64_t>(rb) * k, k, s);
-        if (rc) return rc;
-    }
+    return index_fp_rows(ctx, L, k, idx_out, s, [&](int rb, int re, float* sc, int64_t ldc) {
+        return launch_index_score_prefill(ctx, qI, kI, w, L, H_I, d_I, rb, re, sc, ldc, s);
+    });
+}
+
+// ------------------------------------------------ FP8 prefill indexer
+static int check_index_fp8_args(ic_ctx* ctx, const uint8_t* qI8, const float* q_scale,
+                                const uint8_t* kI8, const float* k_scale, const void* w, int L,
+                                int H_I, int d_I) {
+    if (!ctx) return fail(nullptr, IC_ERR_INVALID_ARG, "context is NULL");
+    if (!qI8 || !q_scale || !kI8 || !k_scale || !w)
+        return fail(ctx, IC_ERR_INVALID_ARG, "index_fp8: NULL input");
+    if (!aligned16(qI8) || !aligned16(kI8))
+        return fail(ctx, IC_ERR_INVALID_ARG, "index_fp8: qI8 and kI8 must be 16-byte aligned");
+    if (L < 1 || L > (1 << 24)) return fail(ctx, IC_ERR_SHAPE, "index_fp8: L=%d", L);
+    if (d_I != 128 || (H_I != 16 && H_I != 32 && H_I != 64))
+        return fail(ctx, IC_ERR_UNSUPPORTED, "index_fp8: H_I=%d d_I=%d (need {16,32,64}, 128)",
+                    H_I, d_I);
     return IC_OK;
+}
+
+extern "C" int ic_index_score_fp8(ic_ctx* ctx, const uint8_t* qI8, const float* q_scale,
+                                  const uint8_t* kI8, const float* k_scale, const void* w, int L,
+                                  int H_I, int d_I, int row_begin, int row_end, float* scores,
+                                  int64_t ld, void* stream) {
+    int rc = check_index_fp8_args(ctx, qI8, q_scale, kI8, k_scale, w, L, H_I, d_I);
+    if (rc) return rc;
+    if (!scores) return fail(ctx, IC_ERR_INVALID_ARG, "index_score_fp8: scores is NULL");
+    if (row_begin < 0 || row_end > L || row_begin > row_end)
+        return fail(ctx, IC_ERR_SHAPE, "index_score_fp8: rows [%d,%d) outside [0,%d)", row_begin,
+                    row_end, L);
+    if (ld < row_end || ld % 4 != 0)
+        return fail(ctx, IC_ERR_SHAPE,
+                    "index_score_fp8: ld=%lld must be >= row_end and a multiple of 4",
+                    (long long)ld);
+    cudaSetDevice(ctx->device);
+    return launch_index_score_prefill_fp8(ctx, qI8, q_scale, kI8, k_scale, w, L, H_I, d_I,
+                                          row_begin, row_end, scores, ld, as_stream(stream));
+}
+
+extern "C" int ic_index_fp_fp8(ic_ctx* ctx, const uint8_t* qI8, const float* q_scale,
+                               const uint8_t* kI8, const float* k_scale, const void* w, int L,
+                               int H_I, int d_I, int k, int32_t* idx_out, void* stream) {
+    int rc = check_index_fp8_args(ctx, qI8, q_scale, kI8, k_scale, w, L, H_I, d_I);
+    if (rc) return rc;
+    if (!idx_out) return fail(ctx, IC_ERR_INVALID_ARG, "index_fp_fp8: idx_out is NULL");
+    if (k < 1 || k > 2048) return fail(ctx, IC_ERR_SHAPE, "index_fp_fp8: k=%d not in [1,2048]", k);
+    cudaSetDevice(ctx->device);
+    cudaStream_t s = as_stream(stream);
+    return index_fp_rows(ctx, L, k, idx_out, s, [&](int rb, int re, float* sc, int64_t ldc) {
+        return launch_index_score_prefill_fp8(ctx, qI8, q_scale, kI8, k_scale, w, L, H_I, d_I, rb,
+                                              re, sc, ldc, s);
+    });
 }
 
 extern "C" int ic_index_reuse(const int32_t* idx_cache, const int32_t** idx_out) {

@@ -82,6 +82,10 @@ int launch_index_score_decode(ic_ctx* ctx, const void* q, const void* w, const u
 int launch_topk(ic_ctx* ctx, const float* scores, int64_t ld, int rows, int k, int causal_base,
                 const int32_t* row_len, int max_len, int32_t* idx_out, int64_t ld_out,
                 cudaStream_t stream);
+int launch_index_score_prefill_fp8(ic_ctx* ctx, const uint8_t* qI8, const float* q_scale,
+                                   const uint8_t* kI8, const float* k_scale, const void* w, int L,
+                                   int H_I, int d_I, int row_begin, int row_end, float* scores,
+                                   int64_t ld, cudaStream_t stream);
 int launch_index_overlap(ic_ctx* ctx, const int32_t* a, const int32_t* b, int rows, int k,
                          int n_keys, int32_t* hits, cudaStream_t stream);
 int launch_sparse_attn(ic_ctx* ctx, const void* Q, const void* K, const void* V,

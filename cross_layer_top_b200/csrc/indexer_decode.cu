@@ -83,29 +83,6 @@ __device__ __forceinline__ float2 float2_of_e4m3x2(uint32_t pair16) {
     return __half22float2(*reinterpret_cast<const __half2*>(&h));
 }
 
-// Packed fp32 pairs (two lanes of one 64-bit register): one add / fma
-// instruction for two heads.
-__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
-    uint64_t r;
-    asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
-    return r;
-}
-__device__ __forceinline__ float2 f2_unpack(uint64_t v) {
-    float2 r;
-    asm("mov.b64 {%0, %1}, %2;" : "=f"(r.x), "=f"(r.y) : "l"(v));
-    return r;
-}
-__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
-    uint64_t d;
-    asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-    return d;
-}
-__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
-    uint64_t d;
-    asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
-    return d;
-}
-
 // The power of two 2^s that brings the largest |q| of a sequence (bf16 bit
 // pattern M of its magnitude) into [2^7, 2^8), clamped to normal floats.
 __device__ __forceinline__ int q_shift_of_max(uint32_t M) {

@@ -32,7 +32,9 @@
 
 namespace ic {
 
-template <int H_I, int NATOM>
+// F8: e4m3 q_I / k_I (d_I = 128, one 128-byte atom per row) on kind::f8f6f4
+// with per-(token, head) and per-token fp32 scales; otherwise bf16.
+template <int H_I, int NATOM, bool F8 = false>
 struct PrefillShape {
     static constexpr int BM = 128;                 // keys per tile (UMMA M, TMEM lanes)
     static constexpr int BN = 256;                 // (token, head) columns per accumulator
@@ -53,44 +55,22 @@ struct PrefillShape {
     static_assert(KSTAGES >= 2, "shared memory too small for the key ring");
     static_assert(SMEM <= SMEM_CAP, "shared memory budget");
     static_assert(64 % H_I == 0, "H_I must divide 64");
+    static_assert(!F8 || NATOM == 1, "e4m3 rows of d_I = 128 are one 128-byte atom");
 };
 
 // Score 64 consecutive accumulator columns held in va (cols 0..31) and vb
 // (cols 32..63); wcol points at the fp32 weights of those 64 columns
 // (token-major, head-minor, same order as the columns).  Produces one score
 // per token covered (64 / H_I tokens).
-template <int H_I>
-__device__ __forceinline__ void score64(const uint32_t (&va)[32], const uint32_t (&vb)[32],
-                                        const float* wcol, float (&out)[64 / H_I]) {
-    constexpr int NT = 64 / H_I;
-#pragma unroll
-    for (int tt = 0; tt < NT; ++tt) {
-        float p[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int j = 0; j < H_I; j += 4) {
-            const int c = tt * H_I + j;
-            const float4 wv = *reinterpret_cast<const float4*>(wcol + c);
-            const float x0 = __uint_as_float(c + 0 < 32 ? va[(c + 0) & 31] : vb[(c + 0) & 31]);
-            const float x1 = __uint_as_float(c + 1 < 32 ? va[(c + 1) & 31] : vb[(c + 1) & 31]);
-            const float x2 = __uint_as_float(c + 2 < 32 ? va[(c + 2) & 31] : vb[(c + 2) & 31]);
-            const float x3 = __uint_as_float(c + 3 < 32 ? va[(c + 3) & 31] : vb[(c + 3) & 31]);
-            p[0] = fmaf(wv.x, fmaxf(x0, 0.f), p[0]);
-            p[1] = fmaf(wv.y, fmaxf(x1, 0.f), p[1]);
-            p[2] = fmaf(wv.z, fmaxf(x2, 0.f), p[2]);
-            p[3] = fmaf(wv.w, fmaxf(x3, 0.f), p[3]);
-        }
-        out[tt] = (p[0] + p[1]) + (p[2] + p[3]);
-    }
-}
-
-template <int H_I, int NATOM>
+template <int H_I, int NATOM, bool F8>
 __global__ void __launch_bounds__(384, 1)
     k_index_score_prefill(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
-                          const __nv_bfloat16* __restrict__ w, float* __restrict__ scores,
+                          const __nv_bfloat16* __restrict__ w, const float* __restrict__ q_scale,
+                          const float* __restrict__ k_scale, float* __restrict__ scores,
                           long long ld, int L, int row_begin, int row_end, int n_items,
                           int* __restrict__ err) {
-    using S = PrefillShape<H_I, NATOM>;
+    using S = PrefillShape<H_I, NATOM, F8>;
     constexpr int KST = S::KSTAGES;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t* sB = smem;
@@ -190,7 +170,7 @@ __global__ void __launch_bounds__(384, 1)
         if (q_last >= 0) mbar_wait_drain(q_full, static_cast<uint32_t>(q_last));
     } else if (warp == 1 && lane == 0 && start_ok) {
         // ------------------------------------------------ MMA issuer
-        constexpr uint32_t IDESC = idesc_bf16_f32(S::BM, S::BN);
+        constexpr uint32_t IDESC = F8 ? idesc_e4m3_f32(S::BM, S::BN) : idesc_bf16_f32(S::BM, S::BN);
         int st = 0;
         uint32_t ph = 0, q_it = 0;
         uint32_t acc_it[2] = {0, 0};
@@ -228,7 +208,11 @@ __global__ void __launch_bounds__(384, 1)
                                 smem_u32(sA + st * S::A_STAGE + k * S::A_ATOM + kk * 32));
                             const uint64_t bd = sdesc_k_sw128(
                                 smem_u32(sB + a * S::B_ACC + k * S::B_ATOM + kk * 32));
-                            umma_bf16(d_tmem, ad, bd, IDESC, (k | kk) != 0 ? 1u : 0u);
+                            // K = 16 bf16 or 32 e4m3: 32 bytes of each row either way
+                            if (F8)
+                                umma_f8(d_tmem, ad, bd, IDESC, (k | kk) != 0 ? 1u : 0u);
+                            else
+                                umma_bf16(d_tmem, ad, bd, IDESC, (k | kk) != 0 ? 1u : 0u);
                         }
                     umma_commit(&acc_full[a]);
                     ++acc_it[a];
@@ -259,7 +243,9 @@ __global__ void __launch_bounds__(384, 1)
             const int t0 = row_begin + (n_items - 1 - it) * S::TQ;
             const int t_last = min(t0 + S::TQ, row_end) - 1;
             const int n_tiles = t_last / S::BM + 1;
-            // weights of this warp's columns, widened to fp32 (private copy)
+            // weights of this warp's columns, widened to fp32 (private copy);
+            // e4m3 inputs fold the query's (token, head) scale in: it is > 0,
+            // so it commutes with ReLU
             __syncwarp();
 #pragma unroll
             for (int a = 0; a < 2; ++a) {
@@ -268,13 +254,17 @@ __global__ void __launch_bounds__(384, 1)
                 for (int q = 0; q < 4; ++q) {
                     const int c = lane * 4 + q;  // column within the half
                     const int t = tok0 + c / H_I;
-                    wW[a * 128 + c] =
-                        t < L ? __bfloat162float(w[static_cast<size_t>(t) * H_I + (c % H_I)]) : 0.f;
+                    const size_t wi = static_cast<size_t>(t) * H_I + (c % H_I);
+                    float wv = t < L ? __bfloat162float(w[wi]) : 0.f;
+                    if (F8 && t < L) wv *= q_scale[wi];
+                    wW[a * 128 + c] = wv;
                 }
             }
             __syncwarp();
             for (int kt = 0; kt < n_tiles && ok; ++kt) {
                 const int s = kt * S::BM + lq * 32 + lane;
+                // the key's scale (e4m3 inputs), applied after the head sum
+                const float ks = F8 ? (s < L ? __ldg(k_scale + s) : 0.f) : 1.f;
 #pragma unroll
                 for (int a = 0; a < 2; ++a) {
                     bool got = mbar_wait(&acc_full[a], acc_it[a] & 1, abort_flag, err,
@@ -289,25 +279,46 @@ __global__ void __launch_bounds__(384, 1)
                     const uint32_t taddr = tmem + (static_cast<uint32_t>(lq * 32) << 16) +
                                            static_cast<uint32_t>(a * S::BN + cg * 128);
                     const int tok_base = a * S::TOK_PER_ACC + cg * TOK_PER_HALF;
-                    uint32_t va[32], vb[32];
-                    float sc[64 / H_I];
+                    const float* wa = wW + a * 128;
+                    // 32-column chunks: chunk c + 1 is loaded while chunk c is
+                    // scored.  Four partial sums per token (heads 0, 1, 2, 3
+                    // mod 4) as two packed pairs; a token's score is stored as
+                    // soon as its last head is in.
+                    uint32_t buf[2][32];
+                    tmem_ld32(taddr, buf[0]);
+                    tmem_ld_wait();
+                    uint64_t p01 = 0, p23 = 0;
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        tmem_ld32(taddr + h * 64, va);
-                        tmem_ld32(taddr + h * 64 + 32, vb);
-                        tmem_ld_wait();
-                        if (h == 1) {
-                            // all of this accumulator is in registers: hand it back
-                            tc_fence_before();
-                            __syncwarp();
-                            if (lane == 0) mbar_arrive(&acc_empty[a]);
+                    for (int c = 0; c < 4; ++c) {
+                        if (c < 3) tmem_ld32(taddr + (c + 1) * 32, buf[(c + 1) & 1]);
+                        const uint32_t(&v)[32] = buf[c & 1];
+#pragma unroll
+                        for (int j = 0; j < 32; j += 4) {
+                            const int col = c * 32 + j;
+                            const ulonglong2 wv = *reinterpret_cast<const ulonglong2*>(wa + col);
+                            p01 = f2_fma(wv.x, f2_pack(fmaxf(__uint_as_float(v[j]), 0.f),
+                                                       fmaxf(__uint_as_float(v[j + 1]), 0.f)), p01);
+                            p23 = f2_fma(wv.y, f2_pack(fmaxf(__uint_as_float(v[j + 2]), 0.f),
+                                                       fmaxf(__uint_as_float(v[j + 3]), 0.f)), p23);
+                            if ((col + 4) % H_I == 0) {
+                                const float2 x = f2_unpack(p01), y = f2_unpack(p23);
+                                const float sc = (x.x + x.y) + (y.x + y.y);
+                                const int t = t0 + tok_base + col / H_I;
+                                if (t < row_end && s <= t)
+                                    scores[static_cast<long long>(t - row_begin) * ld + s] =
+                                        F8 ? sc * ks : sc;
+                                p01 = 0;
+                                p23 = 0;
+                            }
                         }
-                        score64<H_I>(va, vb, wW + a * 128 + h * 64, sc);
-#pragma unroll
-                        for (int tt = 0; tt < 64 / H_I; ++tt) {
-                            const int t = t0 + tok_base + h * (64 / H_I) + tt;
-                            if (t < row_end && s <= t)
-                                scores[static_cast<long long>(t - row_begin) * ld + s] = sc[tt];
+                        if (c < 3) {
+                            tmem_ld_wait();
+                            if (c == 2) {
+                                // all of this accumulator is in registers: hand it back
+                                tc_fence_before();
+                                __syncwarp();
+                                if (lane == 0) mbar_arrive(&acc_empty[a]);
+                            }
                         }
                     }
                 }
@@ -323,12 +334,13 @@ __global__ void __launch_bounds__(384, 1)
     }
 }
 
-template <int H_I, int NATOM>
-static int launch_prefill_t(ic_ctx* ctx, const void* qI, const void* kI, const void* w, int L,
-                            int d_I, int row_begin, int row_end, float* scores, int64_t ld,
+template <int H_I, int NATOM, bool F8>
+static int launch_prefill_t(ic_ctx* ctx, const void* qI, const void* kI, const void* w,
+                            const float* q_scale, const float* k_scale, int L, int d_I,
+                            int row_begin, int row_end, float* scores, int64_t ld,
                             cudaStream_t stream) {
-    using S = PrefillShape<H_I, NATOM>;
-    auto kern = k_index_score_prefill<H_I, NATOM>;
+    using S = PrefillShape<H_I, NATOM, F8>;
+    auto kern = k_index_score_prefill<H_I, NATOM, F8>;
     static bool attr_set = false;
     if (!attr_set) {
         cudaError_t e =
@@ -337,16 +349,23 @@ static int launch_prefill_t(ic_ctx* ctx, const void* qI, const void* kI, const v
         attr_set = true;
     }
     CUtensorMap tm_q, tm_k;
-    int rc = make_tmap_bf16_2d(ctx, &tm_q, qI, static_cast<uint64_t>(L) * H_I, d_I, S::BN);
-    if (rc) return rc;
-    rc = make_tmap_bf16_2d(ctx, &tm_k, kI, static_cast<uint64_t>(L), d_I, S::BM);
+    int rc;
+    if (F8) {
+        rc = make_tmap_u8_2d(ctx, &tm_q, qI, static_cast<uint64_t>(L) * H_I, d_I, 128, S::BN, true);
+        if (rc) return rc;
+        rc = make_tmap_u8_2d(ctx, &tm_k, kI, static_cast<uint64_t>(L), d_I, 128, S::BM, true);
+    } else {
+        rc = make_tmap_bf16_2d(ctx, &tm_q, qI, static_cast<uint64_t>(L) * H_I, d_I, S::BN);
+        if (rc) return rc;
+        rc = make_tmap_bf16_2d(ctx, &tm_k, kI, static_cast<uint64_t>(L), d_I, S::BM);
+    }
     if (rc) return rc;
     const int n_items = (row_end - row_begin + S::TQ - 1) / S::TQ;
     const int grid = n_items < ctx->num_sms ? n_items : ctx->num_sms;
     LaunchScope ls(ctx, IC_K_INDEX_SCORE, stream);
-    k_index_score_prefill<H_I, NATOM><<<grid, 384, S::SMEM, stream>>>(
-        tm_q, tm_k, static_cast<const __nv_bfloat16*>(w), scores, static_cast<long long>(ld), L,
-        row_begin, row_end, n_items, ctx->dev_err);
+    kern<<<grid, 384, S::SMEM, stream>>>(tm_q, tm_k, static_cast<const __nv_bfloat16*>(w), q_scale,
+                                         k_scale, scores, static_cast<long long>(ld), L, row_begin,
+                                         row_end, n_items, ctx->dev_err);
     cudaError_t e = ls.done();
     if (e != cudaSuccess) return cuda_fail(ctx, e, "index_score launch");
     return IC_OK;
@@ -359,10 +378,12 @@ int launch_index_score_prefill(ic_ctx* ctx, const void* qI, const void* kI, cons
     const bool one_atom = d_I <= 64;
 #define IC_PREFILL_CASE(H)                                                                      \
     case H:                                                                                     \
-        return one_atom ? launch_prefill_t<H, 1>(ctx, qI, kI, w, L, d_I, row_begin, row_end,    \
-                                                 scores, ld, stream)                            \
-                        : launch_prefill_t<H, 2>(ctx, qI, kI, w, L, d_I, row_begin, row_end,    \
-                                                 scores, ld, stream);
+        return one_atom ? launch_prefill_t<H, 1, false>(ctx, qI, kI, w, nullptr, nullptr, L,    \
+                                                        d_I, row_begin, row_end, scores, ld,    \
+                                                        stream)                                 \
+                        : launch_prefill_t<H, 2, false>(ctx, qI, kI, w, nullptr, nullptr, L,    \
+                                                        d_I, row_begin, row_end, scores, ld,    \
+                                                        stream);
     switch (H_I) {
         IC_PREFILL_CASE(4)
         IC_PREFILL_CASE(8)
@@ -373,6 +394,28 @@ int launch_index_score_prefill(ic_ctx* ctx, const void* qI, const void* kI, cons
             return fail(ctx, IC_ERR_UNSUPPORTED, "index_score: H_I=%d not in {4,8,16,32,64}", H_I);
     }
 #undef IC_PREFILL_CASE
+}
+
+int launch_index_score_prefill_fp8(ic_ctx* ctx, const uint8_t* qI8, const float* q_scale,
+                                   const uint8_t* kI8, const float* k_scale, const void* w, int L,
+                                   int H_I, int d_I, int row_begin, int row_end, float* scores,
+                                   int64_t ld, cudaStream_t stream) {
+    if (row_end <= row_begin) return IC_OK;
+    if (d_I != 128)
+        return fail(ctx, IC_ERR_UNSUPPORTED, "index_score_fp8: d_I=%d (need 128)", d_I);
+    switch (H_I) {
+        case 16:
+            return launch_prefill_t<16, 1, true>(ctx, qI8, kI8, w, q_scale, k_scale, L, d_I,
+                                                 row_begin, row_end, scores, ld, stream);
+        case 32:
+            return launch_prefill_t<32, 1, true>(ctx, qI8, kI8, w, q_scale, k_scale, L, d_I,
+                                                 row_begin, row_end, scores, ld, stream);
+        case 64:
+            return launch_prefill_t<64, 1, true>(ctx, qI8, kI8, w, q_scale, k_scale, L, d_I,
+                                                 row_begin, row_end, scores, ld, stream);
+        default:
+            return fail(ctx, IC_ERR_UNSUPPORTED, "index_score_fp8: H_I=%d not in {16,32,64}", H_I);
+    }
 }
 
 }  // namespace ic

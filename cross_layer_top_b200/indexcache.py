@@ -82,6 +82,8 @@ _SIGS = {
     "ic_probe_gather": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp], _i),
     "ic_sparse_attn": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64, _i, _f, _vp, _vp], _i),
     "ic_index_overlap": ([_vp, _vp, _vp, _i, _i, _i, _vp, _vp], _i),
+    "ic_index_score_fp8": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _i64, _vp], _i),
+    "ic_index_fp_fp8": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp], _i),
     "ic_probe_wait_timeout": ([_vp, _vp], _i),
     "ic_run_stack": ([_vp, _vp, ctypes.POINTER(ic_layer_io), ctypes.POINTER(ic_stack_dims), _vp,
                       _vp], _i),
@@ -296,6 +298,32 @@ def ic_sparse_attn(ctx: Context, Q, K, V, idx, out, rows_per_seq: int = 0, kv_se
     _check(_lib.ic_sparse_attn(ctx.handle, _ptr(Q), _ptr(K), _ptr(V), _ptr(idx), rows, Hq, d, k,
                                rows_per_seq, kv_seq_stride, kv_len, scale, _ptr(out),
                                _stream(stream)), ctx)
+
+
+def ic_index_score_fp8(ctx: Context, qI8, q_scale, kI8, k_scale, w, row_begin: int, row_end: int,
+                       scores, ld=None, stream=None):
+    """FP8 indexer scores: qI8 uint8 (e4m3 bytes) [L, H_I, d_I], q_scale f32
+    [L, H_I], kI8 uint8 [L, d_I], k_scale f32 [L], w bf16 [L, H_I]."""
+    L, H_I, d_I = qI8.shape
+    for t, dt, n in ((qI8, torch.uint8, "qI8"), (kI8, torch.uint8, "kI8"),
+                     (q_scale, torch.float32, "q_scale"), (k_scale, torch.float32, "k_scale"),
+                     (w, torch.bfloat16, "w"), (scores, torch.float32, "scores")):
+        _dev_tensor(t, dt, n)
+    ld = scores.shape[-1] if ld is None else ld
+    _check(_lib.ic_index_score_fp8(ctx.handle, _ptr(qI8), _ptr(q_scale), _ptr(kI8), _ptr(k_scale),
+                                   _ptr(w), L, H_I, d_I, row_begin, row_end, _ptr(scores), ld,
+                                   _stream(stream)), ctx)
+
+
+def ic_index_fp_fp8(ctx: Context, qI8, q_scale, kI8, k_scale, w, k: int, idx_out, stream=None):
+    """FP8 prefill F layer: scores + top-k into idx_out int32 [L, k]."""
+    L, H_I, d_I = qI8.shape
+    for t, dt, n in ((qI8, torch.uint8, "qI8"), (kI8, torch.uint8, "kI8"),
+                     (q_scale, torch.float32, "q_scale"), (k_scale, torch.float32, "k_scale"),
+                     (w, torch.bfloat16, "w"), (idx_out, torch.int32, "idx_out")):
+        _dev_tensor(t, dt, n)
+    _check(_lib.ic_index_fp_fp8(ctx.handle, _ptr(qI8), _ptr(q_scale), _ptr(kI8), _ptr(k_scale),
+                                _ptr(w), L, H_I, d_I, k, _ptr(idx_out), _stream(stream)), ctx)
 
 
 def ic_index_overlap(ctx: Context, idx_a, idx_b, hits, n_keys: int, stream=None):

@@ -149,6 +149,17 @@ def fp8_e4m3_quantize_per_token(x: torch.Tensor):
     return q.view(torch.uint8), scale
 
 
+def prefill_indexer_fp8(cfg: PrefillConfig, layer: int, device="cpu"):
+    """The indexer inputs of ``prefill_layer`` (same draw) prepared for the
+    FP8 indexer: q_I in e4m3 with one fp32 scale per (token, head), k_I in
+    e4m3 with one per token (amax/448 each), w unchanged."""
+    lay = prefill_layer(cfg, layer, device, indexer=True)
+    qI8, q_scale = fp8_e4m3_quantize_per_token(lay["qI"].float())
+    kI8, k_scale = fp8_e4m3_quantize_per_token(lay["kI"].float())
+    return {"qI8": qI8.contiguous(), "q_scale": q_scale.contiguous(), "kI8": kI8.contiguous(),
+            "k_scale": k_scale.contiguous(), "w": lay["w"]}
+
+
 def decode_layer(cfg: DecodeConfig, layer: int, device="cpu", indexer: bool | None = None,
                  batch=None):
     """Tensors of one decode layer (one step).  'q','w','kI8','kI_scale' only

@@ -148,6 +148,27 @@ int ic_topk(ic_ctx *ctx, const float *scores, int64_t ld, int rows, int k, int c
 int ic_index_fp(ic_ctx *ctx, const void *qI, const void *kI, const void *w, int L, int H_I,
                 int d_I, int k, int32_t *idx_out, void *stream);
 
+/* FP8 prefill indexer ([IC] §2.1: the lightning indexer runs in FP8).  The
+ * same score as ic_index_score on dequantised inputs:
+ *   I[t,s] = sum_j w[t,j] * ReLU((e4m3(qI8[t,j,:]) q_scale[t,j])
+ *                                 . (e4m3(kI8[s,:]) k_scale[s]))
+ *          = k_scale[s] * sum_j (w[t,j] q_scale[t,j]) * ReLU(e4m3(qI8[t,j,:]) . e4m3(kI8[s,:]))
+ * (the scales must be > 0, which makes the two forms equal).  The products of
+ * e4m3 values are exact and accumulate in fp32 on the tensor cores
+ * (kind::f8f6f4).
+ *   qI8: e4m3 bytes [L, H_I, d_I]; q_scale: fp32 [L, H_I] (> 0);
+ *   kI8: e4m3 bytes [L, d_I];      k_scale: fp32 [L] (> 0);  w: bf16 [L, H_I].
+ *   scores: fp32, ld >= row_end, ld % 4 == 0.
+ * Supported: H_I in {16,32,64}, d_I = 128.  Errors as ic_index_score. */
+int ic_index_score_fp8(ic_ctx *ctx, const uint8_t *qI8, const float *q_scale, const uint8_t *kI8,
+                       const float *k_scale, const void *w, int L, int H_I, int d_I, int row_begin,
+                       int row_end, float *scores, int64_t ld, void *stream);
+
+/* FP8 prefill F layer: ic_index_fp on the scores of ic_index_score_fp8. */
+int ic_index_fp_fp8(ic_ctx *ctx, const uint8_t *qI8, const float *q_scale, const uint8_t *kI8,
+                    const float *k_scale, const void *w, int L, int H_I, int d_I, int k,
+                    int32_t *idx_out, void *stream);
+
 /* S layer ([IC] Figure 2 "T <- cache"): the cached tensor itself is used, no
  * copy and no kernel.  *idx_out = idx_cache. */
 int ic_index_reuse(const int32_t *idx_cache, const int32_t **idx_out);

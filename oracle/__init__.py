@@ -49,6 +49,9 @@ def lib():
         L.oracle_e4m3_to_double.restype = ctypes.c_double
         L.oracle_decode_scores.argtypes = [_f32p, _f32p, _u8p, _f32p, ctypes.c_int, ctypes.c_int,
                                            ctypes.c_int, _f64p]
+        L.oracle_index_scores_fp8.argtypes = [_u8p, _f32p, _u8p, _f32p, _f32p, ctypes.c_int,
+                                              ctypes.c_int, ctypes.c_int, _i32p, ctypes.c_int,
+                                              _f64p, ctypes.c_int64]
         L.oracle_topk_row.argtypes = [_f64p, ctypes.c_int, ctypes.c_int, _i32p]
         L.oracle_kth_score.argtypes = [_f64p, ctypes.c_int, ctypes.c_int]
         L.oracle_kth_score.restype = ctypes.c_double
@@ -152,6 +155,25 @@ def decode_scores(q, w, kq, kscale, S=None):
     out = np.empty(S, dtype=np.float64)
     lib().oracle_decode_scores(_p(q, _f32p), _p(w, _f32p), _p(kq, _u8p), _p(kscale, _f32p),
                                S, H, d, _p(out, _f64p))
+    return out
+
+
+def index_scores_fp8(q8, q_scale, k8, k_scale, w, rows=None):
+    """FP8 prefill scores (IndexCache paper §2.1, FP8 indexer) on the
+    dequantised inputs: q8 uint8 [L, H, d] e4m3 bytes with q_scale [L, H],
+    k8 uint8 [L, d] with k_scale [L], w [L, H].  Returns float64
+    [nrows, L] with NaN where s > t."""
+    q8 = _c(q8, np.uint8)
+    k8 = _c(k8, np.uint8)
+    q_scale = _c(q_scale, np.float32)
+    k_scale = _c(k_scale, np.float32)
+    w = _c(w, np.float32)
+    L, H, d = q8.shape
+    rows = np.arange(L, dtype=np.int32) if rows is None else _c(rows, np.int32)
+    out = np.full((len(rows), L), np.nan, dtype=np.float64)
+    lib().oracle_index_scores_fp8(_p(q8, _u8p), _p(q_scale, _f32p), _p(k8, _u8p),
+                                  _p(k_scale, _f32p), _p(w, _f32p), L, H, d, _p(rows, _i32p),
+                                  len(rows), _p(out, _f64p), L)
     return out
 
 

@@ -171,6 +171,43 @@ void oracle_decode_scores(const float *q, const float *w, const uint8_t *kq, con
     }
 }
 
+/* FP8 prefill scores ([IC] §2.1: the lightning indexer in FP8): the [RN]
+ * §2.1 score on the dequantised inputs
+ *   q[t,j,e] = e4m3(q8[t,j,e]) * q_scale[t,j],  k[s,e] = e4m3(k8[s,e]) * k_scale[s],
+ * everything in double.  Query rows rows[r] (0 <= rows[r] < L); out[r*ld + s]
+ * for s <= rows[r].  d <= 1024. */
+void oracle_index_scores_fp8(const uint8_t *q8, const float *q_scale, const uint8_t *k8,
+                             const float *k_scale, const float *w, int L, int H, int d,
+                             const int32_t *rows, int nrows, double *out, int64_t ld)
+{
+    int r;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (r = 0; r < nrows; ++r) {
+        int t = rows[r];
+        if (t < 0 || t >= L)
+            continue;
+        double *qd = (double *)malloc(sizeof(double) * (size_t)H * d);
+        for (int j = 0; j < H; ++j)
+            for (int e = 0; e < d; ++e)
+                qd[(size_t)j * d + e] = oracle_e4m3_to_double(q8[((size_t)t * H + j) * d + e]) *
+                                        (double)q_scale[(size_t)t * H + j];
+        for (int s = 0; s <= t; ++s) {
+            double kd[1024];
+            for (int e = 0; e < d; ++e)
+                kd[e] = oracle_e4m3_to_double(k8[(size_t)s * d + e]) * (double)k_scale[s];
+            double total = 0.0;
+            for (int j = 0; j < H; ++j) {
+                double dot = 0.0;
+                for (int e = 0; e < d; ++e)
+                    dot += qd[(size_t)j * d + e] * kd[e];
+                total += (double)w[(size_t)t * H + j] * (dot > 0.0 ? dot : 0.0);
+            }
+            out[(size_t)r * ld + s] = total;
+        }
+        free(qd);
+    }
+}
+
 /* ------------------------------------------------------------------------
  * Top-k ([IC] notation: T_t = Top-k(I_t), k = 2048): full sort of the n
  * candidates by (score descending, index ascending), keep the first

@@ -173,6 +173,72 @@ def test_integer_scores_are_exact_multiples_of_half():
     assert np.max(np.abs(v)) <= H * d * 9
 
 
+def _e4m3_int(v):
+    """e4m3 byte of an integer with |v| <= 16."""
+    v = int(v)
+    if v == 0:
+        return 0
+    a = abs(v)
+    e = a.bit_length() - 1
+    m = (a - (1 << e)) * 8 >> e
+    return (0x80 if v < 0 else 0) | ((e + 7) << 3) | m
+
+
+def test_fp8_scores_hand_example():
+    # q = [1.5, -2] * 2 = [3, -4]; k0 = [2, 0.5] * 0.5 = [1, 0.25]; k1 = [-2, 1] * 1
+    q8 = np.array([[[0x3C, 0xC0]], [[0x3C, 0xC0]]], np.uint8)
+    q_scale = np.array([[2.0], [2.0]], np.float32)
+    k8 = np.array([[0x40, 0x30], [0xC0, 0x38]], np.uint8)
+    k_scale = np.array([0.5, 1.0], np.float32)
+    w = np.array([[0.5], [0.5]], np.float32)
+    I = oracle.index_scores_fp8(q8, q_scale, k8, k_scale, w)
+    assert I[0, 0] == 0.5 * (3 * 1 - 4 * 0.25)      # 1.0
+    assert I[1, 0] == 1.0
+    assert I[1, 1] == 0.0                          # 3*-2 - 4*1 < 0: ReLU
+    assert np.isnan(I[0, 1])
+
+
+def test_fp8_scores_equal_bf16_scores_on_integer_values():
+    rng = np.random.default_rng(12)
+    L, H, d = 21, 4, 16
+    qi = rng.integers(-16, 17, (L, H, d))
+    ki = rng.integers(-16, 17, (L, d))
+    w = rng.choice([-1.0, -0.5, 0.5, 1.0], (L, H)).astype(np.float32)
+    enc = np.vectorize(_e4m3_int)
+    I8 = oracle.index_scores_fp8(enc(qi).astype(np.uint8), np.ones((L, H), np.float32),
+                                 enc(ki).astype(np.uint8), np.ones(L, np.float32), w)
+    I16 = oracle.index_scores(qi.astype(np.float32), ki.astype(np.float32), w)
+    tri = np.tril(np.ones((L, L), bool))
+    assert np.array_equal(I8[tri], I16[tri])
+
+
+def test_fp8_scores_scale_laws():
+    rng = np.random.default_rng(13)
+    L, H, d = 17, 3, 8
+    q8 = rng.integers(0, 0x7E, (L, H, d)).astype(np.uint8) | (rng.integers(0, 2, (L, H, d)) << 7).astype(np.uint8)
+    k8 = rng.integers(0, 0x7E, (L, d)).astype(np.uint8)
+    qs = rng.uniform(0.5, 2.0, (L, H)).astype(np.float32)
+    ks = rng.uniform(0.5, 2.0, L).astype(np.float32)
+    w = rng.standard_normal((L, H)).astype(np.float32)
+    I = oracle.index_scores_fp8(q8, qs, k8, ks, w)
+    tri = np.tril(np.ones((L, L), bool))
+    # a key's scale multiplies its column (power of two: exact)
+    ks2 = ks.copy()
+    ks2[5] *= 4
+    I2 = oracle.index_scores_fp8(q8, qs, k8, ks2, w)
+    assert np.array_equal(I2[5:, 5], 4 * I[5:, 5])
+    assert np.array_equal(np.delete(I2, 5, axis=1)[np.delete(tri, 5, axis=1)],
+                          np.delete(I, 5, axis=1)[np.delete(tri, 5, axis=1)])
+    # a query head's scale and its weight are interchangeable (both > 0 factors)
+    qs3, w3 = qs.copy(), w.copy()
+    qs3[:, 1] *= 2
+    w3[:, 1] *= 2
+    A = oracle.index_scores_fp8(q8, qs3, k8, ks, w)
+    B = oracle.index_scores_fp8(q8, qs, k8, ks, w3)
+    assert np.allclose(A[tri], B[tri], rtol=1e-12, atol=1e-12)
+    assert not np.allclose(A[tri], I[tri])
+
+
 # ------------------------------------------------------------------- top-k
 def test_topk_page_toy(golden):
     g = golden["topk_average_toy"]
