@@ -501,8 +501,9 @@ extern "C" int ic_sparse_attn(ic_ctx* ctx, const void* Q, const void* K, const v
         return fail(ctx, IC_ERR_UNSUPPORTED, "sparse_attn: kv_len=%d above 2^24", kv_len);
     if (rows == 0) return IC_OK;
     if (!Q || !K || !V || !idx || !out) return fail(ctx, IC_ERR_INVALID_ARG, "sparse_attn: NULL");
-    if (!aligned16(Q) || !aligned16(K) || !aligned16(V))
-        return fail(ctx, IC_ERR_INVALID_ARG, "sparse_attn: Q, K, V must be 16-byte aligned");
+    if (!aligned16(Q) || !aligned16(K) || !aligned16(V) || (reinterpret_cast<uintptr_t>(out) & 7u))
+        return fail(ctx, IC_ERR_INVALID_ARG,
+                    "sparse_attn: Q, K, V must be 16-byte and out 8-byte aligned");
     if (scale <= 0.f) scale = 1.0f / sqrtf(static_cast<float>(d));
     cudaSetDevice(ctx->device);
     return launch_sparse_attn(ctx, Q, K, V, idx, rows, Hq, d, k, rows_per_seq, kv_seq_stride,

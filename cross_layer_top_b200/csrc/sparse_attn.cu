@@ -50,7 +50,8 @@ struct AttnShape {
     static constexpr int OFF_LAST = OFF_IDX + MAXK * 4;
     static constexpr int OFF_ST = OFF_LAST + 128;
     static constexpr int SMEM = OFF_ST + WARPS * WARP_BYTES;
-    static constexpr int MERGE_BYTES = WARPS * (16 * D + 32) * 4;
+    // per-warp O and (m, l), then the per-head factors, M and L
+    static constexpr int MERGE_BYTES = WARPS * (16 * D + 32) * 4 + (WARPS * 16 + 32) * 4;
     static constexpr float kRescaleThreshold = 8.0f;  // log2 units
     static_assert(MERGE_BYTES <= WARPS * WARP_BYTES, "merge buffer must fit in the stages");
 };
@@ -275,30 +276,51 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
         }
     }
     __syncthreads();
-    const int hmax = nsplit == 1 ? Hq : 16;
-    for (int e = tid; e < hmax * D; e += S::THREADS) {
-        const int h = e / D, dd = e % D;
+    // combine the warps: per head M = max_w m_w, factors f_w = 2^(m_w - M),
+    // L = sum_w l_w f_w (computed once per head), then o = sum_w O_w f_w
+    // over float4 columns
+    float* sF = mML + S::WARPS * 32;  // [WARPS][16] factors, then M[16], L[16]
+    if (tid < 16) {
+        const int h = tid;
         float M = -INFINITY;
 #pragma unroll
         for (int w = 0; w < S::WARPS; ++w) M = fmaxf(M, mML[w * 32 + h]);
-        float acc = 0.f, lsum = 0.f;
-        if (M != -INFINITY) {
+        float L = 0.f;
 #pragma unroll
-            for (int w = 0; w < S::WARPS; ++w) {
-                const float f = ex2_approx(mML[w * 32 + h] - M);
-                acc += mO[w * 16 * D + h * D + dd] * f;
-                lsum += mML[w * 32 + 16 + h] * f;
-            }
+        for (int w = 0; w < S::WARPS; ++w) {
+            const float f = M == -INFINITY ? 0.f : ex2_approx(mML[w * 32 + h] - M);
+            sF[w * 16 + h] = f;
+            L += mML[w * 32 + 16 + h] * f;
         }
+        sF[S::WARPS * 16 + h] = M;
+        sF[S::WARPS * 16 + 16 + h] = L;
+    }
+    __syncthreads();
+    const int hmax = nsplit == 1 ? Hq : 16;
+    for (int e4 = tid; e4 < hmax * (D / 4); e4 += S::THREADS) {
+        const int h = e4 / (D / 4), d4 = (e4 % (D / 4)) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int w = 0; w < S::WARPS; ++w) {
+            const float f = sF[w * 16 + h];
+            const float4 v = *reinterpret_cast<const float4*>(mO + w * 16 * D + h * D + d4);
+            acc.x = fmaf(v.x, f, acc.x);
+            acc.y = fmaf(v.y, f, acc.y);
+            acc.z = fmaf(v.z, f, acc.z);
+            acc.w = fmaf(v.w, f, acc.w);
+        }
+        const float L = sF[S::WARPS * 16 + 16 + h];
         if (nsplit == 1) {
-            const float v = lsum > 0.f ? acc / lsum : 0.f;
-            out[(static_cast<long long>(r) * Hq + h) * D + dd] = __float2bfloat16_rn(v);
+            const float iv = L > 0.f ? 1.f / L : 0.f;
+            __nv_bfloat16* op = out + (static_cast<long long>(r) * Hq + h) * D + d4;
+            *reinterpret_cast<uint2*>(op) = make_uint2(pack_bf16x2(acc.x * iv, acc.y * iv),
+                                                       pack_bf16x2(acc.z * iv, acc.w * iv));
         } else {
             float* pr = part + (static_cast<long long>(r) * nsplit + split) * (16 * D + 32);
-            pr[h * D + dd] = acc;
-            if (dd == 0) {
-                pr[16 * D + h] = M;
-                pr[16 * D + 16 + h] = lsum;
+            *reinterpret_cast<float4*>(pr + h * D + d4) = acc;
+            if (d4 == 0) {
+                pr[16 * D + h] = sF[S::WARPS * 16 + h];
+                pr[16 * D + 16 + h] = L;
             }
         }
     }

@@ -220,7 +220,8 @@ int ic_index_fp_decode_noalloc(const void *q, const void *w, const uint8_t *kI8,
  * [kv_len, d].  One shared K/V head.  Entries -1 are skipped; an entry
  * outside [-1, kv_len) is skipped and latched as IC_ERR_DEVICE.  A row with
  * no valid entry produces zeros.  scale <= 0 means 1/sqrt(d).
- * Supported: d in {64,128}, 1 <= Hq <= 16, 1 <= k <= 2048. */
+ * Supported: d in {64,128}, 1 <= Hq <= 16, 1 <= k <= 2048.  Q, K, V 16-byte
+ * aligned, out 8-byte aligned (else IC_ERR_INVALID_ARG). */
 int ic_sparse_attn(ic_ctx *ctx, const void *Q, const void *K, const void *V, const int32_t *idx,
                    int rows, int Hq, int d, int k, int rows_per_seq, int64_t kv_seq_stride,
                    int kv_len, float scale, void *out, void *stream);
