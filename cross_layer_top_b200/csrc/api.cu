@@ -162,7 +162,6 @@ extern "C" int ic_ctx_destroy(ic_ctx* ctx) {
     cudaSetDevice(ctx->device);
     cudaDeviceSynchronize();
     cudaFree(ctx->scores);
-    cudaFree(ctx->attn_part);
     cudaFree(ctx->dev_err);
     for (auto& p : ctx->pool) {
         cudaEventDestroy(p.start);

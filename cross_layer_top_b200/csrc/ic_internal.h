@@ -16,8 +16,6 @@ struct ic_ctx {
     size_t scratch_limit = 0;       // bound on the prefill score scratch (bytes)
     float* scores = nullptr;        // score scratch (fp32 rows)
     size_t scores_cap = 0;          // bytes
-    float* attn_part = nullptr;     // split-attention partials
-    size_t attn_part_cap = 0;       // bytes
     int* dev_err = nullptr;         // device error word (first error wins)
     std::string last_error;
     bool timing = false;

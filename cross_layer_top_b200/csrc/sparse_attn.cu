@@ -51,7 +51,8 @@ struct AttnShape {
     static constexpr int OFF_ST = OFF_LAST + 128;
     static constexpr int SMEM = OFF_ST + WARPS * WARP_BYTES;
     // per-warp O and (m, l), then the per-head factors, M and L
-    static constexpr int MERGE_BYTES = WARPS * (16 * D + 32) * 4 + (WARPS * 16 + 32) * 4;
+    static constexpr int MERGE_BYTES = WARPS * (16 * D + 32) * 4 + (WARPS * 16 + 32) * 4 +
+                                       (16 * D + 16 * 32 + 16 * 16 + 16) * 4;  // split rows
     static constexpr float kRescaleThreshold = 8.0f;  // log2 units
     static_assert(MERGE_BYTES <= WARPS * WARP_BYTES, "merge buffer must fit in the stages");
 };
@@ -59,18 +60,21 @@ struct AttnShape {
 // byte offset of 16-byte piece c of row `row` in a [rows][d] bf16 tile whose
 // pieces are XOR-swizzled by (row mod 8): ldmatrix reads 8 rows of one piece
 // column from 8 different bank groups
+constexpr int kMaxClusterSplits = 16;  // CTAs of one split row's cluster, at most
+
 template <int D>
 __device__ __forceinline__ uint32_t swz(int row, int c) {
     return static_cast<uint32_t>(row * (D * 2) + ((c ^ (row & 7)) << 4));
 }
 
-template <int D>
-__global__ void __launch_bounds__(AttnShape<D>::THREADS)
+// SPLIT: rows split across a cluster of CTAs (few rows, decode); otherwise
+// one CTA per row, and the cluster merge is not compiled in.
+template <int D, bool SPLIT>
+__global__ void __launch_bounds__(AttnShape<D>::THREADS, 2)
     k_sparse_attn(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
                   const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ idx, int Hq,
                   int k, int rows_per_seq, long long kv_seq_stride, int kv_len, float scale_log2,
-                  int nsplit, int kps, __nv_bfloat16* __restrict__ out,
-                  float* __restrict__ part, int* __restrict__ row_done, int* __restrict__ err) {
+                  int nsplit, int kps, __nv_bfloat16* __restrict__ out, int* __restrict__ err) {
     using S = AttnShape<D>;
     extern __shared__ __align__(128) uint8_t smem[];
     const int r = blockIdx.x, split = blockIdx.y;
@@ -280,6 +284,7 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
     // L = sum_w l_w f_w (computed once per head), then o = sum_w O_w f_w
     // over float4 columns
     float* sF = mML + S::WARPS * 32;  // [WARPS][16] factors, then M[16], L[16]
+    float* pO = sF + S::WARPS * 16 + 32;  // split rows: this CTA's combined O [16][D]
     if (tid < 16) {
         const int h = tid;
         float M = -INFINITY;
@@ -296,7 +301,7 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
         sF[S::WARPS * 16 + 16 + h] = L;
     }
     __syncthreads();
-    const int hmax = nsplit == 1 ? Hq : 16;
+    const int hmax = SPLIT ? 16 : Hq;
     for (int e4 = tid; e4 < hmax * (D / 4); e4 += S::THREADS) {
         const int h = e4 / (D / 4), d4 = (e4 % (D / 4)) * 4;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -310,74 +315,65 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS)
             acc.w = fmaf(v.w, f, acc.w);
         }
         const float L = sF[S::WARPS * 16 + 16 + h];
-        if (nsplit == 1) {
+        if (!SPLIT) {
             const float iv = L > 0.f ? 1.f / L : 0.f;
             __nv_bfloat16* op = out + (static_cast<long long>(r) * Hq + h) * D + d4;
             *reinterpret_cast<uint2*>(op) = make_uint2(pack_bf16x2(acc.x * iv, acc.y * iv),
                                                        pack_bf16x2(acc.z * iv, acc.w * iv));
         } else {
-            float* pr = part + (static_cast<long long>(r) * nsplit + split) * (16 * D + 32);
-            *reinterpret_cast<float4*>(pr + h * D + d4) = acc;
-            if (d4 == 0) {
-                pr[16 * D + h] = sF[S::WARPS * 16 + h];
-                pr[16 * D + 16 + h] = L;
-            }
+            *reinterpret_cast<float4*>(pO + h * D + d4) = acc;  // this split's partial O
         }
     }
-    if (nsplit == 1) return;
+    if (!SPLIT) return;
 
-    // The last CTA of the row to finish merges every split's partial:
-    //   out = sum_s O_s 2^(m_s - M) / sum_s l_s 2^(m_s - M),  M = max_s m_s.
-    // Publication: partials -> __threadfence -> counter increment; the CTA
-    // that takes the counter to nsplit resets it for the next launch.
-    __threadfence();
-    __syncthreads();
-    int* s_flag = s_last;  // reuse: the slot scan is long finished
-    if (tid == 0) *s_flag = atomicAdd(&row_done[r], 1) == nsplit - 1;
-    __syncthreads();
-    if (!*s_flag) return;
-    __threadfence();
-    const float* part_row = part + static_cast<long long>(r) * nsplit * (16 * D + 32);
-    constexpr int PSTRIDE = 16 * D + 32;
-    float* sML = mO;                 // [nsplit][32]: m[16], l[16] of every split
-    float* sf = mO + 64 * 32;        // [nsplit][16] merge factors
-    float* sinv = sf + 64 * 16;      // [16]
-    // one parallel round trip for every split's (m, l)
-    for (int i = tid; i < nsplit * 32; i += S::THREADS)
-        sML[i] = __ldcg(part_row + (i >> 5) * PSTRIDE + 16 * D + (i & 31));
+    // Split rows: the row's nsplit CTAs form one thread-block cluster and
+    // merge their partial states through distributed shared memory,
+    //   out = sum_q O_q 2^(M_q - M) / sum_q L_q 2^(M_q - M),  M = max_q M_q;
+    // CTA q of the cluster produces every nsplit-th group of outputs.  Every
+    // CTA reaches both cluster barriers: the first publishes the partials,
+    // the second keeps each CTA's shared memory alive until all have read it.
+    cluster_sync_all();
+    float* cML = pO + 16 * D;       // [nsplit][32]: every split's M[16], L[16]
+    float* cF = cML + 16 * 32;      // [nsplit][16] factors, then 1/L [16]
+    // one parallel round of remote loads for all splits' (M, L)
+    for (int t = tid; t < nsplit * 32; t += S::THREADS)
+        cML[t] = dsmem_ld_f32(dsmem_addr(sF + S::WARPS * 16 + (t & 31), t >> 5));
     __syncthreads();
     if (tid < 16) {
         const int h = tid;
         float M = -INFINITY;
-        for (int q = 0; q < nsplit; ++q) M = fmaxf(M, sML[q * 32 + h]);
-        float L = 0.f;
+        for (int q = 0; q < nsplit; ++q) M = fmaxf(M, cML[q * 32 + h]);
+        float Lt = 0.f;
         for (int q = 0; q < nsplit; ++q) {
-            const float f = M == -INFINITY ? 0.f : ex2_approx(sML[q * 32 + h] - M);
-            sf[q * 16 + h] = f;
-            L += sML[q * 32 + 16 + h] * f;
+            const float f = M == -INFINITY ? 0.f : ex2_approx(cML[q * 32 + h] - M);
+            cF[q * 16 + h] = f;
+            Lt += cML[q * 32 + 16 + h] * f;
         }
-        sinv[h] = L > 0.f ? 1.f / L : 0.f;
+        cF[nsplit * 16 + h] = Lt > 0.f ? 1.f / Lt : 0.f;
     }
     __syncthreads();
-    // O: float4 columns, the split loop unrolled so its loads overlap
-    for (int e = tid; e < Hq * (D / 4); e += S::THREADS) {
-        const int h = e / (D / 4), d4 = (e % (D / 4)) * 4;
+    for (int e4 = split * S::THREADS + tid; e4 < Hq * (D / 4); e4 += nsplit * S::THREADS) {
+        const int h = e4 / (D / 4), d4 = (e4 % (D / 4)) * 4;
+        float4 v[kMaxClusterSplits];
+#pragma unroll
+        for (int q = 0; q < kMaxClusterSplits; ++q)  // all remote loads in flight at once
+            if (q < nsplit) v[q] = dsmem_ld_f4(dsmem_addr(pO + h * D + d4, q));
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-        for (int q = 0; q < nsplit; ++q) {
-            const float4 v = __ldcg(reinterpret_cast<const float4*>(part_row + q * PSTRIDE + h * D + d4));
-            const float f = sf[q * 16 + h];
-            acc.x = fmaf(v.x, f, acc.x);
-            acc.y = fmaf(v.y, f, acc.y);
-            acc.z = fmaf(v.z, f, acc.z);
-            acc.w = fmaf(v.w, f, acc.w);
-        }
-        const float iv = sinv[h];
+#pragma unroll
+        for (int q = 0; q < kMaxClusterSplits; ++q)
+            if (q < nsplit) {
+                const float f = cF[q * 16 + h];
+                acc.x = fmaf(v[q].x, f, acc.x);
+                acc.y = fmaf(v[q].y, f, acc.y);
+                acc.z = fmaf(v[q].z, f, acc.z);
+                acc.w = fmaf(v[q].w, f, acc.w);
+            }
+        const float iv = cF[nsplit * 16 + h];
         __nv_bfloat16* op = out + (static_cast<long long>(r) * Hq + h) * D + d4;
         *reinterpret_cast<uint2*>(op) = make_uint2(pack_bf16x2(acc.x * iv, acc.y * iv),
                                                    pack_bf16x2(acc.z * iv, acc.w * iv));
     }
-    if (tid == 0) row_done[r] = 0;
+    cluster_sync_all();
 }
 
 template <int D>
@@ -388,56 +384,91 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
     using S = AttnShape<D>;
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_sparse_attn<D>,
+        cudaError_t e = cudaFuncSetAttribute(k_sparse_attn<D, false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(k_sparse_attn<D, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
         if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaFuncSetAttribute(sparse_attn)");
         attr_set = true;
     }
     // Split the index slots across CTAs when there are too few rows to fill
     // the GPU (decode): about one wave at two CTAs per SM, whole chunks per
-    // split, at most 64 splits.
+    // split.  A split row's CTAs form one cluster (they merge through
+    // distributed shared memory); the split count is lowered until every
+    // row's cluster can be resident at once (a cluster waiting for a second
+    // wave would double the kernel's time).
+    static int active[kMaxClusterSplits + 1] = {};  // resident clusters per cluster size (0: unknown)
+    static bool nonportable = false, attr_tried = false;
+    if (!attr_tried) {
+        nonportable = cudaFuncSetAttribute(k_sparse_attn<D, true>,
+                                           cudaFuncAttributeNonPortableClusterSizeAllowed,
+                                           1) == cudaSuccess;
+        cudaGetLastError();
+        attr_tried = true;
+    }
+    auto resident_clusters = [&](int cs) -> int {
+        if (active[cs] == 0) {
+            cudaLaunchConfig_t q = {};
+            q.gridDim = dim3(1, cs, 1);
+            q.blockDim = dim3(S::THREADS, 1, 1);
+            q.dynamicSmemBytes = S::SMEM;
+            cudaLaunchAttribute qa[1];
+            qa[0].id = cudaLaunchAttributeClusterDimension;
+            qa[0].val.clusterDim.x = 1;
+            qa[0].val.clusterDim.y = cs;
+            qa[0].val.clusterDim.z = 1;
+            q.attrs = qa;
+            q.numAttrs = 1;
+            int n = 0;
+            if (cudaOccupancyMaxActiveClusters(&n, k_sparse_attn<D, true>, &q) != cudaSuccess) n = -1;
+            cudaGetLastError();  // a refused query leaves no error behind
+            active[cs] = n;
+        }
+        return active[cs];
+    };
     int nsplit = 1;
     const int target = 2 * ctx->num_sms;
     if (rows < target) {
         nsplit = target / rows;
         const int max_split = (k + S::CH - 1) / S::CH;
         if (nsplit > max_split) nsplit = max_split;
-        if (nsplit > 64) nsplit = 64;
+        const int cap = nonportable ? kMaxClusterSplits : 8;
+        if (nsplit > cap) nsplit = cap;
+        while (nsplit > 1 && resident_clusters(nsplit) < rows) --nsplit;
         if (nsplit < 1) nsplit = 1;
     }
     int kps = (k + nsplit - 1) / nsplit;
     kps = (kps + S::CH - 1) / S::CH * S::CH;
     nsplit = (k + kps - 1) / kps;
-    float* part = nullptr;
-    int* row_done = nullptr;
-    if (nsplit > 1) {
-        // partials, then one completion counter per row (zeroed here once;
-        // every launch leaves them at zero)
-        const size_t pbytes = static_cast<size_t>(rows) * nsplit * (16 * D + 32) * sizeof(float);
-        const size_t bytes = pbytes + static_cast<size_t>(rows) * sizeof(int);
-        const bool fresh = ctx->attn_part_cap < bytes || !ctx->attn_part;
-        int rc = ensure_buffer(ctx, reinterpret_cast<void**>(&ctx->attn_part), &ctx->attn_part_cap,
-                               bytes);
-        if (rc) return rc;
-        part = ctx->attn_part;
-        row_done = reinterpret_cast<int*>(reinterpret_cast<char*>(part) + pbytes);
-        if (fresh) {
-            cudaError_t e = cudaMemsetAsync(ctx->attn_part, 0, ctx->attn_part_cap, stream);
-            if (e != cudaSuccess) return cuda_fail(ctx, e, "sparse_attn: counters");
-        }
-    }
     const float scale_log2 = scale * 1.4426950408889634f;
-    {
-        LaunchScope ls(ctx, IC_K_ATTN, stream);
-        dim3 grid(rows, nsplit);
-        k_sparse_attn<D><<<grid, S::THREADS, S::SMEM, stream>>>(
-            static_cast<const __nv_bfloat16*>(Q), static_cast<const __nv_bfloat16*>(K),
-            static_cast<const __nv_bfloat16*>(V), idx, Hq, k, rows_per_seq,
-            static_cast<long long>(kv_seq_stride), kv_len, scale_log2, nsplit, kps,
-            static_cast<__nv_bfloat16*>(out), part, row_done, ctx->dev_err);
-        cudaError_t e = ls.done();
-        if (e != cudaSuccess) return cuda_fail(ctx, e, "sparse_attn launch");
+    LaunchScope ls(ctx, IC_K_ATTN, stream);
+    const auto* Qp = static_cast<const __nv_bfloat16*>(Q);
+    const auto* Kp = static_cast<const __nv_bfloat16*>(K);
+    const auto* Vp = static_cast<const __nv_bfloat16*>(V);
+    auto* op = static_cast<__nv_bfloat16*>(out);
+    const long long kvs = static_cast<long long>(kv_seq_stride);
+    if (nsplit == 1) {
+        k_sparse_attn<D, false><<<dim3(rows, 1), S::THREADS, S::SMEM, stream>>>(
+            Qp, Kp, Vp, idx, Hq, k, rows_per_seq, kvs, kv_len, scale_log2, 1, kps, op, ctx->dev_err);
+    } else {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(rows, nsplit, 1);
+        cfg.blockDim = dim3(S::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = S::SMEM;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 1;
+        attr[0].val.clusterDim.y = nsplit;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        cudaLaunchKernelEx(&cfg, k_sparse_attn<D, true>, Qp, Kp, Vp, idx, Hq, k, rows_per_seq, kvs, kv_len,
+                           scale_log2, nsplit, kps, op, ctx->dev_err);
     }
+    cudaError_t e = ls.done();
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "sparse_attn launch");
     return IC_OK;
 }
 

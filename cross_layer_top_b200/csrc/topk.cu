@@ -243,28 +243,6 @@ __global__ void __launch_bounds__(kTopkThreads)
 // as k_topk.
 constexpr int kClusterCtas = 8;
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-    return r;
-}
-__device__ __forceinline__ void cluster_sync_all() {
-    asm volatile(
-        "barrier.cluster.arrive.release.aligned;\n\t"
-        "barrier.cluster.wait.acquire.aligned;" ::
-            : "memory");
-}
-__device__ __forceinline__ uint32_t dsmem_addr(const void* local, uint32_t rank) {
-    uint32_t r;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(local)), "r"(rank));
-    return r;
-}
-__device__ __forceinline__ uint32_t dsmem_ld(uint32_t addr) {
-    uint32_t v;
-    asm volatile("ld.shared::cluster.u32 %0, [%1];" : "=r"(v) : "r"(addr) : "memory");
-    return v;
-}
-
 struct TopkClusterShared {
     TopkShared S;
     uint32_t hist_all[2048];
