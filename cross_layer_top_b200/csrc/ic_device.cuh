@@ -261,6 +261,14 @@ __device__ __forceinline__ float4 dsmem_ld_f4(uint32_t addr) {
                  : "memory");
     return v;
 }
+__device__ __forceinline__ uint4 dsmem_ld_u4(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
 __device__ __forceinline__ float dsmem_ld_f32(uint32_t addr) {
     return __uint_as_float(dsmem_ld(addr));
 }

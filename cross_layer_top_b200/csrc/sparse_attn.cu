@@ -60,7 +60,9 @@ struct AttnShape {
 // byte offset of 16-byte piece c of row `row` in a [rows][d] bf16 tile whose
 // pieces are XOR-swizzled by (row mod 8): ldmatrix reads 8 rows of one piece
 // column from 8 different bank groups
-constexpr int kMaxClusterSplits = 16;  // CTAs of one split row's cluster, at most
+// CTAs of one split row's cluster, at most: the portable cluster size (on
+// back-to-back decode layers 8-CTA clusters schedule better than 16 or 4)
+constexpr int kMaxClusterSplits = 8;
 
 template <int D>
 __device__ __forceinline__ uint32_t swz(int row, int c) {
@@ -394,19 +396,11 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
     }
     // Split the index slots across CTAs when there are too few rows to fill
     // the GPU (decode): about one wave at two CTAs per SM, whole chunks per
-    // split.  A split row's CTAs form one cluster (they merge through
-    // distributed shared memory); the split count is lowered until every
-    // row's cluster can be resident at once (a cluster waiting for a second
-    // wave would double the kernel's time).
+    // split, at most kMaxClusterSplits.  A split row's CTAs form one cluster
+    // (they merge through distributed shared memory); the split count is
+    // lowered until every row's cluster can be resident at once (a cluster
+    // waiting for a second wave would double the kernel's time).
     static int active[kMaxClusterSplits + 1] = {};  // resident clusters per cluster size (0: unknown)
-    static bool nonportable = false, attr_tried = false;
-    if (!attr_tried) {
-        nonportable = cudaFuncSetAttribute(k_sparse_attn<D, true>,
-                                           cudaFuncAttributeNonPortableClusterSizeAllowed,
-                                           1) == cudaSuccess;
-        cudaGetLastError();
-        attr_tried = true;
-    }
     auto resident_clusters = [&](int cs) -> int {
         if (active[cs] == 0) {
             cudaLaunchConfig_t q = {};
@@ -433,8 +427,7 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
         nsplit = target / rows;
         const int max_split = (k + S::CH - 1) / S::CH;
         if (nsplit > max_split) nsplit = max_split;
-        const int cap = nonportable ? kMaxClusterSplits : 8;
-        if (nsplit > cap) nsplit = cap;
+        if (nsplit > kMaxClusterSplits) nsplit = kMaxClusterSplits;
         while (nsplit > 1 && resident_clusters(nsplit) < rows) --nsplit;
         if (nsplit < 1) nsplit = 1;
     }

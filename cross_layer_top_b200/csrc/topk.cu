@@ -21,6 +21,8 @@
 //     second walk writes the selected positions in ascending order (a key
 //     == T is selected while fewer than krem equal keys precede it).
 // Rows that fit in shared memory are read from global memory once.
+#include <cstddef>
+
 #include "ic_device.cuh"
 #include "ic_internal.h"
 
@@ -41,9 +43,10 @@ __device__ __forceinline__ float key_float(uint32_t u) {
     return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
 }
 
-struct TopkShared {
-    uint32_t hist[2048];
-    uint32_t cand[kCandCap];
+// hist and cand are read with 16-byte (remote) loads in the cluster variant
+struct alignas(16) TopkShared {
+    alignas(16) uint32_t hist[2048];
+    alignas(16) uint32_t cand[kCandCap];
     uint32_t wsum[kTopkWarps];
     uint32_t wcnt[2][kTopkWarps];
     uint32_t ncand;
@@ -243,11 +246,14 @@ __global__ void __launch_bounds__(kTopkThreads)
 // as k_topk.
 constexpr int kClusterCtas = 8;
 
-struct TopkClusterShared {
+struct alignas(16) TopkClusterShared {
     TopkShared S;
-    uint32_t hist_all[2048];
+    alignas(16) uint32_t hist_all[2048];
     uint32_t seg_kmin, seg_kmax, seg_cg, seg_ce;
 };
+static_assert(offsetof(TopkShared, hist) % 16 == 0 && offsetof(TopkShared, cand) % 16 == 0,
+              "16-byte loads of the histogram and candidates");
+static_assert(offsetof(TopkClusterShared, hist_all) % 16 == 0, "16-byte stores of hist_all");
 
 __global__ void __launch_bounds__(kTopkThreads)
     k_topk_cluster(const float* __restrict__ scores, long long ld, int k,
@@ -312,11 +318,19 @@ __global__ void __launch_bounds__(kTopkThreads)
         CS.seg_kmax = b;
     }
     cluster_sync_all();
+    // every CTA's range: all remote loads issued before any is used
+    uint32_t qmin[kClusterCtas], qmax[kClusterCtas];
+#pragma unroll
+    for (uint32_t q = 0; q < kClusterCtas; ++q) {
+        qmin[q] = dsmem_ld(dsmem_addr(&CS.seg_kmin, q));
+        qmax[q] = dsmem_ld(dsmem_addr(&CS.seg_kmax, q));
+    }
     kmin = 0xFFFFFFFFu;
     kmax = 0u;
+#pragma unroll
     for (uint32_t q = 0; q < kClusterCtas; ++q) {
-        kmin = min(kmin, dsmem_ld(dsmem_addr(&CS.seg_kmin, q)));
-        kmax = max(kmax, dsmem_ld(dsmem_addr(&CS.seg_kmax, q)));
+        kmin = min(kmin, qmin[q]);
+        kmax = max(kmax, qmax[q]);
     }
     const float xmin = key_float(kmin), xmax = key_float(kmax);
     const float span = xmax - xmin;
@@ -327,13 +341,23 @@ __global__ void __launch_bounds__(kTopkThreads)
         return static_cast<uint32_t>(fminf((key_float(u) - xmin) * inv, 2047.0f));
     };
     // cluster-wide histogram: local counts, then every CTA sums all of them
+    // each thread sums 4 consecutive bins (2048 = 4 x 512) over the cluster's
+    // CTAs with one 16-byte remote load per CTA, all issued before any is used
+    static_assert(2048 == 4 * kTopkThreads, "four bins per thread");
     auto cluster_hist = [&]() {
         cluster_sync_all();  // every segment histogram is complete
-        for (int bb = tid; bb < 2048; bb += kTopkThreads) {
-            uint32_t t = 0;
-            for (uint32_t q = 0; q < kClusterCtas; ++q) t += dsmem_ld(dsmem_addr(&S.hist[bb], q));
-            CS.hist_all[bb] = t;
+        uint4 hv[kClusterCtas];
+#pragma unroll
+        for (uint32_t q = 0; q < kClusterCtas; ++q) hv[q] = dsmem_ld_u4(dsmem_addr(&S.hist[4 * tid], q));
+        uint4 t = make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+        for (uint32_t q = 0; q < kClusterCtas; ++q) {
+            t.x += hv[q].x;
+            t.y += hv[q].y;
+            t.z += hv[q].z;
+            t.w += hv[q].w;
         }
+        *reinterpret_cast<uint4*>(&CS.hist_all[4 * tid]) = t;
         cluster_sync_all();  // nobody rewrites a histogram another CTA still reads
     };
     for (int i = tid; i < m; i += kTopkThreads) atomicAdd(&S.hist[bin_of(srow[i])], 1u);
@@ -354,11 +378,29 @@ __global__ void __launch_bounds__(kTopkThreads)
             if (bin_of(u) == b1) S.cand[atomicAdd(&S.ncand, 1u)] = u;
         }
         cluster_sync_all();
+        // every CTA's candidate count, then its candidates at the running
+        // offset: 4 per 16-byte remote load, each round's loads (one per CTA)
+        // issued before any is stored
+        int nq[kClusterCtas], off[kClusterCtas];
+#pragma unroll
+        for (uint32_t q = 0; q < kClusterCtas; ++q) nq[q] = static_cast<int>(dsmem_ld(dsmem_addr(&S.ncand, q)));
+#pragma unroll
         for (uint32_t q = 0; q < kClusterCtas; ++q) {
-            const int nq = static_cast<int>(dsmem_ld(dsmem_addr(&S.ncand, q)));
-            for (int i = tid; i < nq; i += kTopkThreads)
-                cand_all[ncand + i] = dsmem_ld(dsmem_addr(&S.cand[i], q));
-            ncand += nq;
+            off[q] = ncand;
+            ncand += nq[q];
+        }
+        for (int i4 = 4 * tid; i4 < kCandCap; i4 += 4 * kTopkThreads) {
+            uint4 cv[kClusterCtas];
+#pragma unroll
+            for (uint32_t q = 0; q < kClusterCtas; ++q)
+                if (i4 < nq[q]) cv[q] = dsmem_ld_u4(dsmem_addr(&S.cand[i4], q));
+#pragma unroll
+            for (uint32_t q = 0; q < kClusterCtas; ++q) {
+                const uint32_t c4[4] = {cv[q].x, cv[q].y, cv[q].z, cv[q].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (i4 + e < nq[q]) cand_all[off[q] + i4 + e] = c4[e];
+            }
         }
         cluster_sync_all();
     }
