@@ -163,6 +163,16 @@ extern "C" int ic_ctx_destroy(ic_ctx* ctx) {
     cudaDeviceSynchronize();
     cudaFree(ctx->scores);
     cudaFree(ctx->dev_err);
+    if (ctx->hs.ready) {
+        for (int i = 0; i < 2; ++i) {
+            cudaFree(ctx->hs.slot[i]);
+            cudaEventDestroy(ctx->hs.in_ready[i]);
+            cudaEventDestroy(ctx->hs.computed[i]);
+            cudaEventDestroy(ctx->hs.out_done[i]);
+        }
+        cudaStreamDestroy(ctx->hs.in);
+        cudaStreamDestroy(ctx->hs.out);
+    }
     for (auto& p : ctx->pool) {
         cudaEventDestroy(p.start);
         cudaEventDestroy(p.stop);
@@ -522,49 +532,60 @@ extern "C" int ic_index_overlap(ic_ctx* ctx, const int32_t* idx_a, const int32_t
 }
 
 // ------------------------------------------------------------ layer stack
-extern "C" int ic_run_stack(ic_ctx* ctx, const ic_pattern* pattern, const ic_layer_io* layers,
-                            const ic_stack_dims* dims, int32_t* idx_cache, void* stream) {
+namespace ic {
+// One layer of the stack ([IC] Figure 2): an F layer runs the indexer and
+// top-k into idx_cache, an S layer reuses it; then the layer's attention.
+int run_stack_layer(ic_ctx* ctx, char c, const ic_layer_io& io, const ic_stack_dims* dims,
+                    int32_t* idx_cache, void* stream) {
+    const bool prefill = dims->mode == IC_PREFILL;
+    const int rows = prefill ? dims->L : dims->B;
+    const int k = dims->k;
+    int rc;
+    if (c == 'F') {
+        if (prefill)
+            rc = ic_index_fp(ctx, io.qI, io.kI, io.w, dims->L, dims->H_I, dims->d_I, k, idx_cache,
+                             stream);
+        else
+            rc = ic_index_fp_decode(ctx, io.qI, io.w, io.kI8, io.kI_scale, dims->seq_len, dims->B,
+                                    dims->S_max, dims->H_I, dims->d_I, k, idx_cache, stream);
+        if (rc) return rc;
+    }
+    // S layer: the cache is used as it stands (no kernel)
+    const int32_t* idx = nullptr;
+    ic_index_reuse(idx_cache, &idx);
+    if (io.idx_snapshot) {
+        cudaError_t e = cudaMemcpyAsync(io.idx_snapshot, idx,
+                                        static_cast<size_t>(rows) * k * sizeof(int32_t),
+                                        cudaMemcpyDeviceToDevice, as_stream(stream));
+        if (e != cudaSuccess) return cuda_fail(ctx, e, "run_stack: snapshot copy");
+    }
+    if (prefill)
+        return ic_sparse_attn(ctx, io.Q, io.K, io.V, idx, rows, dims->Hq, dims->d, k, 0, 0, dims->L,
+                              dims->scale, io.out, stream);
+    return ic_sparse_attn(ctx, io.Q, io.K, io.V, idx, rows, dims->Hq, dims->d, k, 1,
+                          static_cast<int64_t>(dims->S_max) * dims->d, dims->S_max, dims->scale,
+                          io.out, stream);
+}
+
+int check_stack_args(ic_ctx* ctx, const ic_pattern* pattern, const void* layers,
+                     const ic_stack_dims* dims, const int32_t* idx_cache) {
     if (!ctx) return fail(nullptr, IC_ERR_INVALID_ARG, "context is NULL");
     if (!pattern || !layers || !dims || !idx_cache)
         return fail(ctx, IC_ERR_INVALID_ARG, "run_stack: NULL argument");
-    const int N = static_cast<int>(pattern->c.size());
-    const bool prefill = dims->mode == IC_PREFILL;
-    if (!prefill && dims->mode != IC_DECODE)
+    if (dims->mode != IC_PREFILL && dims->mode != IC_DECODE)
         return fail(ctx, IC_ERR_INVALID_ARG, "run_stack: mode %d", dims->mode);
-    const int rows = prefill ? dims->L : dims->B;
-    const int k = dims->k;
-    cudaStream_t s = as_stream(stream);
+    return IC_OK;
+}
+}  // namespace ic
+
+extern "C" int ic_run_stack(ic_ctx* ctx, const ic_pattern* pattern, const ic_layer_io* layers,
+                            const ic_stack_dims* dims, int32_t* idx_cache, void* stream) {
+    int rc = check_stack_args(ctx, pattern, layers, dims, idx_cache);
+    if (rc) return rc;
     cudaSetDevice(ctx->device);
+    const int N = static_cast<int>(pattern->c.size());
     for (int l = 0; l < N; ++l) {
-        const ic_layer_io& io = layers[l];
-        int rc;
-        if (pattern->c[l] == 'F') {
-            // F layer: indexer + top-k, overwriting the cache
-            if (prefill)
-                rc = ic_index_fp(ctx, io.qI, io.kI, io.w, dims->L, dims->H_I, dims->d_I, k,
-                                 idx_cache, stream);
-            else
-                rc = ic_index_fp_decode(ctx, io.qI, io.w, io.kI8, io.kI_scale, dims->seq_len,
-                                        dims->B, dims->S_max, dims->H_I, dims->d_I, k, idx_cache,
-                                        stream);
-            if (rc) return rc;
-        }
-        // S layer: the cache is used as it stands (no kernel)
-        const int32_t* idx = nullptr;
-        ic_index_reuse(idx_cache, &idx);
-        if (io.idx_snapshot) {
-            cudaError_t e = cudaMemcpyAsync(io.idx_snapshot, idx,
-                                            static_cast<size_t>(rows) * k * sizeof(int32_t),
-                                            cudaMemcpyDeviceToDevice, s);
-            if (e != cudaSuccess) return cuda_fail(ctx, e, "run_stack: snapshot copy");
-        }
-        if (prefill)
-            rc = ic_sparse_attn(ctx, io.Q, io.K, io.V, idx, rows, dims->Hq, dims->d, k, 0, 0,
-                                dims->L, dims->scale, io.out, stream);
-        else
-            rc = ic_sparse_attn(ctx, io.Q, io.K, io.V, idx, rows, dims->Hq, dims->d, k, 1,
-                                static_cast<int64_t>(dims->S_max) * dims->d, dims->S_max,
-                                dims->scale, io.out, stream);
+        rc = run_stack_layer(ctx, pattern->c[l], layers[l], dims, idx_cache, stream);
         if (rc) return rc;
     }
     return IC_OK;

@@ -9,6 +9,7 @@
 #include <vector>
 
 #include "ic_errors.h"
+#include "indexcache.h"
 
 struct ic_ctx {
     int device = 0;
@@ -28,6 +29,15 @@ struct ic_ctx {
     double total_ms[IC_K_COUNT] = {0};
     int64_t launches[IC_K_COUNT] = {0};
     int64_t launch_count = 0;
+    // ic_run_stack_host: two device staging slots, a copy-in and a copy-out
+    // stream, and per-slot events (created on first use)
+    struct HostStack {
+        bool ready = false;
+        cudaStream_t in = nullptr, out = nullptr;
+        cudaEvent_t in_ready[2] = {}, computed[2] = {}, out_done[2] = {};
+        void* slot[2] = {nullptr, nullptr};
+        size_t slot_cap = 0;  // bytes per slot
+    } hs;
 };
 
 struct ic_pattern {
@@ -71,6 +81,12 @@ int make_tmap_u8_2d(ic_ctx* ctx, CUtensorMap* map, const void* base, uint64_t ro
                     uint32_t box_cols, uint32_t box_rows, bool swizzle128);
 
 // ----------------------------------------------------------------- launchers
+// One layer of the F/S stack (shared by ic_run_stack and ic_run_stack_host).
+int run_stack_layer(ic_ctx* ctx, char c, const ic_layer_io& io, const ic_stack_dims* dims,
+                    int32_t* idx_cache, void* stream);
+int check_stack_args(ic_ctx* ctx, const ic_pattern* pattern, const void* layers,
+                     const ic_stack_dims* dims, const int32_t* idx_cache);
+
 int launch_index_score_prefill(ic_ctx* ctx, const void* qI, const void* kI, const void* w, int L,
                                int H_I, int d_I, int row_begin, int row_end, float* scores,
                                int64_t ld, cudaStream_t stream);

@@ -87,6 +87,8 @@ _SIGS = {
     "ic_probe_wait_timeout": ([_vp, _vp], _i),
     "ic_run_stack": ([_vp, _vp, ctypes.POINTER(ic_layer_io), ctypes.POINTER(ic_stack_dims), _vp,
                       _vp], _i),
+    "ic_run_stack_host": ([_vp, _vp, ctypes.POINTER(ic_layer_io), ctypes.POINTER(ic_stack_dims),
+                           _vp, _vp], _i),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -373,6 +375,21 @@ def ic_run_stack(ctx: Context, pattern: Pattern, layers, dims: ic_stack_dims, id
     arr = layer_array if layer_array is not None else make_stack_layers(layers, dims.mode)
     _check(_lib.ic_run_stack(ctx.handle, pattern.handle, arr, ctypes.byref(dims),
                              _ptr(idx_cache), _stream(stream)), ctx)
+
+
+def ic_run_stack_host(ctx: Context, pattern: Pattern, layers_host, dims: ic_stack_dims, idx_cache,
+                      stream=None, layer_array=None):
+    """ic_run_stack on inputs in (pinned) host memory: layers_host holds CPU
+    tensors for every field but idx_snapshot; each layer's 'out' (a CPU
+    tensor) receives its output.  Asynchronous on `stream`."""
+    if layer_array is None:
+        for lay in layers_host:
+            for n, t in lay.items():
+                if n != "idx_snapshot" and t is not None and t.is_cuda:
+                    raise ValueError("%s must be a host tensor" % n)
+        layer_array = make_stack_layers(layers_host, dims.mode)
+    _check(_lib.ic_run_stack_host(ctx.handle, pattern.handle, layer_array, ctypes.byref(dims),
+                                  _ptr(idx_cache), _stream(stream)), ctx)
 
 
 def stack_dims(mode, H_I, d_I, k, Hq, d, L=0, B=0, S_max=0, seq_len=None, scale=0.0):
