@@ -295,7 +295,7 @@ def run_ours(args, rank, world, local_rank):
 # DRAM traffic per launch of the prefill attention kernel from its ncu
 # capture (profiles/sparse_attn_prefill_L16384.md); None until measured for
 # the current kernel.
-ATTN_PREFILL_DRAM_BYTES = 210140928 + 52539904
+ATTN_PREFILL_DRAM_BYTES = None  # re-measured after the next capture of the changed kernel
 
 
 def measure_gather_ceiling(cache, lay, L, k, stream):

@@ -76,7 +76,8 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, 2)
     k_sparse_attn(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
                   const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ idx, int Hq,
                   int k, int rows_per_seq, long long kv_seq_stride, int kv_len, float scale_log2,
-                  int nsplit, int kps, __nv_bfloat16* __restrict__ out, int* __restrict__ err) {
+                  int nsplit, int kps, int pf_ahead, __nv_bfloat16* __restrict__ out,
+                  int* __restrict__ err) {
     using S = AttnShape<D>;
     extern __shared__ __align__(128) uint8_t smem[];
     const int r = blockIdx.x, split = blockIdx.y;
@@ -90,6 +91,19 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, 2)
     const __nv_bfloat16* Kb = K + seq * kv_seq_stride;
     const __nv_bfloat16* Vb = V + seq * kv_seq_stride;
 
+    // rows run about one wave of CTAs apart: warm L2 with the index and
+    // query rows of the row one wave ahead, so whichever CTA takes it does not
+    // start on an HBM round trip
+    if (!SPLIT && pf_ahead > 0 && r + pf_ahead < gridDim.x) {
+        const int rr = r + pf_ahead;
+        const char* pidx = reinterpret_cast<const char*>(idx + static_cast<long long>(rr) * k);
+        const char* pq = reinterpret_cast<const char*>(Q + static_cast<long long>(rr) * Hq * D);
+        const int idx_lines = (k * 4 + 127) / 128, q_lines = (Hq * D * 2 + 127) / 128;
+        if (tid < idx_lines)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(pidx + tid * 128));
+        else if (tid < idx_lines + q_lines)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(pq + (tid - idx_lines) * 128));
+    }
     if (tid == 0) *s_last = -1;
     __syncthreads();
     // index slots of this split (validated), the last valid slot, the query heads
@@ -443,7 +457,8 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
     const long long kvs = static_cast<long long>(kv_seq_stride);
     if (nsplit == 1) {
         k_sparse_attn<D, false><<<dim3(rows, 1), S::THREADS, S::SMEM, stream>>>(
-            Qp, Kp, Vp, idx, Hq, k, rows_per_seq, kvs, kv_len, scale_log2, 1, kps, op, ctx->dev_err);
+            Qp, Kp, Vp, idx, Hq, k, rows_per_seq, kvs, kv_len, scale_log2, 1, kps, 2 * ctx->num_sms,
+            op, ctx->dev_err);
     } else {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(rows, nsplit, 1);
@@ -458,7 +473,7 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         cudaLaunchKernelEx(&cfg, k_sparse_attn<D, true>, Qp, Kp, Vp, idx, Hq, k, rows_per_seq, kvs, kv_len,
-                           scale_log2, nsplit, kps, op, ctx->dev_err);
+                           scale_log2, nsplit, kps, 0, op, ctx->dev_err);
     }
     cudaError_t e = ls.done();
     if (e != cudaSuccess) return cuda_fail(ctx, e, "sparse_attn launch");
