@@ -227,6 +227,16 @@ def run_ours(args, rank, world, local_rank):
             extra_ceiling = None
     else:
         extra_ceiling = None
+    if top_k["launches"]:
+        # algorithmic bytes per F layer: the fp32 scores of every scored row
+        # t >= k read once (4(t+1) B), and k int32 indices written for every row
+        bytes_f = sum(4 * (t + 1) for t in range(k, L)) + 4 * k * L
+        per_f = top_k["ms"] / (args.steps * n_f)
+        gbs = bytes_f / (per_f / 1e3) / 1e9
+        roof["topk"] = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
+                        "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
+                        "peak_kind": "HBM copy, " + peak_src,
+                        "ms_per_f_layer": round(per_f, 4), "bytes_per_f_layer": bytes_f}
     overlap = measure_overlap(ctx, layers, cfg, stream)
     dominant = max(("index_score", "sparse_attn"), key=lambda n: ktimes[n]["ms"])
     roofline = dict(roof.get(dominant, {}))

@@ -105,7 +105,7 @@ template <bool IN_SMEM>
 __global__ void __launch_bounds__(kTopkThreads)
     k_topk(const float* __restrict__ scores, long long ld, int row0, int k, int causal_base,
            const int32_t* __restrict__ row_len, int max_len, int32_t* __restrict__ out,
-           long long ld_out) {
+           long long ld_out, int pf_ahead) {
     extern __shared__ uint32_t srow[];
     __shared__ TopkShared S;
 
@@ -122,6 +122,18 @@ __global__ void __launch_bounds__(kTopkThreads)
     auto key_at = [&](int i) -> uint32_t {
         return IN_SMEM ? srow[i] : order_key(__ldg(row + i));
     };
+    // rows run about one wave of CTAs apart: warm L2 with the scores of the
+    // row one wave ahead, so whichever CTA takes it loads from L2
+    if (pf_ahead > 0 && static_cast<int>(blockIdx.x) + pf_ahead < static_cast<int>(gridDim.x)) {
+        const int rr = r + pf_ahead;
+        const int nn = row_len ? min(row_len[rr], max_len) : causal_base + rr + 1;
+        if (nn > k) {
+            const char* pr = reinterpret_cast<const char*>(scores + static_cast<long long>(rr) * ld);
+            const int lines = (nn * 4 + 127) / 128;
+            for (int i = tid; i < lines; i += kTopkThreads)
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(pr + static_cast<long long>(i) * 128));
+        }
+    }
 
     // ---- A: keys + histogram of the top 11 bits
     for (int i = tid; i < 2048; i += kTopkThreads) S.hist[i] = 0;
@@ -553,14 +565,16 @@ int launch_topk(ic_ctx* ctx, const float* scores, int64_t ld, int rows, int k, i
         const int smem = ((nmax < kTopkSmemCap ? nmax : kTopkSmemCap) + 3) / 4 * 16;
         LaunchScope ls(ctx, IC_K_TOPK, stream);
         k_topk<true><<<split, kTopkThreads, smem, stream>>>(scores, ld, 0, k, causal_base, row_len,
-                                                             max_len, idx_out, ld_out);
+                                                             max_len, idx_out, ld_out,
+                                                             scores ? 2 * ctx->num_sms : 0);
         cudaError_t e = ls.done();
         if (e != cudaSuccess) return cuda_fail(ctx, e, "topk launch");
     }
     if (split < rows) {
         LaunchScope ls(ctx, IC_K_TOPK, stream);
         k_topk<false><<<rows - split, kTopkThreads, 0, stream>>>(scores, ld, split, k, causal_base,
-                                                                 row_len, max_len, idx_out, ld_out);
+                                                                 row_len, max_len, idx_out, ld_out,
+                                                                 0);
         cudaError_t e = ls.done();
         if (e != cudaSuccess) return cuda_fail(ctx, e, "topk launch");
     }
