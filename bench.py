@@ -198,7 +198,8 @@ def run_ours(args, rank, world, local_rank):
         peak = peaks.get("bf16_tflops_sustained", peaks.get("bf16_tflops"))
         roof["index_score"] = {"bound": "tensor", "achieved": round(tflops, 1), "peak": peak,
                                "unit": "TFLOP/s", "frac": round(tflops / peak, 4),
-                               "traffic": None, "peak_kind": "sustained bf16, " + peak_src,
+                               "traffic": INDEX_SCORE_PREFILL_DRAM_BYTES,
+                               "peak_kind": "sustained bf16, " + peak_src,
                                "avg_launch_ms": round(avg_ms, 4),
                                "flop_per_launch": 2 * cfg.H_I * cfg.d_I * pairs_launch}
     if att_k["launches"]:
@@ -302,10 +303,12 @@ def run_ours(args, rank, world, local_rank):
     ctx.close()
 
 
-# DRAM traffic per launch of the prefill attention kernel from its ncu
-# capture (profiles/sparse_attn_prefill_L16384.md); None until measured for
-# the current kernel.
-ATTN_PREFILL_DRAM_BYTES = None  # re-measured after the next capture of the changed kernel
+# DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
+# the prefill kernels, from one ncu capture of the current kernel each
+# (profiles/sparse_attn_prefill_L16384.md, profiles/indexer_prefill_L16384.md);
+# None once a kernel changes until it is captured again.
+ATTN_PREFILL_DRAM_BYTES = 209.74e6 + 51.84e6
+INDEX_SCORE_PREFILL_DRAM_BYTES = 248.2e6 + 487.7e6
 
 
 def measure_gather_ceiling(cache, lay, L, k, stream):
@@ -434,21 +437,8 @@ def run_decode(args, ctx, peaks, peak_src, local_rank):
         ic.ic_run_stack(ctx, pat, None, dims, cache, layer_array=arr)
     ctx.sync_status()
     steps = max(args.steps, 5)
-    ctx.reset_timing()
-    ctx.set_timing(True)
-    stream = torch.cuda.current_stream()
-    tot = 0.0
-    for i in range(steps):
-        flush.fill_(float(i))
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        ic.ic_run_stack(ctx, pat, None, dims, cache, layer_array=arr)
-        b.record(stream)
-        b.synchronize()
-        tot += a.elapsed_time(b)
-    ctx.set_timing(False)
-    ctx.sync_status()
-    kt = {n: ctx.get_timing(i) for i, n in enumerate(ic.KERNEL_NAMES)}
+    t = _time_stack(ctx, pat, dims, cache, arr, steps, torch.cuda.current_stream(), flush)
+    kt = t.pop("kernels")
     n_f = cfg.pattern.count("F")
     scan_bytes = B * S * (cfg.d_I + 4) + B * S * 4  # e4m3 keys + scales read, fp32 scores written
     scan_ms, scan_n = kt["index_score_decode"]
@@ -456,7 +446,7 @@ def run_decode(args, ctx, peaks, peak_src, local_rank):
     gather_bytes = B * k * 2 * cfg.d * 2
     res = {"workload": "decode: 32 sequences x (65536 cached + 1 new) tokens, 16 layers FSSS x4, "
                        "FP8 e4m3 indexer keys + fp32 per-token scale, k=2048",
-           "step_ms": tot / steps,
+           **t,
            "kernels_ms_per_step": {n: round(v[0] / steps, 4) for n, v in kt.items()}}
     if scan_n:
         gbs = scan_bytes / (scan_ms / scan_n / 1e3) / 1e9
@@ -474,22 +464,50 @@ def run_decode(args, ctx, peaks, peak_src, local_rank):
     return res
 
 
-def _time_stack(ctx, pat, dims, cache, arr, steps, stream):
+def _time_stack(ctx, pat, dims, cache, arr, steps, stream, flush=None, graph=True):
+    """One step of the stack timed three ways, each over `steps`
+    steps with CUDA events around the step only: "step_ms" through
+    ic_run_stack, "graph_step_ms" as a replay of the stack captured with
+    ic_stack_graph_create, and "events_step_ms" with the library's
+    per-kernel timing events on (the per-kernel breakdown, "kernels", comes
+    from that pass; its events add launch gaps to a step of many small
+    kernels).  `flush`, when given, is rewritten before every step;
+    graph=False skips the graph pass."""
     from cross_layer_top_b200 import indexcache as ic
+
+    def timed(run):
+        tot = 0.0
+        for i in range(steps):
+            if flush is not None:
+                flush.fill_(float(i))
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            run()
+            b.record(stream)
+            b.synchronize()
+            tot += a.elapsed_time(b)
+        ctx.sync_status(stream)
+        return tot / steps
+
+    def eager():
+        ic.ic_run_stack(ctx, pat, None, dims, cache, stream=stream, layer_array=arr)
+
+    plain = timed(eager)
+    res = {"step_ms": plain}
+    if graph:
+        g = ic.ic_stack_graph_create(ctx, pat, None, dims, cache, layer_array=arr)
+        for _ in range(2):
+            g.launch(stream)
+        res["graph_step_ms"] = timed(lambda: g.launch(stream))
+        res["kernels_per_step"] = g.kernels()
+        g.close()
     ctx.reset_timing()
     ctx.set_timing(True)
-    tot = 0.0
-    for _ in range(steps):
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        ic.ic_run_stack(ctx, pat, None, dims, cache, layer_array=arr)
-        b.record(stream)
-        b.synchronize()
-        tot += a.elapsed_time(b)
+    with_events = timed(eager)
     ctx.set_timing(False)
-    ctx.sync_status()
-    kt = {n: ctx.get_timing(i)[0] / steps for i, n in enumerate(ic.KERNEL_NAMES)}
-    return tot / steps, kt
+    res["events_step_ms"] = with_events
+    res["kernels"] = {n: ctx.get_timing(i) for i, n in enumerate(ic.KERNEL_NAMES)}
+    return res
 
 
 def run_long_prefill(args, ctx, peaks, local_rank):
@@ -515,7 +533,9 @@ def run_long_prefill(args, ctx, peaks, local_rank):
     for pattern in ("FSSS", "FFFF"):
         pat = ic.ic_create_pattern(pattern)
         ic.ic_run_stack(ctx, pat, None, dims, cache, layer_array=arr)  # warm-up
-        ms, kt = _time_stack(ctx, pat, dims, cache, arr, 2, stream)
+        t = _time_stack(ctx, pat, dims, cache, arr, 2, stream, graph=False)
+        ms = t["step_ms"]
+        kt = {n: v[0] / 2 for n, v in t["kernels"].items()}
         pairs = scored_pairs(L, k, pattern.count("F"))
         ent = {"stack_ms": ms, "kernels_ms": {n: round(v, 3) for n, v in kt.items()},
                "scored_pairs_per_s": pairs / (ms / 1e3)}
@@ -602,20 +622,25 @@ def run_decode_sweep(args, ctx, local_rank):
         pat = ic.ic_pattern_uniform(cfg.n_layers, r)
         for _ in range(2):
             ic.ic_run_stack(ctx, pat, None, dims, cache, layer_array=arr)
-        ms, kt = _time_stack(ctx, pat, dims, cache, arr, 5, stream)
-        res["r%d" % r] = {"pattern_F_layers": str(pat).count("F"), "step_ms": ms,
-                          "tokens_per_s": B / (ms / 1e3),
-                          "kernels_ms": {n: round(v, 4) for n, v in kt.items()}}
+        t = _time_stack(ctx, pat, dims, cache, arr, 5, stream)
+        kt = t.pop("kernels")
+        res["r%d" % r] = {"pattern_F_layers": str(pat).count("F"), **t,
+                          "tokens_per_s": B / (t["step_ms"] / 1e3),
+                          "tokens_per_s_graph": B / (t["graph_step_ms"] / 1e3),
+                          "kernels_ms": {n: round(v[0] / 5, 4) for n, v in kt.items()}}
     # the searched patterns of the 47-layer model (same layer tensors)
     for ret, c in synth.SEARCHED_PATTERNS_47.items():
         pat = ic.ic_create_pattern(c)
         for _ in range(2):
             ic.ic_run_stack(ctx, pat, None, dims, cache, layer_array=arr)
-        ms, kt = _time_stack(ctx, pat, dims, cache, arr, 5, stream)
+        t = _time_stack(ctx, pat, dims, cache, arr, 5, stream)
+        kt = t.pop("kernels")
         res["searched_" + ret.replace("/", "_")] = {
-            "pattern_F_layers": c.count("F"), "step_ms": ms, "tokens_per_s": B / (ms / 1e3),
-            "kernels_ms": {n: round(v, 4) for n, v in kt.items()}}
+            "pattern_F_layers": c.count("F"), **t, "tokens_per_s": B / (t["step_ms"] / 1e3),
+            "tokens_per_s_graph": B / (t["graph_step_ms"] / 1e3),
+            "kernels_ms": {n: round(v[0] / 5, 4) for n, v in kt.items()}}
     res["speedup_r4_vs_r1"] = res["r1"]["step_ms"] / res["r4"]["step_ms"]
+    res["speedup_r4_vs_r1_graph"] = res["r1"]["graph_step_ms"] / res["r4"]["graph_step_ms"]
     del layers, arr, cache
     torch.cuda.empty_cache()
     return res

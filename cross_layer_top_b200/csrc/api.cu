@@ -58,6 +58,11 @@ cudaError_t LaunchScope::done() {
 
 int ensure_buffer(ic_ctx* ctx, void** buf, size_t* cap, size_t bytes) {
     if (*cap >= bytes && *buf) return IC_OK;
+    if (ctx->graphs_alive > 0)
+        return fail(ctx, IC_ERR_NOMEM,
+                    "scratch of %zu bytes needed while %d captured graph(s) hold the current "
+                    "%zu-byte buffer; destroy them first",
+                    bytes, ctx->graphs_alive, *cap);
     if (*buf) {
         cudaError_t e = cudaDeviceSynchronize();  // the old buffer may still be in use
         if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaDeviceSynchronize");
@@ -159,6 +164,9 @@ extern "C" int ic_ctx_create(ic_ctx** out, int device, size_t scratch_bytes) {
 
 extern "C" int ic_ctx_destroy(ic_ctx* ctx) {
     if (!ctx) return IC_ERR_INVALID_ARG;
+    if (ctx->graphs_alive > 0)
+        return fail(ctx, IC_ERR_INVALID_ARG, "ic_ctx_destroy: %d stack graph(s) still exist",
+                    ctx->graphs_alive);
     cudaSetDevice(ctx->device);
     cudaDeviceSynchronize();
     cudaFree(ctx->scores);

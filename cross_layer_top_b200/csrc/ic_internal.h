@@ -29,6 +29,7 @@ struct ic_ctx {
     double total_ms[IC_K_COUNT] = {0};
     int64_t launches[IC_K_COUNT] = {0};
     int64_t launch_count = 0;
+    int graphs_alive = 0;           // captured stack graphs that use this context's buffers
     // ic_run_stack_host: two device staging slots, a copy-in and a copy-out
     // stream, and per-slot events (created on first use)
     struct HostStack {

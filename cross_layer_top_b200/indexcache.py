@@ -9,6 +9,7 @@ ImportError when it is missing — there is no fallback path.
 from __future__ import annotations
 
 import ctypes
+import weakref
 import os
 
 import torch
@@ -89,6 +90,11 @@ _SIGS = {
                       _vp], _i),
     "ic_run_stack_host": ([_vp, _vp, ctypes.POINTER(ic_layer_io), ctypes.POINTER(ic_stack_dims),
                            _vp, _vp], _i),
+    "ic_stack_graph_create": ([_vp, _vp, ctypes.POINTER(ic_layer_io),
+                               ctypes.POINTER(ic_stack_dims), _vp, ctypes.POINTER(_vp)], _i),
+    "ic_stack_graph_launch": ([_vp, _vp], _i),
+    "ic_stack_graph_kernels": ([_vp], _i64),
+    "ic_stack_graph_destroy": ([_vp], _i),
 }
 for _name, (_args, _res) in _SIGS.items():
     _fn = getattr(_lib, _name)
@@ -146,8 +152,11 @@ class Context:
         _check(_lib.ic_ctx_create(ctypes.byref(h), device, scratch_bytes))
         self.handle = h
         self.device = device
+        self._graphs = weakref.WeakSet()
 
     def close(self):
+        for g in list(self._graphs):
+            g.close()
         if self.handle:
             _lib.ic_ctx_destroy(self.handle)
             self.handle = None
@@ -390,6 +399,46 @@ def ic_run_stack_host(ctx: Context, pattern: Pattern, layers_host, dims: ic_stac
         layer_array = make_stack_layers(layers_host, dims.mode)
     _check(_lib.ic_run_stack_host(ctx.handle, pattern.handle, layer_array, ctypes.byref(dims),
                                   _ptr(idx_cache), _stream(stream)), ctx)
+
+
+class StackGraph:
+    """ic_stack_graph_*: the stack captured once and replayed.  The graph
+    keeps the device addresses of the layer tensors, dims.seq_len and
+    idx_cache, so this object holds references to them; change their
+    contents in place between launches."""
+
+    def __init__(self, ctx: Context, pattern: Pattern, layers, dims: ic_stack_dims, idx_cache,
+                 layer_array=None):
+        arr = layer_array if layer_array is not None else make_stack_layers(layers, dims.mode)
+        h = _vp()
+        _check(_lib.ic_stack_graph_create(ctx.handle, pattern.handle, arr, ctypes.byref(dims),
+                                          _ptr(idx_cache), ctypes.byref(h)), ctx)
+        self.handle = h
+        self.ctx = ctx
+        ctx._graphs.add(self)
+        self._keep = (pattern, layers, dims, idx_cache, arr)
+
+    def launch(self, stream=None):
+        _check(_lib.ic_stack_graph_launch(self.handle, _stream(stream)), self.ctx)
+
+    def kernels(self) -> int:
+        return int(_lib.ic_stack_graph_kernels(self.handle))
+
+    def close(self):
+        if self.handle:
+            _lib.ic_stack_graph_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def ic_stack_graph_create(ctx: Context, pattern: Pattern, layers, dims: ic_stack_dims, idx_cache,
+                          layer_array=None) -> StackGraph:
+    return StackGraph(ctx, pattern, layers, dims, idx_cache, layer_array)
 
 
 def stack_dims(mode, H_I, d_I, k, Hq, d, L=0, B=0, S_max=0, seq_len=None, scale=0.0):

@@ -279,6 +279,23 @@ typedef struct ic_stack_dims {
 int ic_run_stack(ic_ctx *ctx, const ic_pattern *pattern, const ic_layer_io *layers,
                  const ic_stack_dims *dims, int32_t *idx_cache, void *stream);
 
+/* A stack captured once as a CUDA graph and replayed: a decode step of
+ * many small dependent kernels then costs one graph launch.  Create runs
+ * ic_run_stack once eagerly (sizing scratch, setting kernel attributes),
+ * then captures the same calls; the graph keeps the device pointers of
+ * layers, dims->seq_len and idx_cache as they are now, so the caller keeps
+ * those buffers alive and changes only their contents between launches.
+ * While a graph of ctx exists, calls that would need larger scratch than it
+ * captured fail with IC_ERR_NOMEM.  Launch is asynchronous on `stream`.
+ * ic_stack_graph_kernels: kernel launches in one replay.  Destroy before
+ * ic_ctx_destroy. */
+typedef struct ic_graph ic_graph;
+int ic_stack_graph_create(ic_ctx *ctx, const ic_pattern *pattern, const ic_layer_io *layers,
+                          const ic_stack_dims *dims, int32_t *idx_cache, ic_graph **out);
+int ic_stack_graph_launch(ic_graph *graph, void *stream);
+int64_t ic_stack_graph_kernels(const ic_graph *graph);
+int ic_stack_graph_destroy(ic_graph *graph);
+
 /* The same stack on inputs in host memory, with the copies overlapped with
  * the compute.  Every pointer of layers_host[l] that ic_run_stack reads on
  * the device (qI, kI, w, kI8, kI_scale, Q, K, V) is read from host memory
