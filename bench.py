@@ -218,6 +218,20 @@ def run_ours(args, rank, world, local_rank):
                                "note": "the layer's K/V (8 MB) stays in L2: the gathered rows are "
                                        "served from L2, so the bound is the L2 random-row gather "
                                        "rate (see l2_gather_ceiling), not HBM"}
+        # Every gathered K/V byte crosses shared memory twice (the cp.async
+        # write, the ldmatrix read): against the SMs' nominal shared-memory
+        # bandwidth of 128 B per clock at the clock sampled during the timed
+        # steps, that is the floor of this staged design.
+        mhz = clk.get("sm_mhz") or clk.get("sm_max_mhz") or 1965.0
+        sms = torch.cuda.get_device_properties(stream.device).multi_processor_count
+        smem_bytes = 2 * keys * 2 * cfg.d * 2
+        smem_peak = sms * 128 * mhz * 1e6 / 1e9
+        smem_gbs = smem_bytes / (avg_ms / 1e3) / 1e9
+        roof["sparse_attn"]["smem_floor"] = {
+            "bytes_per_launch": smem_bytes, "peak_gbs": round(smem_peak, 1),
+            "achieved_gbs": round(smem_gbs, 1), "frac": round(smem_gbs / smem_peak, 4),
+            "floor_ms": round(smem_bytes / smem_peak / 1e6, 4),
+            "peak_kind": "nominal 128 B/clock/SM x %d SMs x %.0f MHz (sampled)" % (sms, mhz)}
         ceiling = measure_gather_ceiling(cache, layers[-1], L, k, stream)
         if ceiling:
             roof["sparse_attn"]["l2_gather_ceiling_gbs"] = ceiling["achieved_gbs"]

@@ -280,6 +280,12 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
                  "r"(valid ? 16 : 0)
                  : "memory");
 }
+// 4-byte copy (cp.async.ca); src-size 0 writes zeros and reads nothing
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, bool valid) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
+                 "r"(valid ? 4 : 0)
+                 : "memory");
+}
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {

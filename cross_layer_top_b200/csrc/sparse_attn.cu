@@ -53,7 +53,6 @@ struct AttnShape {
     // per-warp O and (m, l), then the per-head factors, M and L
     static constexpr int MERGE_BYTES = WARPS * (16 * D + 32) * 4 + (WARPS * 16 + 32) * 4 +
                                        (16 * D + 16 * 32 + 16 * 16 + 16) * 4;  // split rows
-    static constexpr float kRescaleThreshold = 8.0f;  // log2 units
     static_assert(MERGE_BYTES <= WARPS * WARP_BYTES, "merge buffer must fit in the stages");
 };
 
@@ -67,6 +66,97 @@ constexpr int kMaxClusterSplits = 8;
 template <int D>
 __device__ __forceinline__ uint32_t swz(int row, int c) {
     return static_cast<uint32_t>(row * (D * 2) + ((c ^ (row & 7)) << 4));
+}
+
+// One chunk of CH = 16 gathered slots (K rows at kb, V rows at vb, swizzled)
+// folded into a warp's running state: S = Q K^T on the tensor cores, slots
+// whose cmask bit is clear set to -inf, an online softmax in the base-2
+// domain with a lazy rescale (the reference m moves only when a logit passes
+// it by 2^kRescaleThreshold), then O += P V.  Rows g = lane/4 and g + 8 of
+// the 16 heads; m, l per row (l is this lane's partial sum).
+constexpr float kRescaleThreshold = 8.0f;  // log2 units
+
+template <int D>
+__device__ __forceinline__ void attn_chunk(uint32_t kb, uint32_t vb, uint32_t cmask,
+                                           const uint32_t (&qa)[D / 16][4], float (&o)[D / 8][4],
+                                           float& m0, float& m1, float& l0, float& l1,
+                                           float scale_log2, int lane) {
+    float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+    for (int kk = 0; kk < D / 16; ++kk) {
+        const int m = lane >> 3;
+        const int key = (m >> 1) * 8 + (lane & 7);
+        const int c = 2 * kk + (m & 1);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(kb + swz<D>(key, c), b0, b1, b2, b3);
+        mma_bf16_16816(s[0], qa[kk], b0, b1);
+        mma_bf16_16816(s[1], qa[kk], b2, b3);
+    }
+    if (cmask != 0xffffu) {  // warp-uniform: only chunks with masked slots
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+                const int col = nt * 8 + 2 * (lane & 3) + (e & 1);
+                if (!((cmask >> col) & 1u)) s[nt][e] = -INFINITY;
+            }
+    }
+    float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
+    float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
+    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
+    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
+    mx0 *= scale_log2;  // scale > 0 keeps the order
+    mx1 *= scale_log2;
+    // lazy rescale: move the reference only when a logit passes it by 2^8
+    if (mx0 > m0 + kRescaleThreshold) {
+        const float a = ex2_approx(m0 - mx0);  // 0 while nothing was seen
+        l0 *= a;
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) {
+            o[i][0] *= a;
+            o[i][1] *= a;
+        }
+        m0 = mx0;
+    }
+    if (mx1 > m1 + kRescaleThreshold) {
+        const float a = ex2_approx(m1 - mx1);
+        l1 *= a;
+#pragma unroll
+        for (int i = 0; i < D / 8; ++i) {
+            o[i][2] *= a;
+            o[i][3] *= a;
+        }
+        m1 = mx1;
+    }
+    const float n0 = m0 == -INFINITY ? 0.f : -m0;
+    const float n1 = m1 == -INFINITY ? 0.f : -m1;
+    float p[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+        p[nt][0] = ex2_approx(fmaf(s[nt][0], scale_log2, n0));
+        p[nt][1] = ex2_approx(fmaf(s[nt][1], scale_log2, n0));
+        p[nt][2] = ex2_approx(fmaf(s[nt][2], scale_log2, n1));
+        p[nt][3] = ex2_approx(fmaf(s[nt][3], scale_log2, n1));
+    }
+    l0 += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
+    l1 += (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
+    uint32_t pa[4];
+    pa[0] = pack_bf16x2(p[0][0], p[0][1]);
+    pa[1] = pack_bf16x2(p[0][2], p[0][3]);
+    pa[2] = pack_bf16x2(p[1][0], p[1][1]);
+    pa[3] = pack_bf16x2(p[1][2], p[1][3]);
+#pragma unroll
+    for (int dn = 0; dn < D / 16; ++dn) {
+        const int m = lane >> 3;
+        const int key = (m & 1) * 8 + (lane & 7);
+        const int c = 2 * dn + (m >> 1);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(vb + swz<D>(key, c), b0, b1, b2, b3);
+        mma_bf16_16816(o[2 * dn], pa, b0, b1);
+        mma_bf16_16816(o[2 * dn + 1], pa, b2, b3);
+    }
 }
 
 // SPLIT: rows split across a cluster of CTAs (few rows, decode); otherwise
@@ -192,82 +282,7 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, 2)
         const int c0 = (warp + j * S::WARPS) * S::CH;
         const uint32_t cmask = __ballot_sync(0xffffffffu, sIdx[c0 + (lane & 15)] >= 0) & 0xffffu;
 
-        float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-            const int m = lane >> 3;
-            const int key = (m >> 1) * 8 + (lane & 7);
-            const int c = 2 * kk + (m & 1);
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4(kb + swz<D>(key, c), b0, b1, b2, b3);
-            mma_bf16_16816(s[0], qa[kk], b0, b1);
-            mma_bf16_16816(s[1], qa[kk], b2, b3);
-        }
-        if (cmask != 0xffffu) {  // warp-uniform: only chunks with masked slots
-#pragma unroll
-            for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int col = nt * 8 + 2 * (lane & 3) + (e & 1);
-                    if (!((cmask >> col) & 1u)) s[nt][e] = -INFINITY;
-                }
-        }
-        float mx0 = fmaxf(fmaxf(s[0][0], s[0][1]), fmaxf(s[1][0], s[1][1]));
-        float mx1 = fmaxf(fmaxf(s[0][2], s[0][3]), fmaxf(s[1][2], s[1][3]));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 1));
-        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
-        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-        mx0 *= scale_log2;  // scale > 0 keeps the order
-        mx1 *= scale_log2;
-        // lazy rescale: move the reference only when a logit passes it by 2^8
-        if (mx0 > m0 + S::kRescaleThreshold) {
-            const float a = ex2_approx(m0 - mx0);  // 0 while nothing was seen
-            l0 *= a;
-#pragma unroll
-            for (int i = 0; i < D / 8; ++i) {
-                o[i][0] *= a;
-                o[i][1] *= a;
-            }
-            m0 = mx0;
-        }
-        if (mx1 > m1 + S::kRescaleThreshold) {
-            const float a = ex2_approx(m1 - mx1);
-            l1 *= a;
-#pragma unroll
-            for (int i = 0; i < D / 8; ++i) {
-                o[i][2] *= a;
-                o[i][3] *= a;
-            }
-            m1 = mx1;
-        }
-        const float n0 = m0 == -INFINITY ? 0.f : -m0;
-        const float n1 = m1 == -INFINITY ? 0.f : -m1;
-        float p[2][4];
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            p[nt][0] = ex2_approx(fmaf(s[nt][0], scale_log2, n0));
-            p[nt][1] = ex2_approx(fmaf(s[nt][1], scale_log2, n0));
-            p[nt][2] = ex2_approx(fmaf(s[nt][2], scale_log2, n1));
-            p[nt][3] = ex2_approx(fmaf(s[nt][3], scale_log2, n1));
-        }
-        l0 += (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
-        l1 += (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
-        uint32_t pa[4];
-        pa[0] = pack_bf16x2(p[0][0], p[0][1]);
-        pa[1] = pack_bf16x2(p[0][2], p[0][3]);
-        pa[2] = pack_bf16x2(p[1][0], p[1][1]);
-        pa[3] = pack_bf16x2(p[1][2], p[1][3]);
-#pragma unroll
-        for (int dn = 0; dn < D / 16; ++dn) {
-            const int m = lane >> 3;
-            const int key = (m & 1) * 8 + (lane & 7);
-            const int c = 2 * dn + (m >> 1);
-            uint32_t b0, b1, b2, b3;
-            ldsm_x4_t(vb + swz<D>(key, c), b0, b1, b2, b3);
-            mma_bf16_16816(o[2 * dn], pa, b0, b1);
-            mma_bf16_16816(o[2 * dn + 1], pa, b2, b3);
-        }
+        attn_chunk<D>(kb, vb, cmask, qa, o, m0, m1, l0, l1, scale_log2, lane);
         __syncwarp();              // every lane is done reading stage st
         issue(j + S::STAGES);      // refill it
     }

@@ -6,11 +6,14 @@
  * gather of sparse attention and nothing else: for each of `rows` query
  * rows it copies the k rows K[idx[r, j]], V[idx[r, j]] (d bf16 each) into
  * shared memory with 16-byte cp.async (4 warps per CTA, 2-deep per-warp
- * rings, ctas_per_sm CTAs per SM), then discards them.  Timing it with CUDA
+ * rings, ctas_per_sm CTAs per SM; each chunk's 16 index slots reach a
+ * shared ring two chunks before its gather is issued, so no gather waits
+ * on an index load), then discards them.  Timing it with CUDA
  * events gives the random-row gather ceiling (bytes = rows*k*2*d*2) that
  * bounds the attention kernel when K/V are resident in L2.
  *   K, V: device bf16 [kv_len, d]; idx: device int32 [rows, k], every entry
- *   in [0, kv_len).  d = 128, k a multiple of 64, 1 <= ctas_per_sm <= 3.
+ *   in [0, kv_len), 16-byte aligned.  d = 128, k a multiple of 64,
+ *   1 <= ctas_per_sm <= 3.
  * Returns IC_OK or IC_ERR_INVALID_ARG / IC_ERR_UNSUPPORTED / IC_ERR_CUDA;
  * asynchronous on `stream`; allocates nothing.
  *
