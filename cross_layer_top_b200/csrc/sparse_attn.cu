@@ -51,7 +51,10 @@ struct AttnShape {
     static constexpr int OFF_ST = OFF_LAST + 128;
     static constexpr int SMEM = OFF_ST + WARPS * WARP_BYTES;
     // per-warp O and (m, l), then the per-head factors, M and L
-    static constexpr int MERGE_BYTES = WARPS * (16 * D + 32) * 4 + (WARPS * 16 + 32) * 4 +
+    // per-warp partial O rows are OS = D + 8 floats apart (OS = 8 mod 32 banks):
+    // a warp's float2 fragment stores then take the minimal two wavefronts
+    static constexpr int OS = D + 8;
+    static constexpr int MERGE_BYTES = WARPS * (16 * OS + 32) * 4 + (WARPS * 16 + 32) * 4 +
                                        (16 * D + 16 * 32 + 16 * 16 + 16) * 4;  // split rows
     static_assert(MERGE_BYTES <= WARPS * WARP_BYTES, "merge buffer must fit in the stages");
 };
@@ -293,15 +296,16 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, 2)
     l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
     __syncthreads();  // every warp is done with its stages: reuse them for the merge
 
-    float* mO = reinterpret_cast<float*>(smem + S::OFF_ST);  // [WARPS][16][D]
-    float* mML = mO + S::WARPS * 16 * D;                     // [WARPS][32]: m[16], l[16]
+    float* mO = reinterpret_cast<float*>(smem + S::OFF_ST);  // [WARPS][16][OS]
+    float* mML = mO + S::WARPS * 16 * S::OS;                 // [WARPS][32]: m[16], l[16]
     {
         const int g = lane >> 2, cc = 2 * (lane & 3);
-        float* ow = mO + warp * 16 * D;
+        float* ow = mO + warp * 16 * S::OS;
 #pragma unroll
         for (int i = 0; i < D / 8; ++i) {
-            *reinterpret_cast<float2*>(ow + g * D + i * 8 + cc) = make_float2(o[i][0], o[i][1]);
-            *reinterpret_cast<float2*>(ow + (g + 8) * D + i * 8 + cc) = make_float2(o[i][2], o[i][3]);
+            *reinterpret_cast<float2*>(ow + g * S::OS + i * 8 + cc) = make_float2(o[i][0], o[i][1]);
+            *reinterpret_cast<float2*>(ow + (g + 8) * S::OS + i * 8 + cc) =
+                make_float2(o[i][2], o[i][3]);
         }
         if ((lane & 3) == 0) {
             mML[warp * 32 + g] = m0;
@@ -339,7 +343,7 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, 2)
 #pragma unroll
         for (int w = 0; w < S::WARPS; ++w) {
             const float f = sF[w * 16 + h];
-            const float4 v = *reinterpret_cast<const float4*>(mO + w * 16 * D + h * D + d4);
+            const float4 v = *reinterpret_cast<const float4*>(mO + (w * 16 + h) * S::OS + d4);
             acc.x = fmaf(v.x, f, acc.x);
             acc.y = fmaf(v.y, f, acc.y);
             acc.z = fmaf(v.z, f, acc.z);
