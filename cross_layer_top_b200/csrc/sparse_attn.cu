@@ -169,7 +169,7 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, 2)
     k_sparse_attn(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
                   const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ idx, int Hq,
                   int k, int rows_per_seq, long long kv_seq_stride, int kv_len, float scale_log2,
-                  int nsplit, int kps, int pf_ahead, __nv_bfloat16* __restrict__ out,
+                  int nsplit, int kps, int pf_ahead, int vec_idx, __nv_bfloat16* __restrict__ out,
                   int* __restrict__ err) {
     using S = AttnShape<D>;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -204,17 +204,30 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, 2)
     bool bad = false;
     int last = -1;
     const int nk_pad = (nk + S::CH - 1) / S::CH * S::CH;  // whole chunks, padded with -1
-    for (int i = tid; i < nk_pad; i += S::THREADS) {
-        int v = i < nk ? irow[i] : -1;
+    auto take = [&](int i, int v) {  // validate slot i; -1 (masked) for a bad index
         if (v < -1 || v >= kv_len) {
             bad = true;
             v = -1;
         }
-        sIdx[i] = v;
         if (v >= 0) last = i;
+        return v;
+    };
+    if (vec_idx) {  // 16-byte aligned slot rows, nk a multiple of 4: four slots per load
+        for (int i = 4 * tid; i < nk_pad; i += 4 * S::THREADS) {
+            int4 v = make_int4(-1, -1, -1, -1);
+            if (i < nk) v = __ldg(reinterpret_cast<const int4*>(irow + i));
+            v.x = take(i, v.x);
+            v.y = take(i + 1, v.y);
+            v.z = take(i + 2, v.z);
+            v.w = take(i + 3, v.w);
+            *reinterpret_cast<int4*>(sIdx + i) = v;
+        }
+    } else {
+        for (int i = tid; i < nk_pad; i += S::THREADS) sIdx[i] = take(i, i < nk ? irow[i] : -1);
     }
     if (bad) atomicCAS(err, 0, kDevBadIndex);
-    if (last >= 0) atomicMax(s_last, last);
+    last = __reduce_max_sync(0xffffffffu, last);
+    if (lane == 0 && last >= 0) atomicMax(s_last, last);
     const __nv_bfloat16* qrow = Q + static_cast<long long>(r) * Hq * D;
     for (int p = tid; p < 16 * (D / 8); p += S::THREADS) {
         const int h = p / (D / 8), c = p % (D / 8);
@@ -468,6 +481,8 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
     kps = (kps + S::CH - 1) / S::CH * S::CH;
     nsplit = (k + kps - 1) / kps;
     const float scale_log2 = scale * 1.4426950408889634f;
+    // slot rows start 16-byte aligned when idx does and k, kps are multiples of 4
+    const int vec_idx = (reinterpret_cast<uintptr_t>(idx) & 15) == 0 && k % 4 == 0 && kps % 4 == 0;
     LaunchScope ls(ctx, IC_K_ATTN, stream);
     const auto* Qp = static_cast<const __nv_bfloat16*>(Q);
     const auto* Kp = static_cast<const __nv_bfloat16*>(K);
@@ -477,7 +492,7 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
     if (nsplit == 1) {
         k_sparse_attn<D, false><<<dim3(rows, 1), S::THREADS, S::SMEM, stream>>>(
             Qp, Kp, Vp, idx, Hq, k, rows_per_seq, kvs, kv_len, scale_log2, 1, kps, 2 * ctx->num_sms,
-            op, ctx->dev_err);
+            vec_idx, op, ctx->dev_err);
     } else {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(rows, nsplit, 1);
@@ -492,7 +507,7 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
         cfg.attrs = attr;
         cfg.numAttrs = 1;
         cudaLaunchKernelEx(&cfg, k_sparse_attn<D, true>, Qp, Kp, Vp, idx, Hq, k, rows_per_seq, kvs, kv_len,
-                           scale_log2, nsplit, kps, 0, op, ctx->dev_err);
+                           scale_log2, nsplit, kps, 0, vec_idx, op, ctx->dev_err);
     }
     cudaError_t e = ls.done();
     if (e != cudaSuccess) return cuda_fail(ctx, e, "sparse_attn launch");
