@@ -50,6 +50,7 @@ struct alignas(16) TopkShared {
     uint32_t wsum[kTopkWarps];
     uint32_t wcnt[2][kTopkWarps];
     uint32_t ncand;
+    uint32_t wcand[kTopkWarps];  // staged rows: candidates in each warp's slice
     uint32_t bin;
     uint32_t above;
 };
@@ -105,7 +106,9 @@ template <bool IN_SMEM>
 __global__ void __launch_bounds__(kTopkThreads)
     k_topk(const float* __restrict__ scores, long long ld, int row0, int k, int causal_base,
            const int32_t* __restrict__ row_len, int max_len, int32_t* __restrict__ out,
-           long long ld_out, int pf_ahead) {
+           long long ld_out, int pf_ahead, int scap) {
+    // dynamic shared memory (IN_SMEM): the row's keys [scap], then the
+    // candidates' positions [kCandCap], then the selection bitmap
     extern __shared__ uint32_t srow[];
     __shared__ TopkShared S;
 
@@ -168,7 +171,41 @@ __global__ void __launch_bounds__(kTopkThreads)
     // ---- B: resolve bits 20..10 and 9..0 within bin b1
     uint32_t prefix = b1 << 21, mask = 0xFFE00000u;
     const bool use_cand = in_bin <= static_cast<uint32_t>(kCandCap);
-    if (use_cand) {
+    const int seg = ((n + kTopkWarps - 1) / kTopkWarps + 31) / 32 * 32;  // warp segments
+    const int sb = warp * seg, se = min(n, sb + seg);
+    const unsigned lt = (1u << lane) - 1u;
+    uint16_t* cpos = reinterpret_cast<uint16_t*>(srow + scap);  // IN_SMEM only
+    uint32_t* bits = reinterpret_cast<uint32_t*>(cpos + kCandCap);
+    constexpr int kSlice = kCandCap / kTopkWarps;  // candidate slots per warp
+    bool sliced = false;  // staged rows: candidates in per-warp slices of the list
+    if (IN_SMEM && use_cand) {
+        // one pass over the warp's segment: the keys above bin b1 (selected
+        // whatever T is) become bitmap words straight from the ballot; the
+        // keys of bin b1 go to the warp's own slice of the candidate list
+        // with their positions (a count in registers: no shared atomics)
+        uint32_t wc = 0;
+        for (int base = sb; base < se; base += 32) {
+            const int i = base + lane;
+            const bool in = i < se;
+            const uint32_t u = in ? srow[i] : 0u;
+            const unsigned wa = __ballot_sync(0xffffffffu, in && (u >> 21) > b1);
+            const unsigned wb = __ballot_sync(0xffffffffu, in && (u >> 21) == b1);
+            if (lane == 0) bits[base >> 5] = wa;
+            const uint32_t j = wc + __popc(wb & lt);
+            if (((wb >> lane) & 1u) && j < static_cast<uint32_t>(kSlice)) {
+                S.cand[warp * kSlice + j] = u;
+                cpos[warp * kSlice + j] = static_cast<uint16_t>(i);
+            }
+            wc += __popc(wb);
+        }
+        if (lane == 0) S.wcand[warp] = wc;
+        __syncthreads();
+        bool over = false;  // a slice overflowed: take the general path
+#pragma unroll
+        for (int w = 0; w < kTopkWarps; ++w) over |= S.wcand[w] > static_cast<uint32_t>(kSlice);
+        sliced = !over;
+    }
+    if (use_cand && !sliced) {
         for (int i = tid; i < n; i += kTopkThreads) {
             const uint32_t u = key_at(i);
             if ((u >> 21) == b1) S.cand[atomicAdd(&S.ncand, 1u)] = u;
@@ -176,13 +213,17 @@ __global__ void __launch_bounds__(kTopkThreads)
         __syncthreads();
     }
     const int ncand = use_cand ? static_cast<int>(S.ncand) : n;
+    // sliced: each warp walks its own slice; otherwise the threads stride the list (or row)
+    const int c0 = sliced ? warp * kSlice + lane : tid;
+    const int c1 = sliced ? warp * kSlice + static_cast<int>(S.wcand[warp]) : ncand;
+    const int cstep = sliced ? 32 : kTopkThreads;
 #pragma unroll 1
     for (int pass = 0; pass < 2; ++pass) {
         const int shift = pass == 0 ? 10 : 0;
         const uint32_t dmask = pass == 0 ? 0x7FFu : 0x3FFu;
         for (int i = tid; i < 2048; i += kTopkThreads) S.hist[i] = 0;
         __syncthreads();
-        for (int i = tid; i < ncand; i += kTopkThreads) {
+        for (int i = c0; i < c1; i += cstep) {
             const uint32_t u = use_cand ? S.cand[i] : key_at(i);
             if ((u & mask) == prefix) atomicAdd(&S.hist[(u >> shift) & dmask], 1u);
         }
@@ -198,9 +239,38 @@ __global__ void __launch_bounds__(kTopkThreads)
     }
     const uint32_t T = prefix;
 
-    // ---- C: per-warp segments, counts, offsets, ordered writes
-    const int seg = ((n + kTopkWarps - 1) / kTopkWarps + 31) / 32 * 32;
-    const int sb = warp * seg, se = min(n, sb + seg);
+    // ---- C (bitmap): when every key equal to T is taken, mark the
+    // candidates >= T in the bitmap and write its set positions in order
+    if (IN_SMEM && sliced && krem == S.hist[T & 0x3FFu]) {
+        for (int j = c0; j < c1; j += 32)
+            if (S.cand[j] >= T) {
+                const int pos = cpos[j];
+                atomicOr(&bits[pos >> 5], 1u << (pos & 31));
+            }
+        __syncthreads();
+        const int nw = (n + 31) >> 5;
+        const int wpt = (nw + kTopkThreads - 1) / kTopkThreads;  // words per thread
+        const int w0 = min(nw, tid * wpt), w1 = min(nw, w0 + wpt);
+        uint32_t cnt = 0;
+        for (int w = w0; w < w1; ++w) cnt += __popc(bits[w]);
+        uint32_t incl = cnt;  // inclusive scan of the counts in thread order
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t v = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += v;
+        }
+        if (lane == 31) S.wsum[warp] = incl;
+        __syncthreads();
+        uint32_t at = incl - cnt;
+#pragma unroll
+        for (int w = 0; w < kTopkWarps; ++w)
+            if (w < warp) at += S.wsum[w];
+        for (int w = w0; w < w1; ++w)
+            for (uint32_t x = bits[w]; x; x &= x - 1u) o[at++] = (w << 5) + (__ffs(x) - 1);
+        return;  // exactly k positions were written
+    }
+
+    // ---- C (ordered passes): per-warp segments, counts, offsets, writes
     uint32_t cg = 0, ce = 0;
     for (int base = sb; base < se; base += 32) {
         const int i = base + lane;
@@ -222,7 +292,6 @@ __global__ void __launch_bounds__(kTopkThreads)
             G += S.wcnt[0][w];
             E += S.wcnt[1][w];
         }
-    const unsigned lt = (1u << lane) - 1u;
     for (int base = sb; base < se; base += 32) {
         const int i = base + lane;
         uint32_t u = 0;
@@ -545,9 +614,9 @@ int launch_topk(ic_ctx* ctx, const float* scores, int64_t ld, int rows, int k, i
                                    ld_out, stream);
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_topk<true>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kTopkSmemCap * 4);
+        cudaError_t e = cudaFuncSetAttribute(
+            k_topk<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            kTopkSmemCap * 4 + kCandCap * 2 + kTopkSmemCap / 32 * 4);
         if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaFuncSetAttribute(topk)");
         attr_set = true;
     }
@@ -562,11 +631,13 @@ int launch_topk(ic_ctx* ctx, const float* scores, int64_t ld, int rows, int k, i
     }
     if (split > 0) {
         const int nmax = row_len ? max_len : causal_base + split;
-        const int smem = ((nmax < kTopkSmemCap ? nmax : kTopkSmemCap) + 3) / 4 * 16;
+        const int rowcap = nmax < kTopkSmemCap ? nmax : kTopkSmemCap;
+        const int scap = (rowcap + 3) / 4 * 4;  // keys; then positions, then the bitmap
+        const int smem = scap * 4 + kCandCap * 2 + ((rowcap + 31) / 32 + 3) / 4 * 16;
         LaunchScope ls(ctx, IC_K_TOPK, stream);
         k_topk<true><<<split, kTopkThreads, smem, stream>>>(scores, ld, 0, k, causal_base, row_len,
                                                              max_len, idx_out, ld_out,
-                                                             scores ? 2 * ctx->num_sms : 0);
+                                                             scores ? 2 * ctx->num_sms : 0, scap);
         cudaError_t e = ls.done();
         if (e != cudaSuccess) return cuda_fail(ctx, e, "topk launch");
     }
@@ -574,7 +645,7 @@ int launch_topk(ic_ctx* ctx, const float* scores, int64_t ld, int rows, int k, i
         LaunchScope ls(ctx, IC_K_TOPK, stream);
         k_topk<false><<<rows - split, kTopkThreads, 0, stream>>>(scores, ld, split, k, causal_base,
                                                                  row_len, max_len, idx_out, ld_out,
-                                                                 0);
+                                                                 0, 0);
         cudaError_t e = ls.done();
         if (e != cudaSuccess) return cuda_fail(ctx, e, "topk launch");
     }
