@@ -7,20 +7,25 @@
 // by -1 padding.  -0.0 and +0.0 compare equal.
 //
 // Algorithm (one 512-thread CTA per row), on order-preserving uint32 keys:
-//  A. one pass: keys (staged in shared memory when the row fits) and a
-//     2048-bin histogram of their top 11 bits;
-//  B. the bin holding the k-th largest key is found by a block suffix scan;
-//     the keys of that bin are compacted into a candidate list (usually a
-//     small fraction of the row) and two more radix digits (11 + 10 bits)
-//     are resolved on the candidates only.  If the bin is too large for
-//     the list (massive ties), those digits are resolved on the full row.
-//     Result: the threshold key T and krem, the number of keys equal to T
-//     still to take;
-//  C. each warp owns a contiguous segment of the row: it counts keys > T
-//     and == T, one block scan turns the counts into output offsets, and a
-//     second walk writes the selected positions in ascending order (a key
-//     == T is selected while fewer than krem equal keys precede it).
-// Rows that fit in shared memory are read from global memory once.
+//  A. one pass over the row: a 2048-bin histogram of the keys' top 11 bits;
+//     the bin b1 holding the k-th largest key is found by a block suffix
+//     scan;
+//  B. a second pass, each warp over a contiguous segment: the ballot of
+//     "bin above b1" is stored as a 32-bit word of a shared selection bitmap
+//     (those keys are selected whatever the threshold), and the keys of bin
+//     b1 go with their positions to the warp's own slice of a candidate
+//     list.  Two more radix digits (11 + 10 bits) are resolved on the
+//     candidates: the threshold key T and krem, the number of keys equal to
+//     T still to take;
+//  C. when every key equal to T is taken (no tie split), the candidates
+//     >= T are OR-ed into the bitmap and its set positions are written in
+//     ascending order (a block scan of the words' popcounts gives each
+//     warp's offset).  Otherwise (a tie split, a candidate bin too large
+//     for the list, or a row longer than the bitmap) the general path:
+//     digits resolved on the full row, then per-warp counts of keys > T and
+//     == T, a block scan, and an ordered walk that takes a key == T while
+//     fewer than krem equal keys precede it.
+// The row is read from global memory twice (L2 holds it between the passes).
 #include <cstddef>
 
 #include "ic_device.cuh"
@@ -30,13 +35,14 @@ namespace ic {
 
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
-constexpr int kTopkSmemCap = 32768;  // scores per row staged in shared memory
 constexpr int kCandCap = 4096;
+constexpr int kBitmapCap = 131072;  // longest row (keys) with a shared selection bitmap
 
 __device__ __forceinline__ uint32_t order_key(float x) {
-    uint32_t b = __float_as_uint(x);
-    if ((b & 0x7fffffffu) == 0) b = 0;  // -0.0 == +0.0
-    return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+    // x + (+0.0) turns -0.0 into +0.0 and leaves every other value as it is
+    const uint32_t b = __float_as_uint(__fadd_rn(x, 0.0f));
+    // negative: all bits flipped; non-negative: the sign bit set
+    return b ^ (static_cast<uint32_t>(static_cast<int32_t>(b) >> 31) | 0x80000000u);
 }
 // inverse of order_key (up to the sign of zero)
 __device__ __forceinline__ float key_float(uint32_t u) {
@@ -50,7 +56,7 @@ struct alignas(16) TopkShared {
     uint32_t wsum[kTopkWarps];
     uint32_t wcnt[2][kTopkWarps];
     uint32_t ncand;
-    uint32_t wcand[kTopkWarps];  // staged rows: candidates in each warp's slice
+    uint32_t wcand[kTopkWarps];  // bitmap path: candidates in each warp's slice
     uint32_t bin;
     uint32_t above;
 };
@@ -102,19 +108,18 @@ __device__ __forceinline__ void find_bin(TopkShared& S, uint32_t krem) {
     find_bin<NB>(S, krem, S.hist);
 }
 
-template <bool IN_SMEM>
 __global__ void __launch_bounds__(kTopkThreads)
-    k_topk(const float* __restrict__ scores, long long ld, int row0, int k, int causal_base,
+    k_topk(const float* __restrict__ scores, long long ld, int k, int causal_base,
            const int32_t* __restrict__ row_len, int max_len, int32_t* __restrict__ out,
-           long long ld_out, int pf_ahead, int scap) {
-    // dynamic shared memory (IN_SMEM): the row's keys [scap], then the
-    // candidates' positions [kCandCap], then the selection bitmap
-    extern __shared__ uint32_t srow[];
+           long long ld_out, int bcap) {
+    // dynamic shared memory: the candidates' positions [kCandCap], then the
+    // selection bitmap of rows up to bcap keys [bcap / 32]
+    extern __shared__ uint32_t dsm[];
     __shared__ TopkShared S;
 
-    const int r = row0 + blockIdx.x;
+    const int r = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    // a given length above max_len (what shared memory was sized for) counts as max_len
+    // a given length above max_len (the row stride) counts as max_len
     const int n = row_len ? min(row_len[r], max_len) : causal_base + r + 1;
     int32_t* o = out + static_cast<long long>(r) * ld_out;
     if (n <= k) {
@@ -122,22 +127,7 @@ __global__ void __launch_bounds__(kTopkThreads)
         return;
     }
     const float* row = scores + static_cast<long long>(r) * ld;
-    auto key_at = [&](int i) -> uint32_t {
-        return IN_SMEM ? srow[i] : order_key(__ldg(row + i));
-    };
-    // rows run about one wave of CTAs apart: warm L2 with the scores of the
-    // row one wave ahead, so whichever CTA takes it loads from L2
-    if (pf_ahead > 0 && static_cast<int>(blockIdx.x) + pf_ahead < static_cast<int>(gridDim.x)) {
-        const int rr = r + pf_ahead;
-        const int nn = row_len ? min(row_len[rr], max_len) : causal_base + rr + 1;
-        if (nn > k) {
-            const char* pr = reinterpret_cast<const char*>(scores + static_cast<long long>(rr) * ld);
-            const int lines = (nn * 4 + 127) / 128;
-            for (int i = tid; i < lines; i += kTopkThreads)
-                asm volatile("prefetch.global.L2 [%0];" ::"l"(pr + static_cast<long long>(i) * 128));
-        }
-    }
-
+    auto key_at = [&](int i) -> uint32_t { return order_key(__ldg(row + i)); };
     // ---- A: keys + histogram of the top 11 bits
     for (int i = tid; i < 2048; i += kTopkThreads) S.hist[i] = 0;
     if (tid == 0) S.ncand = 0;
@@ -149,7 +139,6 @@ __global__ void __launch_bounds__(kTopkThreads)
             const float4 v = __ldg(row4 + i);
             const uint32_t u0 = order_key(v.x), u1 = order_key(v.y);
             const uint32_t u2 = order_key(v.z), u3 = order_key(v.w);
-            if (IN_SMEM) *reinterpret_cast<uint4*>(srow + 4 * i) = make_uint4(u0, u1, u2, u3);
             atomicAdd(&S.hist[u0 >> 21], 1u);
             atomicAdd(&S.hist[u1 >> 21], 1u);
             atomicAdd(&S.hist[u2 >> 21], 1u);
@@ -157,7 +146,6 @@ __global__ void __launch_bounds__(kTopkThreads)
         }
         for (int i = 4 * n4 + tid; i < n; i += kTopkThreads) {
             const uint32_t u = order_key(__ldg(row + i));
-            if (IN_SMEM) srow[i] = u;
             atomicAdd(&S.hist[u >> 21], 1u);
         }
     }
@@ -174,11 +162,11 @@ __global__ void __launch_bounds__(kTopkThreads)
     const int seg = ((n + kTopkWarps - 1) / kTopkWarps + 31) / 32 * 32;  // warp segments
     const int sb = warp * seg, se = min(n, sb + seg);
     const unsigned lt = (1u << lane) - 1u;
-    uint16_t* cpos = reinterpret_cast<uint16_t*>(srow + scap);  // IN_SMEM only
-    uint32_t* bits = reinterpret_cast<uint32_t*>(cpos + kCandCap);
+    uint32_t* cpos = dsm;
+    uint32_t* bits = cpos + kCandCap;
     constexpr int kSlice = kCandCap / kTopkWarps;  // candidate slots per warp
-    bool sliced = false;  // staged rows: candidates in per-warp slices of the list
-    if (IN_SMEM && use_cand) {
+    bool sliced = false;  // candidates in per-warp slices of the list, bitmap path
+    if (use_cand && n <= bcap) {
         // one pass over the warp's segment: the keys above bin b1 (selected
         // whatever T is) become bitmap words straight from the ballot; the
         // keys of bin b1 go to the warp's own slice of the candidate list
@@ -187,14 +175,14 @@ __global__ void __launch_bounds__(kTopkThreads)
         for (int base = sb; base < se; base += 32) {
             const int i = base + lane;
             const bool in = i < se;
-            const uint32_t u = in ? srow[i] : 0u;
+            const uint32_t u = in ? key_at(i) : 0u;
             const unsigned wa = __ballot_sync(0xffffffffu, in && (u >> 21) > b1);
             const unsigned wb = __ballot_sync(0xffffffffu, in && (u >> 21) == b1);
             if (lane == 0) bits[base >> 5] = wa;
             const uint32_t j = wc + __popc(wb & lt);
             if (((wb >> lane) & 1u) && j < static_cast<uint32_t>(kSlice)) {
                 S.cand[warp * kSlice + j] = u;
-                cpos[warp * kSlice + j] = static_cast<uint16_t>(i);
+                cpos[warp * kSlice + j] = static_cast<uint32_t>(i);
             }
             wc += __popc(wb);
         }
@@ -241,7 +229,7 @@ __global__ void __launch_bounds__(kTopkThreads)
 
     // ---- C (bitmap): when every key equal to T is taken, mark the
     // candidates >= T in the bitmap and write its set positions in order
-    if (IN_SMEM && sliced && krem == S.hist[T & 0x3FFu]) {
+    if (sliced && krem == S.hist[T & 0x3FFu]) {
         for (int j = c0; j < c1; j += 32)
             if (S.cand[j] >= T) {
                 const int pos = cpos[j];
@@ -614,41 +602,21 @@ int launch_topk(ic_ctx* ctx, const float* scores, int64_t ld, int rows, int k, i
                                    ld_out, stream);
     static bool attr_set = false;
     if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(
-            k_topk<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-            kTopkSmemCap * 4 + kCandCap * 2 + kTopkSmemCap / 32 * 4);
+        cudaError_t e = cudaFuncSetAttribute(k_topk, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             kCandCap * 4 + kBitmapCap / 8);
         if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaFuncSetAttribute(topk)");
         attr_set = true;
     }
-    // Causal rows r have n = causal_base + r + 1: rows whose n fits in shared
-    // memory take the staged kernel, the rest the global-memory kernel.
-    int split = rows;  // rows [0, split) staged, [split, rows) global
-    if (row_len == nullptr) {
-        const long long fit = static_cast<long long>(kTopkSmemCap) - causal_base;  // n <= cap
-        split = fit < 0 ? 0 : (fit > rows ? rows : static_cast<int>(fit));
-    } else if (max_len > kTopkSmemCap) {
-        split = 0;
-    }
-    if (split > 0) {
-        const int nmax = row_len ? max_len : causal_base + split;
-        const int rowcap = nmax < kTopkSmemCap ? nmax : kTopkSmemCap;
-        const int scap = (rowcap + 3) / 4 * 4;  // keys; then positions, then the bitmap
-        const int smem = scap * 4 + kCandCap * 2 + ((rowcap + 31) / 32 + 3) / 4 * 16;
-        LaunchScope ls(ctx, IC_K_TOPK, stream);
-        k_topk<true><<<split, kTopkThreads, smem, stream>>>(scores, ld, 0, k, causal_base, row_len,
-                                                             max_len, idx_out, ld_out,
-                                                             scores ? 2 * ctx->num_sms : 0, scap);
-        cudaError_t e = ls.done();
-        if (e != cudaSuccess) return cuda_fail(ctx, e, "topk launch");
-    }
-    if (split < rows) {
-        LaunchScope ls(ctx, IC_K_TOPK, stream);
-        k_topk<false><<<rows - split, kTopkThreads, 0, stream>>>(scores, ld, split, k, causal_base,
-                                                                 row_len, max_len, idx_out, ld_out,
-                                                                 0, 0);
-        cudaError_t e = ls.done();
-        if (e != cudaSuccess) return cuda_fail(ctx, e, "topk launch");
-    }
+    // causal row r has n = causal_base + r + 1 keys; rows longer than the
+    // bitmap holds take the general path
+    const long long nmax = row_len ? max_len : static_cast<long long>(causal_base) + rows;
+    const int bcap = static_cast<int>(((nmax < kBitmapCap ? nmax : kBitmapCap) + 127) / 128 * 128);
+    const int smem = kCandCap * 4 + bcap / 8;
+    LaunchScope ls(ctx, IC_K_TOPK, stream);
+    k_topk<<<rows, kTopkThreads, smem, stream>>>(scores, ld, k, causal_base, row_len, max_len,
+                                                 idx_out, ld_out, bcap);
+    cudaError_t e = ls.done();
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "topk launch");
     return IC_OK;
 }
 
