@@ -272,6 +272,16 @@ __device__ __forceinline__ uint4 dsmem_ld_u4(uint32_t addr) {
 __device__ __forceinline__ float dsmem_ld_f32(uint32_t addr) {
     return __uint_as_float(dsmem_ld(addr));
 }
+// stores into another CTA's shared memory (visible to it after a cluster
+// barrier: arrive.release here, wait.acquire there)
+__device__ __forceinline__ void dsmem_st_f4(uint32_t addr, float4 v) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y),
+                 "f"(v.z), "f"(v.w)
+                 : "memory");
+}
+__device__ __forceinline__ void dsmem_st_f32(uint32_t addr, float v) {
+    asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
+}
 
 // ------------------------------------------------------- cp.async / ldmatrix
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {

@@ -16,10 +16,11 @@
 // reference only moves when a logit exceeds it by 2^8, so O is rarely
 // rescaled), and O += P V.  Slots holding -1 (or an out-of-range index,
 // which is also latched as an error) are masked and gather zeros; the
-// chunks after the last valid slot are skipped.  The four warps' (m, l, O)
+// chunks after the last valid slot are skipped.  The warps' (m, l, O)
 // merge through shared memory; one split writes bf16 output; with several
-// splits (decode) each CTA writes an fp32 partial and the row's last CTA to
-// finish merges them (counter + threadfence, no second launch).
+// splits (decode) the row's CTAs form a thread-block cluster and merge
+// through distributed shared memory (each CTA owns a share of the heads and
+// receives the other CTAs' partials of them).
 #include "ic_device.cuh"
 #include "ic_internal.h"
 
@@ -32,6 +33,10 @@
 #endif
 
 namespace ic {
+
+// Split rows: rows of the receive area, >= nsplit * ceil(16 / nsplit) for
+// every nsplit from 2 to 8 (at most 21, for nsplit = 7)
+constexpr int kRecvRows = 24;
 
 template <int D>
 struct AttnShape {
@@ -55,7 +60,7 @@ struct AttnShape {
     // a warp's float2 fragment stores then take the minimal two wavefronts
     static constexpr int OS = D + 8;
     static constexpr int MERGE_BYTES = WARPS * (16 * OS + 32) * 4 + (WARPS * 16 + 32) * 4 +
-                                       (16 * D + 16 * 32 + 16 * 16 + 16) * 4;  // split rows
+                                       (kRecvRows * D + kRecvRows * 2) * 4;  // split: receive area
     static_assert(MERGE_BYTES <= WARPS * WARP_BYTES, "merge buffer must fit in the stages");
 };
 
@@ -332,7 +337,6 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, 2)
     // L = sum_w l_w f_w (computed once per head), then o = sum_w O_w f_w
     // over float4 columns
     float* sF = mML + S::WARPS * 32;  // [WARPS][16] factors, then M[16], L[16]
-    float* pO = sF + S::WARPS * 16 + 32;  // split rows: this CTA's combined O [16][D]
     if (tid < 16) {
         const int h = tid;
         float M = -INFINITY;
@@ -349,9 +353,8 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, 2)
         sF[S::WARPS * 16 + 16 + h] = L;
     }
     __syncthreads();
-    const int hmax = SPLIT ? 16 : Hq;
-    for (int e4 = tid; e4 < hmax * (D / 4); e4 += S::THREADS) {
-        const int h = e4 / (D / 4), d4 = (e4 % (D / 4)) * 4;
+    // this CTA's combined o[h][d4..d4+3] = sum_w O_w f_w (relative to its M[h])
+    auto combine = [&](int h, int d4) {
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
         for (int w = 0; w < S::WARPS; ++w) {
@@ -362,66 +365,68 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, 2)
             acc.z = fmaf(v.z, f, acc.z);
             acc.w = fmaf(v.w, f, acc.w);
         }
-        const float L = sF[S::WARPS * 16 + 16 + h];
-        if (!SPLIT) {
+        return acc;
+    };
+    if (!SPLIT) {
+        for (int e4 = tid; e4 < Hq * (D / 4); e4 += S::THREADS) {
+            const int h = e4 / (D / 4), d4 = (e4 % (D / 4)) * 4;
+            const float4 acc = combine(h, d4);
+            const float L = sF[S::WARPS * 16 + 16 + h];
             const float iv = L > 0.f ? 1.f / L : 0.f;
             __nv_bfloat16* op = out + (static_cast<long long>(r) * Hq + h) * D + d4;
             *reinterpret_cast<uint2*>(op) = make_uint2(pack_bf16x2(acc.x * iv, acc.y * iv),
                                                        pack_bf16x2(acc.z * iv, acc.w * iv));
-        } else {
-            *reinterpret_cast<float4*>(pO + h * D + d4) = acc;  // this split's partial O
         }
+        return;
     }
-    if (!SPLIT) return;
 
-    // Split rows: the row's nsplit CTAs form one thread-block cluster and
-    // merge their partial states through distributed shared memory,
-    //   out = sum_q O_q 2^(M_q - M) / sum_q L_q 2^(M_q - M),  M = max_q M_q;
-    // CTA q of the cluster produces every nsplit-th group of outputs.  Every
-    // CTA reaches both cluster barriers: the first publishes the partials,
-    // the second keeps each CTA's shared memory alive until all have read it.
+    // Split rows: the row's nsplit CTAs form one thread-block cluster.  CTA q
+    // owns heads [q*hpc, (q+1)*hpc); every CTA stores its combined partial of
+    // those heads (O relative to its M, and M, L) into the owner's receive
+    // area with distributed-shared-memory stores, and each owner merges
+    //   out = sum_q O_q 2^(M_q - M) / sum_q L_q 2^(M_q - M),  M = max_q M_q.
+    // The first cluster barrier is reached once every CTA's gather ring is
+    // idle (the receive area lies in the ring, past this CTA's merge
+    // buffers); the second makes the stores visible.  After it each CTA reads
+    // only its own shared memory, so it may exit when done.
     cluster_sync_all();
-    float* cML = pO + 16 * D;       // [nsplit][32]: every split's M[16], L[16]
-    float* cF = cML + 16 * 32;      // [nsplit][16] factors, then 1/L [16]
-    // one parallel round of remote loads for all splits' (M, L)
-    for (int t = tid; t < nsplit * 32; t += S::THREADS)
-        cML[t] = dsmem_ld_f32(dsmem_addr(sF + S::WARPS * 16 + (t & 31), t >> 5));
-    __syncthreads();
-    if (tid < 16) {
-        const int h = tid;
-        float M = -INFINITY;
-        for (int q = 0; q < nsplit; ++q) M = fmaxf(M, cML[q * 32 + h]);
-        float Lt = 0.f;
-        for (int q = 0; q < nsplit; ++q) {
-            const float f = M == -INFINITY ? 0.f : ex2_approx(cML[q * 32 + h] - M);
-            cF[q * 16 + h] = f;
-            Lt += cML[q * 32 + 16 + h] * f;
-        }
-        cF[nsplit * 16 + h] = Lt > 0.f ? 1.f / Lt : 0.f;
-    }
-    __syncthreads();
-    for (int e4 = split * S::THREADS + tid; e4 < Hq * (D / 4); e4 += nsplit * S::THREADS) {
+    const int hpc = (16 + nsplit - 1) / nsplit;  // heads per owner
+    const uint32_t q = cluster_rank();
+    float* rO = sF + S::WARPS * 16 + 32;           // [nsplit][hpc][D] received partial O
+    float* rML = rO + kRecvRows * D;               // [nsplit][hpc][2] received M, L
+    for (int e4 = tid; e4 < 16 * (D / 4); e4 += S::THREADS) {
         const int h = e4 / (D / 4), d4 = (e4 % (D / 4)) * 4;
-        float4 v[kMaxClusterSplits];
-#pragma unroll
-        for (int q = 0; q < kMaxClusterSplits; ++q)  // all remote loads in flight at once
-            if (q < nsplit) v[q] = dsmem_ld_f4(dsmem_addr(pO + h * D + d4, q));
+        const int owner = h / hpc, hl = h - owner * hpc;
+        dsmem_st_f4(dsmem_addr(rO + (q * hpc + hl) * D + d4, owner), combine(h, d4));
+    }
+    if (tid < 16) {
+        const int h = tid, owner = h / hpc, hl = h - owner * hpc;
+        dsmem_st_f32(dsmem_addr(rML + (q * hpc + hl) * 2, owner), sF[S::WARPS * 16 + h]);
+        dsmem_st_f32(dsmem_addr(rML + (q * hpc + hl) * 2 + 1, owner), sF[S::WARPS * 16 + 16 + h]);
+    }
+    cluster_sync_all();
+    for (int e4 = tid; e4 < hpc * (D / 4); e4 += S::THREADS) {
+        const int hl = e4 / (D / 4), d4 = (e4 % (D / 4)) * 4;
+        const int h = static_cast<int>(q) * hpc + hl;
+        if (h >= Hq) continue;
+        float M = -INFINITY;
+        for (int p = 0; p < nsplit; ++p) M = fmaxf(M, rML[(p * hpc + hl) * 2]);
+        float L = 0.f;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-        for (int q = 0; q < kMaxClusterSplits; ++q)
-            if (q < nsplit) {
-                const float f = cF[q * 16 + h];
-                acc.x = fmaf(v[q].x, f, acc.x);
-                acc.y = fmaf(v[q].y, f, acc.y);
-                acc.z = fmaf(v[q].z, f, acc.z);
-                acc.w = fmaf(v[q].w, f, acc.w);
-            }
-        const float iv = cF[nsplit * 16 + h];
+        for (int p = 0; p < nsplit; ++p) {
+            const float f = M == -INFINITY ? 0.f : ex2_approx(rML[(p * hpc + hl) * 2] - M);
+            L += rML[(p * hpc + hl) * 2 + 1] * f;
+            const float4 v = *reinterpret_cast<const float4*>(rO + (p * hpc + hl) * D + d4);
+            acc.x = fmaf(v.x, f, acc.x);
+            acc.y = fmaf(v.y, f, acc.y);
+            acc.z = fmaf(v.z, f, acc.z);
+            acc.w = fmaf(v.w, f, acc.w);
+        }
+        const float iv = L > 0.f ? 1.f / L : 0.f;
         __nv_bfloat16* op = out + (static_cast<long long>(r) * Hq + h) * D + d4;
         *reinterpret_cast<uint2*>(op) = make_uint2(pack_bf16x2(acc.x * iv, acc.y * iv),
                                                    pack_bf16x2(acc.z * iv, acc.w * iv));
     }
-    cluster_sync_all();
 }
 
 template <int D>
