@@ -283,6 +283,20 @@ __device__ __forceinline__ void dsmem_st_f32(uint32_t addr, float v) {
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
+// ------------------------------------------ programmatic dependent launch
+// Wait until the previous kernel in the stream has completed and its writes
+// are visible (returns at once when the kernel was not launched as a
+// programmatic dependent).
+__device__ __forceinline__ void griddep_wait() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+// Let the next kernel in the stream (launched as a programmatic dependent)
+// start; called only after griddep_wait, so that a dependent that starts
+// early still finds every kernel before this one complete.
+__device__ __forceinline__ void griddep_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
 // ------------------------------------------------------- cp.async / ldmatrix
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
     // src-size 0 fills the 16 bytes with zeros and reads nothing

@@ -30,6 +30,12 @@ struct ic_ctx {
     int64_t launches[IC_K_COUNT] = {0};
     int64_t launch_count = 0;
     int graphs_alive = 0;           // captured stack graphs that use this context's buffers
+    // Programmatic dependent launch, set by the decode stack around its own
+    // launches: 0 off; 1 the kernel may start while the previous kernel in the
+    // stream finishes and waits for it before reading anything; 2 (attention
+    // of an S layer) it may also read the index cache and warm L2 with the
+    // K/V rows it will gather before that wait.
+    int pdl = 0;
     // ic_run_stack_host: two device staging slots, a copy-in and a copy-out
     // stream, and per-slot events (created on first use)
     struct HostStack {
@@ -54,6 +60,15 @@ int cuda_fail(ic_ctx* ctx, cudaError_t e, const char* what);
 
 // Brackets one kernel launch with timing events when timing is enabled and
 // counts it.  Usage: LaunchScope ls(ctx, IC_K_TOPK, stream); kernel<<<>>>; ls.done();
+// Appends the programmatic-dependent-launch attribute to attrs[n] when the
+// context asks for it (ctx->pdl != 0).
+inline void add_pdl_attr(const ic_ctx* ctx, cudaLaunchAttribute* attrs, unsigned int& n) {
+    if (!ctx->pdl) return;
+    attrs[n].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attrs[n].val.programmaticStreamSerializationAllowed = 1;
+    ++n;
+}
+
 struct LaunchScope {
     ic_ctx* ctx;
     int kernel;

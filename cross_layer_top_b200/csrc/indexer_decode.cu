@@ -165,6 +165,9 @@ __global__ void __launch_bounds__(512, 1)
     const long long total = static_cast<long long>(B) * tps;
     const long long g_begin = total * blockIdx.x / gridDim.x;
     const long long g_end = total * (blockIdx.x + 1) / gridDim.x;
+    // as a programmatic dependent: nothing is read before the previous kernel completes
+    griddep_wait();
+    griddep_launch_dependents();
 
     if (threadIdx.x == 0) {
         *abort_flag = 0;
@@ -503,10 +506,20 @@ static int launch_decode_t(ic_ctx* ctx, const void* q, const void* w, const uint
     const int tps = (S_max + S::BM - 1) / S::BM;
     const long long total = static_cast<long long>(B) * tps;
     const int grid = total < ctx->num_sms ? static_cast<int>(total) : ctx->num_sms;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid, 1, 1);
+    cfg.blockDim = dim3(512, 1, 1);
+    cfg.dynamicSmemBytes = S::SMEM;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    unsigned int na = 0;
+    add_pdl_attr(ctx, attr, na);
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
     LaunchScope ls(ctx, IC_K_INDEX_SCORE_DECODE, stream);
-    k_index_score_decode<H_I><<<grid, 512, S::SMEM, stream>>>(
-        tm_k, static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(w), kI_scale,
-        seq_len, B, S_max, tps, scores, static_cast<long long>(ld), ctx->dev_err);
+    cudaLaunchKernelEx(&cfg, k_index_score_decode<H_I>, tm_k, static_cast<const __nv_bfloat16*>(q),
+                       static_cast<const __nv_bfloat16*>(w), kI_scale, seq_len, B, S_max, tps,
+                       scores, static_cast<long long>(ld), ctx->dev_err);
     cudaError_t e = ls.done();
     if (e != cudaSuccess) return cuda_fail(ctx, e, "index_score_decode launch");
     return IC_OK;

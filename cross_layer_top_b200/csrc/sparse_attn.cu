@@ -174,7 +174,8 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, 2)
     k_sparse_attn(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
                   const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ idx, int Hq,
                   int k, int rows_per_seq, long long kv_seq_stride, int kv_len, float scale_log2,
-                  int nsplit, int kps, int pf_ahead, int vec_idx, __nv_bfloat16* __restrict__ out,
+                  int nsplit, int kps, int pf_ahead, int vec_idx, int pdl,
+                  __nv_bfloat16* __restrict__ out,
                   int* __restrict__ err) {
     using S = AttnShape<D>;
     extern __shared__ __align__(128) uint8_t smem[];
@@ -204,6 +205,9 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, 2)
     }
     if (tid == 0) *s_last = -1;
     __syncthreads();
+    // as a programmatic dependent (pdl 1): nothing is read before the previous
+    // kernel completes; pdl 2 (an S layer) waits below, after the index slots
+    if (pdl != 2) griddep_wait();
     // index slots of this split (validated), the last valid slot, the query heads
     const int32_t* irow = idx + static_cast<long long>(r) * k + slot0;
     bool bad = false;
@@ -233,6 +237,25 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, 2)
     if (bad) atomicCAS(err, 0, kDevBadIndex);
     last = __reduce_max_sync(0xffffffffu, last);
     if (lane == 0 && last >= 0) atomicMax(s_last, last);
+    if (pdl == 2) {
+        // An S layer's index slots and its cached K/V rows are not written by
+        // the previous kernel: warm L2 with the rows this split will gather,
+        // then wait for that kernel before reading the query heads (and, in
+        // the main loop, the rows themselves, the newest one included).
+        __syncthreads();  // every slot is staged
+        constexpr int LPR = (D * 2 + 127) / 128;  // 128-byte lines per row
+        for (int t = tid; t < nk * 2 * LPR; t += S::THREADS) {
+            const int slot = t / (2 * LPR), part = t - slot * (2 * LPR);
+            const int v = sIdx[slot];
+            if (v >= 0) {
+                const char* row = reinterpret_cast<const char*>(part < LPR ? Kb : Vb) +
+                                  static_cast<long long>(v) * D * 2 + (part % LPR) * 128;
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(row));
+            }
+        }
+        griddep_wait();
+    }
+    griddep_launch_dependents();
     const __nv_bfloat16* qrow = Q + static_cast<long long>(r) * Hq * D;
     for (int p = tid; p < 16 * (D / 8); p += S::THREADS) {
         const int h = p / (D / 8), c = p % (D / 8);
@@ -495,24 +518,36 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
     auto* op = static_cast<__nv_bfloat16*>(out);
     const long long kvs = static_cast<long long>(kv_seq_stride);
     if (nsplit == 1) {
-        k_sparse_attn<D, false><<<dim3(rows, 1), S::THREADS, S::SMEM, stream>>>(
-            Qp, Kp, Vp, idx, Hq, k, rows_per_seq, kvs, kv_len, scale_log2, 1, kps, 2 * ctx->num_sms,
-            vec_idx, op, ctx->dev_err);
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(rows, 1, 1);
+        cfg.blockDim = dim3(S::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = S::SMEM;
+        cfg.stream = stream;
+        cudaLaunchAttribute attr[1];
+        unsigned int na = 0;
+        add_pdl_attr(ctx, attr, na);
+        cfg.attrs = attr;
+        cfg.numAttrs = na;
+        cudaLaunchKernelEx(&cfg, k_sparse_attn<D, false>, Qp, Kp, Vp, idx, Hq, k, rows_per_seq, kvs,
+                           kv_len, scale_log2, 1, kps, 2 * ctx->num_sms, vec_idx, ctx->pdl, op,
+                           ctx->dev_err);
     } else {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(rows, nsplit, 1);
         cfg.blockDim = dim3(S::THREADS, 1, 1);
         cfg.dynamicSmemBytes = S::SMEM;
         cfg.stream = stream;
-        cudaLaunchAttribute attr[1];
+        cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
         attr[0].val.clusterDim.x = 1;
         attr[0].val.clusterDim.y = nsplit;
         attr[0].val.clusterDim.z = 1;
+        unsigned int na = 1;
+        add_pdl_attr(ctx, attr, na);
         cfg.attrs = attr;
-        cfg.numAttrs = 1;
+        cfg.numAttrs = na;
         cudaLaunchKernelEx(&cfg, k_sparse_attn<D, true>, Qp, Kp, Vp, idx, Hq, k, rows_per_seq, kvs, kv_len,
-                           scale_log2, nsplit, kps, 0, vec_idx, op, ctx->dev_err);
+                           scale_log2, nsplit, kps, 0, vec_idx, ctx->pdl, op, ctx->dev_err);
     }
     cudaError_t e = ls.done();
     if (e != cudaSuccess) return cuda_fail(ctx, e, "sparse_attn launch");

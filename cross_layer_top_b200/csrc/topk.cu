@@ -119,6 +119,9 @@ __global__ void __launch_bounds__(kTopkThreads)
 
     const int r = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // as a programmatic dependent: nothing is read before the previous kernel completes
+    griddep_wait();
+    griddep_launch_dependents();
     // a given length above max_len (the row stride) counts as max_len
     const int n = row_len ? min(row_len[r], max_len) : causal_base + r + 1;
     int32_t* o = out + static_cast<long long>(r) * ld_out;
@@ -336,6 +339,9 @@ __global__ void __launch_bounds__(kTopkThreads)
     const int r = blockIdx.y;
     const uint32_t rank = cluster_rank();
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    // as a programmatic dependent: nothing is read before the previous kernel completes
+    griddep_wait();
+    griddep_launch_dependents();
     const int n = row_len ? min(row_len[r], max_len) : causal_base + r + 1;
     int32_t* o = out + static_cast<long long>(r) * ld_out;
     if (n <= k) {  // the same for every CTA of the cluster: no cluster barrier is reached
@@ -576,13 +582,15 @@ static int launch_topk_cluster(ic_ctx* ctx, const float* scores, int64_t ld, int
     cfg.blockDim = dim3(kTopkThreads, 1, 1);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = kClusterCtas;
     attr[0].val.clusterDim.y = 1;
     attr[0].val.clusterDim.z = 1;
+    unsigned int na = 1;
+    add_pdl_attr(ctx, attr, na);
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = na;
     LaunchScope ls(ctx, IC_K_TOPK, stream);
     cudaLaunchKernelEx(&cfg, k_topk_cluster, scores, static_cast<long long>(ld), k, row_len,
                        max_len, causal_base, idx_out, static_cast<long long>(ld_out), seg_cap);
@@ -612,9 +620,19 @@ int launch_topk(ic_ctx* ctx, const float* scores, int64_t ld, int rows, int k, i
     const long long nmax = row_len ? max_len : static_cast<long long>(causal_base) + rows;
     const int bcap = static_cast<int>(((nmax < kBitmapCap ? nmax : kBitmapCap) + 127) / 128 * 128);
     const int smem = kCandCap * 4 + bcap / 8;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(rows, 1, 1);
+    cfg.blockDim = dim3(kTopkThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    unsigned int na = 0;
+    add_pdl_attr(ctx, attr, na);
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
     LaunchScope ls(ctx, IC_K_TOPK, stream);
-    k_topk<<<rows, kTopkThreads, smem, stream>>>(scores, ld, k, causal_base, row_len, max_len,
-                                                 idx_out, ld_out, bcap);
+    cudaLaunchKernelEx(&cfg, k_topk, scores, static_cast<long long>(ld), k, causal_base, row_len,
+                       max_len, idx_out, static_cast<long long>(ld_out), bcap);
     cudaError_t e = ls.done();
     if (e != cudaSuccess) return cuda_fail(ctx, e, "topk launch");
     return IC_OK;
