@@ -275,7 +275,14 @@ typedef struct ic_stack_dims {
 /* [IC] Figure 2: for l = 0..N-1, if c_l = F run the indexer and top-k into
  * idx_cache (device int32 [rows, k], overwritten), else reuse idx_cache as
  * it stands; then sparse attention of layer l with its own Q/K/V at those
- * indices.  Everything is enqueued on `stream` with no host sync. */
+ * indices.  Everything is enqueued on `stream` with no host sync.
+ * Decode stacks with B * 8 <= the SM count launch each kernel as a
+ * programmatic dependent of the one before it: a kernel may start before
+ * its predecessor in the stream finishes, but reads nothing a previous
+ * kernel writes until that predecessor has completed, except that an S
+ * layer's attention reads the index cache and prefetches (into L2 only) the
+ * K/V rows at those slots first.  A caller's own kernel before the stack is
+ * always complete before the stack reads anything. */
 int ic_run_stack(ic_ctx *ctx, const ic_pattern *pattern, const ic_layer_io *layers,
                  const ic_stack_dims *dims, int32_t *idx_cache, void *stream);
 
