@@ -290,13 +290,23 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, 2)
     for (int i = 0; i < NI; ++i) dsto[i] = swz<D>(prow + i * RPI, piece);
     const char* Kc = reinterpret_cast<const char*>(Kb) + piece * 16;
     const char* Vc = reinterpret_cast<const char*>(Vb) + piece * 16;
+    static_assert(RPI == 2 || RPI == 4, "slot selection below");
     auto issue = [&](int j) {
         if (j < my_n) {
             const int c0 = (warp + j * S::WARPS) * S::CH;
             const uint32_t kdst = wst + (j % S::STAGES) * S::STAGE_BYTES;
+            // the chunk's CH slots as CH / 4 16-byte broadcast loads; this lane's
+            // rows prow + i * RPI sit in vector (i * RPI) / 4, element
+            // prow + (i * RPI) % 4
+            int4 sv[S::CH / 4];
+#pragma unroll
+            for (int q = 0; q < S::CH / 4; ++q) sv[q] = *reinterpret_cast<const int4*>(sIdx + c0 + 4 * q);
 #pragma unroll
             for (int i = 0; i < NI; ++i) {
-                const int sidx = sIdx[c0 + prow + i * RPI];
+                const int4 v = sv[(i * RPI) / 4];
+                const bool b0 = prow & 1;
+                const bool b1 = RPI == 2 ? ((i * RPI) & 2) != 0 : (prow & 2) != 0;
+                const int sidx = b1 ? (b0 ? v.w : v.z) : (b0 ? v.y : v.x);
                 const bool ok = sidx >= 0;
                 const uint32_t off = static_cast<uint32_t>(ok ? sidx : 0) * S::ROWB;
                 cp_async16(kdst + dsto[i], Kc + off, ok);
