@@ -20,9 +20,10 @@
 //    shared memory while the causal key tiles 0..t_last/128 stream through
 //    a TMA ring.  Two 256-column TMEM accumulators ping-pong so the epilogue
 //    of one overlaps the MMAs of the other.
-//  * Warp roles (384 threads, one CTA per SM, persistent): warp 0 = TMA
-//    producer, warp 1 = MMA issuer, warp 2 = TMEM allocator, warps 4..11 =
-//    epilogue (warp w reads TMEM lanes 32*(w%4).., columns half (w-4)/4).
+//  * Warp roles (one CTA per SM, persistent): warp 0 = TMA producer, warp 1
+//    = MMA issuer, warp 2 = TMEM allocator, warps 4.. = epilogue (8 for bf16,
+//    16 for e4m3; warp w reads TMEM lanes 32*(w%4).. and column group
+//    (w-4)/4 of each accumulator).
 //  * Work items are handed out longest-first (latest rows first), round
 //    robin over the persistent CTAs.
 //  * Every mbarrier wait is bounded; on timeout the CTA aborts cleanly
@@ -46,7 +47,12 @@ struct PrefillShape {
     static constexpr int B_ATOM = BN * 128;
     static constexpr int B_ACC = NATOM * B_ATOM;
     static constexpr int B_BYTES = NACC * B_ACC;
-    static constexpr int W_BYTES = 8 * 1024;       // per epilogue warp: 256 fp32 weights
+    // epilogue warps: at the fp8 MMA rate 8 warps (two per TMEM lane
+    // quarter) score too slowly, so e4m3 inputs take 16
+    static constexpr int EPI = F8 ? 16 : 8;
+    static constexpr int THREADS = (4 + EPI) * 32;
+    static constexpr int COLS = BN / (EPI / 4);    // columns per epilogue warp and accumulator
+    static constexpr int W_BYTES = 8 * 1024;       // EPI warps x NACC x COLS fp32 weights
     static constexpr int BAR_BYTES = 256;
     static constexpr int SMEM_CAP = 232448;
     static constexpr int KST_RAW = (SMEM_CAP - B_BYTES - W_BYTES - BAR_BYTES) / A_STAGE;
@@ -63,7 +69,7 @@ struct PrefillShape {
 // (token-major, head-minor, same order as the columns).  Produces one score
 // per token covered (64 / H_I tokens).
 template <int H_I, int NATOM, bool F8>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(PrefillShape<H_I, NATOM, F8>::THREADS, 1)
     k_index_score_prefill(const __grid_constant__ CUtensorMap tm_q,
                           const __grid_constant__ CUtensorMap tm_k,
                           const __nv_bfloat16* __restrict__ w, const float* __restrict__ q_scale,
@@ -104,7 +110,7 @@ __global__ void __launch_bounds__(384, 1)
         mbar_init(q_empty, 1);
         for (int i = 0; i < 2; ++i) {
             mbar_init(&acc_full[i], 1);
-            mbar_init(&acc_empty[i], 8);  // one arrival per epilogue warp
+            mbar_init(&acc_empty[i], S::EPI);  // one arrival per epilogue warp
         }
         mbar_init(done_bar, 1);
         fence_mbar_init();
@@ -232,13 +238,16 @@ __global__ void __launch_bounds__(384, 1)
         if (!mbar_wait_drain(done_bar, 0)) atomicCAS(err, 0, kDevTimeoutDrain);
     } else if (warp >= 4 && start_ok) {
         // ------------------------------------------------ epilogue
-        const int ew = warp - 4;  // 0..7
+        constexpr int COLS = S::COLS;
+        constexpr int CPL = COLS / 32;        // staged weights per lane and accumulator
+        constexpr int NCHUNK = COLS / 32;     // 32-column TMEM loads per accumulator
+        const int ew = warp - 4;  // 0..EPI-1
         const int lq = warp & 3;  // TMEM lane quarter
-        const int cg = ew >> 2;   // column half of each accumulator
-        float* wW = sW + ew * 256;  // this warp's weights: [acc][128 columns]
+        const int cg = ew >> 2;   // column group of each accumulator
+        float* wW = sW + ew * 2 * COLS;  // this warp's weights: [acc][COLS columns]
         uint32_t acc_it[2] = {0, 0};
         bool ok = true;
-        constexpr int TOK_PER_HALF = 128 / H_I;  // tokens in this warp's 128 columns
+        constexpr int TOK_PER_HALF = COLS / H_I;  // tokens in this warp's columns
         for (int it = blockIdx.x; it < n_items && ok; it += gridDim.x) {
             const int t0 = row_begin + (n_items - 1 - it) * S::TQ;
             const int t_last = min(t0 + S::TQ, row_end) - 1;
@@ -251,13 +260,13 @@ __global__ void __launch_bounds__(384, 1)
             for (int a = 0; a < 2; ++a) {
                 const int tok0 = t0 + a * S::TOK_PER_ACC + cg * TOK_PER_HALF;
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int c = lane * 4 + q;  // column within the half
+                for (int q = 0; q < CPL; ++q) {
+                    const int c = lane * CPL + q;  // column within the group
                     const int t = tok0 + c / H_I;
                     const size_t wi = static_cast<size_t>(t) * H_I + (c % H_I);
                     float wv = t < L ? __bfloat162float(w[wi]) : 0.f;
                     if (F8 && t < L) wv *= q_scale[wi];
-                    wW[a * 128 + c] = wv;
+                    wW[a * COLS + c] = wv;
                 }
             }
             __syncwarp();
@@ -277,9 +286,9 @@ __global__ void __launch_bounds__(384, 1)
                     ++acc_it[a];
                     tc_fence_after();
                     const uint32_t taddr = tmem + (static_cast<uint32_t>(lq * 32) << 16) +
-                                           static_cast<uint32_t>(a * S::BN + cg * 128);
+                                           static_cast<uint32_t>(a * S::BN + cg * COLS);
                     const int tok_base = a * S::TOK_PER_ACC + cg * TOK_PER_HALF;
-                    const float* wa = wW + a * 128;
+                    const float* wa = wW + a * COLS;
                     // 32-column chunks: chunk c + 1 is loaded while chunk c is
                     // scored.  Four partial sums per token (heads 0, 1, 2, 3
                     // mod 4) as two packed pairs; a token's score is stored as
@@ -289,8 +298,8 @@ __global__ void __launch_bounds__(384, 1)
                     tmem_ld_wait();
                     uint64_t p01 = 0, p23 = 0;
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        if (c < 3) tmem_ld32(taddr + (c + 1) * 32, buf[(c + 1) & 1]);
+                    for (int c = 0; c < NCHUNK; ++c) {
+                        if (c < NCHUNK - 1) tmem_ld32(taddr + (c + 1) * 32, buf[(c + 1) & 1]);
                         const uint32_t(&v)[32] = buf[c & 1];
 #pragma unroll
                         for (int j = 0; j < 32; j += 4) {
@@ -311,9 +320,9 @@ __global__ void __launch_bounds__(384, 1)
                                 p23 = 0;
                             }
                         }
-                        if (c < 3) {
+                        if (c < NCHUNK - 1) {
                             tmem_ld_wait();
-                            if (c == 2) {
+                            if (c == NCHUNK - 2) {
                                 // all of this accumulator is in registers: hand it back
                                 tc_fence_before();
                                 __syncwarp();
@@ -363,7 +372,7 @@ static int launch_prefill_t(ic_ctx* ctx, const void* qI, const void* kI, const v
     const int n_items = (row_end - row_begin + S::TQ - 1) / S::TQ;
     const int grid = n_items < ctx->num_sms ? n_items : ctx->num_sms;
     LaunchScope ls(ctx, IC_K_INDEX_SCORE, stream);
-    kern<<<grid, 384, S::SMEM, stream>>>(tm_q, tm_k, static_cast<const __nv_bfloat16*>(w), q_scale,
+    kern<<<grid, S::THREADS, S::SMEM, stream>>>(tm_q, tm_k, static_cast<const __nv_bfloat16*>(w), q_scale,
                                          k_scale, scores, static_cast<long long>(ld), L, row_begin,
                                          row_end, n_items, ctx->dev_err);
     cudaError_t e = ls.done();
