@@ -291,16 +291,18 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, 2)
     const char* Kc = reinterpret_cast<const char*>(Kb) + piece * 16;
     const char* Vc = reinterpret_cast<const char*>(Vb) + piece * 16;
     static_assert(RPI == 2 || RPI == 4, "slot selection below");
-    auto issue = [&](int j) {
-        if (j < my_n) {
-            const int c0 = (warp + j * S::WARPS) * S::CH;
-            const uint32_t kdst = wst + (j % S::STAGES) * S::STAGE_BYTES;
-            // the chunk's CH slots as CH / 4 16-byte broadcast loads; this lane's
-            // rows prow + i * RPI sit in vector (i * RPI) / 4, element
-            // prow + (i * RPI) % 4
-            int4 sv[S::CH / 4];
+    // a chunk's CH slots as CH / 4 16-byte broadcast loads (chunks past the
+    // warp's last read chunk 0's, unused)
+    auto load_slots = [&](int j, int4 (&sv)[S::CH / 4]) {
+        const int c0 = (warp + (j < my_n ? j : 0) * S::WARPS) * S::CH;
 #pragma unroll
-            for (int q = 0; q < S::CH / 4; ++q) sv[q] = *reinterpret_cast<const int4*>(sIdx + c0 + 4 * q);
+        for (int q = 0; q < S::CH / 4; ++q) sv[q] = *reinterpret_cast<const int4*>(sIdx + c0 + 4 * q);
+    };
+    // gather chunk j's K and V rows into its stage; this lane's rows
+    // prow + i * RPI sit in vector (i * RPI) / 4, element prow + (i * RPI) % 4
+    auto issue_with = [&](int j, const int4 (&sv)[S::CH / 4]) {
+        if (j < my_n) {
+            const uint32_t kdst = wst + (j % S::STAGES) * S::STAGE_BYTES;
 #pragma unroll
             for (int i = 0; i < NI; ++i) {
                 const int4 v = sv[(i * RPI) / 4];
@@ -314,6 +316,11 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, 2)
             }
         }
         cp_async_commit();
+    };
+    auto issue = [&](int j) {
+        int4 sv[S::CH / 4];
+        load_slots(j, sv);
+        issue_with(j, sv);
     };
 
     float o[D / 8][4];
@@ -336,9 +343,13 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, 2)
         const int c0 = (warp + j * S::WARPS) * S::CH;
         const uint32_t cmask = __ballot_sync(0xffffffffu, sIdx[c0 + (lane & 15)] >= 0) & 0xffffu;
 
+        // the slots of the gather that refills this stage are read before the
+        // compute, so their latency is not paid between chunks
+        int4 nsv[S::CH / 4];
+        load_slots(j + S::STAGES, nsv);
         attn_chunk<D>(kb, vb, cmask, qa, o, m0, m1, l0, l1, scale_log2, lane);
-        __syncwarp();              // every lane is done reading stage st
-        issue(j + S::STAGES);      // refill it
+        __syncwarp();                    // every lane is done reading stage st
+        issue_with(j + S::STAGES, nsv);  // refill it
     }
     cp_async_wait<0>();
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
