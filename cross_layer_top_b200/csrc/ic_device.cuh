@@ -81,9 +81,6 @@ __device__ __forceinline__ bool mbar_wait_drain(uint64_t* bar, uint32_t parity) 
     return true;
 }
 
-__device__ __forceinline__ void named_bar_sync(int id, int nthreads) {
-    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
-}
 
 // ----------------------------------------------------------------------- TMA
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
@@ -99,16 +96,6 @@ __device__ __forceinline__ void tma_load_2d(void* dst, const CUtensorMap* map, u
         : "memory");
 }
 
-// 1-D bulk copy global -> this CTA's shared memory, completing on `bar`
-// (both addresses 16-byte aligned, bytes a multiple of 16).
-__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
-                                          uint64_t* bar) {
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            dst),
-        "l"(src), "r"(bytes), "r"(smem_u32(bar))
-        : "memory");
-}
 
 // ------------------------------------------------------------------- tcgen05
 __device__ __forceinline__ void tmem_alloc(uint32_t* dst_smem, uint32_t ncols) {
@@ -253,14 +240,6 @@ __device__ __forceinline__ uint32_t dsmem_ld(uint32_t addr) {
     return v;
 }
 
-__device__ __forceinline__ float4 dsmem_ld_f4(uint32_t addr) {
-    float4 v;
-    asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-                 : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
-                 : "r"(addr)
-                 : "memory");
-    return v;
-}
 __device__ __forceinline__ uint4 dsmem_ld_u4(uint32_t addr) {
     uint4 v;
     asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];"
@@ -268,9 +247,6 @@ __device__ __forceinline__ uint4 dsmem_ld_u4(uint32_t addr) {
                  : "r"(addr)
                  : "memory");
     return v;
-}
-__device__ __forceinline__ float dsmem_ld_f32(uint32_t addr) {
-    return __uint_as_float(dsmem_ld(addr));
 }
 // stores into another CTA's shared memory (visible to it after a cluster
 // barrier: arrive.release here, wait.acquire there)
@@ -302,12 +278,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool v
     // src-size 0 fills the 16 bytes with zeros and reads nothing
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src),
                  "r"(valid ? 16 : 0)
-                 : "memory");
-}
-// 4-byte copy (cp.async.ca); src-size 0 writes zeros and reads nothing
-__device__ __forceinline__ void cp_async4(uint32_t dst, const void* src, bool valid) {
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst), "l"(src),
-                 "r"(valid ? 4 : 0)
                  : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
