@@ -5,7 +5,7 @@
 // Accelerating Sparse Attention via Cross-Layer Index Reuse", Figure 2 step
 // SPARSEATTN).  One K/V head is shared by all Hq <= 16 query heads.
 //
-// Design: one CTA (6 warps, two CTAs per SM) per (query row, key split).
+// Design: one CTA (4 warps, three CTAs per SM) per (query row, key split).
 // The 16 query heads form the M = 16 rows of mma.m16n8k16 tiles, so one
 // gathered K/V row serves every head.  Each warp owns chunks of 16 index
 // slots and a 2-deep ring: lane l always copies the same 16-byte piece
@@ -26,7 +26,7 @@
 
 // Warps per CTA and gather-ring depth (compile-time tuning knobs).
 #ifndef IC_ATTN_WARPS
-#define IC_ATTN_WARPS 6
+#define IC_ATTN_WARPS 4
 #endif
 #ifndef IC_ATTN_STAGES
 #define IC_ATTN_STAGES 2
@@ -50,11 +50,17 @@ struct AttnShape {
     static constexpr int WARP_BYTES = STAGES * STAGE_BYTES;
     static constexpr int Q_BYTES = 16 * ROWP;
     static constexpr int MAXK = 2048;
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_IDX = Q_BYTES;
+    static constexpr int OFF_IDX = 0;
     static constexpr int OFF_LAST = OFF_IDX + MAXK * 4;
     static constexpr int OFF_ST = OFF_LAST + 128;
+    // Q is staged in the last warp's second ring buffer: every warp reads it
+    // into registers before any gather fills that buffer
+    static constexpr int OFF_Q = OFF_ST + (WARPS - 1) * WARP_BYTES + STAGE_BYTES;
     static constexpr int SMEM = OFF_ST + WARPS * WARP_BYTES;
+    // resident CTAs per SM (228 KB of shared memory, 1 KB reserved per CTA);
+    // three 4-warp CTAs keep three rows' prologues and merges in flight
+    static constexpr int CTAS_PER_SM = 3 * (SMEM + 1024) <= 233472 ? 3 : 2;
+    static_assert(Q_BYTES <= STAGE_BYTES && STAGES >= 2, "Q lives in a second ring buffer");
     // per-warp O and (m, l), then the per-head factors, M and L
     // per-warp partial O rows are OS = D + 8 floats apart (OS = 8 mod 32 banks):
     // a warp's float2 fragment stores then take the minimal two wavefronts
@@ -170,7 +176,7 @@ __device__ __forceinline__ void attn_chunk(uint32_t kb, uint32_t vb, uint32_t cm
 // SPLIT: rows split across a cluster of CTAs (few rows, decode); otherwise
 // one CTA per row, and the cluster merge is not compiled in.
 template <int D, bool SPLIT>
-__global__ void __launch_bounds__(AttnShape<D>::THREADS, 2)
+__global__ void __launch_bounds__(AttnShape<D>::THREADS, AttnShape<D>::CTAS_PER_SM)
     k_sparse_attn(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
                   const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ idx, int Hq,
                   int k, int rows_per_seq, long long kv_seq_stride, int kv_len, float scale_log2,
@@ -274,6 +280,7 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, 2)
         const int c = 2 * kk + (m >> 1);
         ldsm_x4(sQ + swz<D>(row, c), qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
     }
+    __syncthreads();  // every warp holds Q: its staging buffer may now be filled
 
     const uint32_t wst = smem_u32(smem + S::OFF_ST + warp * S::WARP_BYTES);
     const int nch = (nk_eff + S::CH - 1) / S::CH;
@@ -490,7 +497,7 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
         attr_set = true;
     }
     // Split the index slots across CTAs when there are too few rows to fill
-    // the GPU (decode): about one wave at two CTAs per SM, whole chunks per
+    // the GPU (decode): about one wave of resident CTAs, whole chunks per
     // split, at most kMaxClusterSplits.  A split row's CTAs form one cluster
     // (they merge through distributed shared memory); the split count is
     // lowered until every row's cluster can be resident at once (a cluster
@@ -517,7 +524,7 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
         return active[cs];
     };
     int nsplit = 1;
-    const int target = 2 * ctx->num_sms;
+    const int target = S::CTAS_PER_SM * ctx->num_sms;
     if (rows < target) {
         nsplit = target / rows;
         const int max_split = (k + S::CH - 1) / S::CH;
@@ -550,8 +557,8 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
         cfg.attrs = attr;
         cfg.numAttrs = na;
         cudaLaunchKernelEx(&cfg, k_sparse_attn<D, false>, Qp, Kp, Vp, idx, Hq, k, rows_per_seq, kvs,
-                           kv_len, scale_log2, 1, kps, 2 * ctx->num_sms, vec_idx, ctx->pdl, op,
-                           ctx->dev_err);
+                           kv_len, scale_log2, 1, kps, S::CTAS_PER_SM * ctx->num_sms, vec_idx,
+                           ctx->pdl, op, ctx->dev_err);
     } else {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(rows, nsplit, 1);
