@@ -60,13 +60,17 @@ struct AttnShape {
     // resident CTAs per SM (228 KB of shared memory, 1 KB reserved per CTA);
     // three 4-warp CTAs keep three rows' prologues and merges in flight
     static constexpr int CTAS_PER_SM = 3 * (SMEM + 1024) <= 233472 ? 3 : 2;
+    // split rows: a receive area of its own past the ring, for the cluster
+    // merge ([kRecvRows][D] partial O, then [kRecvRows][2] M, L)
+    static constexpr int OFF_RECV = SMEM;
+    static constexpr int SMEM_SPLIT = OFF_RECV + (kRecvRows * D + kRecvRows * 2) * 4;
+    static constexpr int CTAS_SPLIT = 233472 / (SMEM_SPLIT + 1024) < 3 ? 233472 / (SMEM_SPLIT + 1024) : 3;
     static_assert(Q_BYTES <= STAGE_BYTES && STAGES >= 2, "Q lives in a second ring buffer");
     // per-warp O and (m, l), then the per-head factors, M and L
     // per-warp partial O rows are OS = D + 8 floats apart (OS = 8 mod 32 banks):
     // a warp's float2 fragment stores then take the minimal two wavefronts
     static constexpr int OS = D + 8;
-    static constexpr int MERGE_BYTES = WARPS * (16 * OS + 32) * 4 + (WARPS * 16 + 32) * 4 +
-                                       (kRecvRows * D + kRecvRows * 2) * 4;  // split: receive area
+    static constexpr int MERGE_BYTES = WARPS * (16 * OS + 32) * 4 + (WARPS * 16 + 32) * 4;
     static_assert(MERGE_BYTES <= WARPS * WARP_BYTES, "merge buffer must fit in the stages");
 };
 
@@ -76,6 +80,12 @@ struct AttnShape {
 // CTAs of one split row's cluster, at most: the portable cluster size (on
 // back-to-back decode layers 8-CTA clusters schedule better than 16 or 4)
 constexpr int kMaxClusterSplits = 8;
+// receive rows an owner needs for nsplit splits of 16 heads: nsplit * ceil(16 / nsplit)
+constexpr int recv_rows_for(int n) {
+    return n <= 1 ? 16 : (n * ((16 + n - 1) / n) > recv_rows_for(n - 1) ? n * ((16 + n - 1) / n)
+                                                                          : recv_rows_for(n - 1));
+}
+static_assert(recv_rows_for(kMaxClusterSplits) <= kRecvRows, "receive area holds every split");
 
 template <int D>
 __device__ __forceinline__ uint32_t swz(int row, int c) {
@@ -176,7 +186,8 @@ __device__ __forceinline__ void attn_chunk(uint32_t kb, uint32_t vb, uint32_t cm
 // SPLIT: rows split across a cluster of CTAs (few rows, decode); otherwise
 // one CTA per row, and the cluster merge is not compiled in.
 template <int D, bool SPLIT>
-__global__ void __launch_bounds__(AttnShape<D>::THREADS, AttnShape<D>::CTAS_PER_SM)
+__global__ void __launch_bounds__(AttnShape<D>::THREADS,
+                                  SPLIT ? AttnShape<D>::CTAS_SPLIT : AttnShape<D>::CTAS_PER_SM)
     k_sparse_attn(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
                   const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ idx, int Hq,
                   int k, int rows_per_seq, long long kv_seq_stride, int kv_len, float scale_log2,
@@ -209,11 +220,29 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, AttnShape<D>::CTAS_PER_
         else if (tid < idx_lines + q_lines)
             asm volatile("prefetch.global.L2 [%0];" ::"l"(pq + (tid - idx_lines) * 128));
     }
+    // a split row's CTAs arrive on the cluster barrier at once and wait on it
+    // only before their first remote store, so that every CTA of the cluster
+    // is known to be running by then
+    if constexpr (SPLIT) cluster_arrive_relaxed();
     if (tid == 0) *s_last = -1;
     __syncthreads();
+    // the query heads go to shared memory by cp.async, in flight while the
+    // index slots load (zeros for heads past Hq)
+    const __nv_bfloat16* qrow = Q + static_cast<long long>(r) * Hq * D;
+    auto stage_q = [&]() {
+        for (int p = tid; p < 16 * (D / 8); p += S::THREADS) {
+            const int h = p / (D / 8), c = p % (D / 8);
+            const bool ok = h < Hq;
+            cp_async16(sQ + swz<D>(h, c), ok ? qrow + h * D + c * 8 : qrow, ok);
+        }
+        cp_async_commit();
+    };
     // as a programmatic dependent (pdl 1): nothing is read before the previous
     // kernel completes; pdl 2 (an S layer) waits below, after the index slots
-    if (pdl != 2) griddep_wait();
+    if (pdl != 2) {
+        griddep_wait();
+        stage_q();
+    }
     // index slots of this split (validated), the last valid slot, the query heads
     const int32_t* irow = idx + static_cast<long long>(r) * k + slot0;
     bool bad = false;
@@ -260,15 +289,10 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, AttnShape<D>::CTAS_PER_
             }
         }
         griddep_wait();
+        stage_q();
     }
     griddep_launch_dependents();
-    const __nv_bfloat16* qrow = Q + static_cast<long long>(r) * Hq * D;
-    for (int p = tid; p < 16 * (D / 8); p += S::THREADS) {
-        const int h = p / (D / 8), c = p % (D / 8);
-        uint4 v = make_uint4(0, 0, 0, 0);
-        if (h < Hq) v = *reinterpret_cast<const uint4*>(qrow + h * D + c * 8);
-        *reinterpret_cast<uint4*>(smem + S::OFF_Q + swz<D>(h, c)) = v;
-    }
+    cp_async_wait<0>();
     __syncthreads();
     const int nk_eff = *s_last + 1;  // slots after the last valid one hold nothing
 
@@ -436,15 +460,15 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, AttnShape<D>::CTAS_PER_
     // those heads (O relative to its M, and M, L) into the owner's receive
     // area with distributed-shared-memory stores, and each owner merges
     //   out = sum_q O_q 2^(M_q - M) / sum_q L_q 2^(M_q - M),  M = max_q M_q.
-    // The first cluster barrier is reached once every CTA's gather ring is
-    // idle (the receive area lies in the ring, past this CTA's merge
-    // buffers); the second makes the stores visible.  After it each CTA reads
-    // only its own shared memory, so it may exit when done.
-    cluster_sync_all();
+    // The receive area is used by nothing else, so a CTA stores as soon as
+    // its own partial is ready; one cluster barrier (arrive with release,
+    // wait with acquire) then makes every store visible to its owner.  After
+    // it each CTA reads only its own shared memory, so it may exit when done.
+    cluster_wait_acquire();  // every CTA of the cluster is running
     const int hpc = (16 + nsplit - 1) / nsplit;  // heads per owner
     const uint32_t q = cluster_rank();
-    float* rO = sF + S::WARPS * 16 + 32;           // [nsplit][hpc][D] received partial O
-    float* rML = rO + kRecvRows * D;               // [nsplit][hpc][2] received M, L
+    float* rO = reinterpret_cast<float*>(smem + S::OFF_RECV);  // [nsplit][hpc][D] received O
+    float* rML = rO + kRecvRows * D;                           // [nsplit][hpc][2] received M, L
     for (int e4 = tid; e4 < 16 * (D / 4); e4 += S::THREADS) {
         const int h = e4 / (D / 4), d4 = (e4 % (D / 4)) * 4;
         const int owner = h / hpc, hl = h - owner * hpc;
@@ -455,7 +479,8 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS, AttnShape<D>::CTAS_PER_
         dsmem_st_f32(dsmem_addr(rML + (q * hpc + hl) * 2, owner), sF[S::WARPS * 16 + h]);
         dsmem_st_f32(dsmem_addr(rML + (q * hpc + hl) * 2 + 1, owner), sF[S::WARPS * 16 + 16 + h]);
     }
-    cluster_sync_all();
+    cluster_arrive_release();
+    cluster_wait_acquire();
     for (int e4 = tid; e4 < hpc * (D / 4); e4 += S::THREADS) {
         const int hl = e4 / (D / 4), d4 = (e4 % (D / 4)) * 4;
         const int h = static_cast<int>(q) * hpc + hl;
@@ -492,7 +517,7 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(k_sparse_attn<D, true>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_SPLIT);
         if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaFuncSetAttribute(sparse_attn)");
         attr_set = true;
     }
@@ -508,7 +533,7 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
             cudaLaunchConfig_t q = {};
             q.gridDim = dim3(1, cs, 1);
             q.blockDim = dim3(S::THREADS, 1, 1);
-            q.dynamicSmemBytes = S::SMEM;
+            q.dynamicSmemBytes = S::SMEM_SPLIT;
             cudaLaunchAttribute qa[1];
             qa[0].id = cudaLaunchAttributeClusterDimension;
             qa[0].val.clusterDim.x = 1;
@@ -563,7 +588,7 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(rows, nsplit, 1);
         cfg.blockDim = dim3(S::THREADS, 1, 1);
-        cfg.dynamicSmemBytes = S::SMEM;
+        cfg.dynamicSmemBytes = S::SMEM_SPLIT;
         cfg.stream = stream;
         cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
