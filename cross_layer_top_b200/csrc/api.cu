@@ -172,7 +172,7 @@ extern "C" int ic_ctx_destroy(ic_ctx* ctx) {
     cudaFree(ctx->scores);
     cudaFree(ctx->dev_err);
     if (ctx->hs.ready) {
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < ic_ctx::kHostSlots; ++i) {
             cudaFree(ctx->hs.slot[i]);
             cudaEventDestroy(ctx->hs.in_ready[i]);
             cudaEventDestroy(ctx->hs.computed[i]);

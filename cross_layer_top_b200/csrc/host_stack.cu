@@ -2,15 +2,17 @@
 // Attention via Cross-Layer Index Reuse", Figure 2) on inputs that live in
 // host memory, with the host<->device copies overlapped with the compute.
 //
-// The context stages the layers through two device slots.  Layer l uses slot
-// l % 2:
-//   copy-in stream : wait until layer l-2 has computed (its inputs are no
+// The context stages the layers through n = 4 device slots.  Layer l uses
+// slot l % n:
+//   copy-in stream : wait until layer l-n has computed (its inputs are no
 //                    longer read), copy layer l's inputs in, record in_ready;
-//   caller's stream: wait in_ready and until layer l-2's output has been
+//   caller's stream: wait in_ready and until layer l-n's output has been
 //                    copied out, run the layer, record computed;
 //   copy-out stream: wait computed, copy the output to host, record out_done.
-// So layer l+1's inputs cross PCIe while layer l computes, and layer l's
-// output crosses back while layer l+1 computes.  The events persist in the
+// So later layers' inputs cross PCIe while layer l computes, and layer l's
+// output crosses back while the next layers compute.  With two slots the
+// copy-in stream would idle behind every layer that computes longer than
+// the next layer's inputs take to copy (an F layer followed by S layers).  The events persist in the
 // context, which also orders consecutive calls.  At the end the caller's
 // stream waits for the last outputs, so its completion means every output
 // is in host memory.
@@ -60,7 +62,7 @@ int init_host_stack(ic_ctx* ctx) {
     if (hs.ready) return IC_OK;
     cudaError_t e = cudaStreamCreateWithFlags(&hs.in, cudaStreamNonBlocking);
     if (e == cudaSuccess) e = cudaStreamCreateWithFlags(&hs.out, cudaStreamNonBlocking);
-    for (int i = 0; i < 2 && e == cudaSuccess; ++i) {
+    for (int i = 0; i < ic_ctx::kHostSlots && e == cudaSuccess; ++i) {
         e = cudaEventCreateWithFlags(&hs.in_ready[i], cudaEventDisableTiming);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hs.computed[i], cudaEventDisableTiming);
         if (e == cudaSuccess) e = cudaEventCreateWithFlags(&hs.out_done[i], cudaEventDisableTiming);
@@ -89,20 +91,21 @@ extern "C" int ic_run_stack_host(ic_ctx* ctx, const ic_pattern* pattern,
         if (e == cudaSuccess) e = cudaStreamSynchronize(hs.out);
         if (e == cudaSuccess) e = cudaDeviceSynchronize();
         if (e != cudaSuccess) return cuda_fail(ctx, e, "run_stack_host: drain before regrow");
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < ic_ctx::kHostSlots; ++i) {
             cudaFree(hs.slot[i]);
             hs.slot[i] = nullptr;
         }
         hs.slot_cap = 0;
-        for (int i = 0; i < 2; ++i) {
+        for (int i = 0; i < ic_ctx::kHostSlots; ++i) {
             e = cudaMalloc(&hs.slot[i], need);
             if (e != cudaSuccess) {
-                for (int j = 0; j < 2; ++j) {
+                for (int j = 0; j < ic_ctx::kHostSlots; ++j) {
                     cudaFree(hs.slot[j]);
                     hs.slot[j] = nullptr;
                 }
                 cudaGetLastError();
-                return fail(ctx, IC_ERR_NOMEM, "run_stack_host: two slots of %zu bytes", need);
+                return fail(ctx, IC_ERR_NOMEM, "run_stack_host: %d slots of %zu bytes",
+                            ic_ctx::kHostSlots, need);
             }
         }
         hs.slot_cap = need;
@@ -110,7 +113,7 @@ extern "C" int ic_run_stack_host(ic_ctx* ctx, const ic_pattern* pattern,
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const int N = static_cast<int>(pattern->c.size());
     for (int l = 0; l < N; ++l) {
-        const int sl = l & 1;
+        const int sl = l % ic_ctx::kHostSlots;
         const ic_layer_io& h = layers_host[l];
         if (!h.Q || !h.K || !h.V || !h.out)
             return fail(ctx, IC_ERR_INVALID_ARG, "run_stack_host: layer %d lacks Q/K/V/out", l);
@@ -167,8 +170,9 @@ extern "C" int ic_run_stack_host(ic_ctx* ctx, const ic_pattern* pattern,
         if (e == cudaSuccess) e = cudaEventRecord(hs.out_done[sl], hs.out);
         if (e != cudaSuccess) return cuda_fail(ctx, e, "run_stack_host: copy out");
     }
-    cudaError_t e = cudaStreamWaitEvent(s, hs.out_done[0], 0);
-    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, hs.out_done[1], 0);
+    cudaError_t e = cudaSuccess;
+    for (int i = 0; i < ic_ctx::kHostSlots && e == cudaSuccess; ++i)
+        e = cudaStreamWaitEvent(s, hs.out_done[i], 0);
     if (e != cudaSuccess) return cuda_fail(ctx, e, "run_stack_host: final wait");
     return IC_OK;
 }

@@ -36,13 +36,14 @@ struct ic_ctx {
     // of an S layer) it may also read the index cache and warm L2 with the
     // K/V rows it will gather before that wait.
     int pdl = 0;
-    // ic_run_stack_host: two device staging slots, a copy-in and a copy-out
-    // stream, and per-slot events (created on first use)
+    // ic_run_stack_host: kHostSlots device staging slots, a copy-in and a
+    // copy-out stream, and per-slot events (created on first use)
+    static constexpr int kHostSlots = 4;
     struct HostStack {
         bool ready = false;
         cudaStream_t in = nullptr, out = nullptr;
-        cudaEvent_t in_ready[2] = {}, computed[2] = {}, out_done[2] = {};
-        void* slot[2] = {nullptr, nullptr};
+        cudaEvent_t in_ready[kHostSlots] = {}, computed[kHostSlots] = {}, out_done[kHostSlots] = {};
+        void* slot[kHostSlots] = {};
         size_t slot_cap = 0;  // bytes per slot
     } hs;
 };

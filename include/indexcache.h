@@ -309,14 +309,15 @@ int ic_stack_graph_destroy(ic_graph *graph);
  * instead, and out receives the layer's output in host memory; use pinned
  * (page-locked) host memory, or the copies neither overlap nor run at full
  * speed.  idx_snapshot (optional), idx_cache and dims->seq_len stay on the
- * device.  The context stages layers through two device slots sized for the
- * largest layer (allocated on first use, grown when dims grow): layer l+1's
- * inputs are copied in on a context-owned stream while layer l computes on
- * `stream`, and layer l's output is copied out on another context-owned
- * stream while layer l+1 computes.  Asynchronous: when `stream` reaches the
- * point after this call, every output is in host memory; the host inputs
- * must not change before then.  Errors as ic_run_stack, plus IC_ERR_NOMEM
- * when the two slots cannot be allocated. */
+ * device.  The context stages layers through four device slots, each sized
+ * for the largest layer (allocated on first use, grown when dims grow):
+ * later layers' inputs are copied in on a context-owned stream while layer l
+ * computes on `stream` (layer l+4 waits for slot l % 4 to be free), and layer
+ * l's output is copied out on another context-owned stream while the next
+ * layers compute.  Asynchronous: when `stream` reaches the point after this
+ * call, every output is in host memory; the host inputs must not change
+ * before then.  Errors as ic_run_stack, plus IC_ERR_NOMEM when the four
+ * slots cannot be allocated. */
 int ic_run_stack_host(ic_ctx *ctx, const ic_pattern *pattern, const ic_layer_io *layers_host,
                       const ic_stack_dims *dims, int32_t *idx_cache, void *stream);
 
