@@ -83,10 +83,16 @@ __device__ __forceinline__ void find_bin(TopkShared& S, uint32_t krem, const uin
     }
     if (lane == 0) S.wsum[warp] = suf;  // the warp's total
     __syncthreads();
-    uint32_t higher = 0;  // keys in the warps above this one
+    // keys in the warps above this one: a suffix scan of the warp totals
+    // across lanes (lane w ends with the keys in warps >= w; lanes past the
+    // last warp hold 0)
+    uint32_t ws = lane < kTopkWarps ? S.wsum[lane] : 0u;
 #pragma unroll
-    for (int w = 0; w < kTopkWarps; ++w)
-        if (w > warp) higher += S.wsum[w];
+    for (int off = 1; off < kTopkWarps; off <<= 1) {
+        const uint32_t v = __shfl_down_sync(0xffffffffu, ws, off);
+        if (lane + off < kTopkWarps) ws += v;
+    }
+    const uint32_t higher = __shfl_sync(0xffffffffu, ws, warp + 1);
     const uint32_t incl = suf + higher;       // keys in bins >= my first bin
     const uint32_t above = incl - tot;        // keys in bins above mine
     if (above < krem && krem <= incl) {
@@ -162,7 +168,8 @@ __global__ void __launch_bounds__(kTopkThreads)
     // ---- B: resolve bits 20..10 and 9..0 within bin b1
     uint32_t prefix = b1 << 21, mask = 0xFFE00000u;
     const bool use_cand = in_bin <= static_cast<uint32_t>(kCandCap);
-    const int seg = ((n + kTopkWarps - 1) / kTopkWarps + 31) / 32 * 32;  // warp segments
+    // warp segments, whole 128-key blocks (a warp's float4 load of 4 keys per lane)
+    const int seg = ((n + kTopkWarps - 1) / kTopkWarps + 127) / 128 * 128;
     const int sb = warp * seg, se = min(n, sb + seg);
     const unsigned lt = (1u << lane) - 1u;
     uint32_t* cpos = dsm;
@@ -174,20 +181,50 @@ __global__ void __launch_bounds__(kTopkThreads)
         // whatever T is) become bitmap words straight from the ballot; the
         // keys of bin b1 go to the warp's own slice of the candidate list
         // with their positions (a count in registers: no shared atomics)
+        // Lane l takes keys base + 4l .. base + 4l + 3 (one float4; the row
+        // start is 16-byte aligned and its stride a multiple of 4 floats, so
+        // a load that starts before n stays inside the row's storage).
         uint32_t wc = 0;
-        for (int base = sb; base < se; base += 32) {
-            const int i = base + lane;
-            const bool in = i < se;
-            const uint32_t u = in ? key_at(i) : 0u;
-            const unsigned wa = __ballot_sync(0xffffffffu, in && (u >> 21) > b1);
-            const unsigned wb = __ballot_sync(0xffffffffu, in && (u >> 21) == b1);
-            if (lane == 0) bits[base >> 5] = wa;
-            const uint32_t j = wc + __popc(wb & lt);
-            if (((wb >> lane) & 1u) && j < static_cast<uint32_t>(kSlice)) {
-                S.cand[warp * kSlice + j] = u;
-                cpos[warp * kSlice + j] = static_cast<uint32_t>(i);
+        for (int base = sb; base < se; base += 128) {
+            const int i0 = base + 4 * lane;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (i0 < se) v = __ldg(reinterpret_cast<const float4*>(row + i0));
+            const float x[4] = {v.x, v.y, v.z, v.w};
+            uint32_t u[4], nib = 0;
+            bool c[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const bool in = i0 + j < se;
+                u[j] = order_key(x[j]);
+                const uint32_t bin = u[j] >> 21;
+                nib |= static_cast<uint32_t>(in && bin > b1) << j;
+                c[j] = in && bin == b1;
             }
-            wc += __popc(wb);
+            // bitmap word m of the block holds lanes 8m .. 8m+7's nibbles
+            uint32_t word = nib << (4 * (lane & 7));
+            word |= __shfl_xor_sync(0xffffffffu, word, 1);
+            word |= __shfl_xor_sync(0xffffffffu, word, 2);
+            word |= __shfl_xor_sync(0xffffffffu, word, 4);
+            if ((lane & 7) == 0 && base + 4 * lane < se) bits[(base >> 5) + (lane >> 3)] = word;
+            // keys of bin b1: this lane's slots follow the lower lanes' (all j)
+            unsigned bc[4];
+            uint32_t j0 = wc;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                bc[j] = __ballot_sync(0xffffffffu, c[j]);
+                j0 += __popc(bc[j] & lt);
+                wc += __popc(bc[j]);
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (c[j]) {
+                    if (j0 < static_cast<uint32_t>(kSlice)) {
+                        S.cand[warp * kSlice + j0] = u[j];
+                        cpos[warp * kSlice + j0] = static_cast<uint32_t>(i0 + j);
+                    }
+                    ++j0;
+                }
+            }
         }
         if (lane == 0) S.wcand[warp] = wc;
         __syncthreads();
@@ -252,10 +289,16 @@ __global__ void __launch_bounds__(kTopkThreads)
         }
         if (lane == 31) S.wsum[warp] = incl;
         __syncthreads();
-        uint32_t at = incl - cnt;
+        // positions in the warps before this one: a prefix scan of the warp
+        // totals across lanes (lane w ends with the positions in warps <= w)
+        uint32_t ws = lane < kTopkWarps ? S.wsum[lane] : 0u;
 #pragma unroll
-        for (int w = 0; w < kTopkWarps; ++w)
-            if (w < warp) at += S.wsum[w];
+        for (int off = 1; off < kTopkWarps; off <<= 1) {
+            const uint32_t v = __shfl_up_sync(0xffffffffu, ws, off);
+            if (lane >= off) ws += v;
+        }
+        const uint32_t before = __shfl_sync(0xffffffffu, ws, warp > 0 ? warp - 1 : 0);
+        uint32_t at = incl - cnt + (warp > 0 ? before : 0u);
         for (int w = w0; w < w1; ++w)
             for (uint32_t x = bits[w]; x; x &= x - 1u) o[at++] = (w << 5) + (__ffs(x) - 1);
         return;  // exactly k positions were written
