@@ -543,8 +543,8 @@ extern "C" int ic_index_overlap(ic_ctx* ctx, const int32_t* idx_a, const int32_t
 namespace ic {
 // One layer of the stack ([IC] Figure 2): an F layer runs the indexer and
 // top-k into idx_cache, an S layer reuses it; then the layer's attention.
-int run_stack_layer(ic_ctx* ctx, char c, const ic_layer_io& io, const ic_stack_dims* dims,
-                    int32_t* idx_cache, void* stream) {
+int run_stack_layer(ic_ctx* ctx, char c, const ic_layer_io& io, const ic_layer_io* next,
+                    const ic_stack_dims* dims, int32_t* idx_cache, void* stream) {
     const bool prefill = dims->mode == IC_PREFILL;
     const int rows = prefill ? dims->L : dims->B;
     const int k = dims->k;
@@ -562,7 +562,10 @@ int run_stack_layer(ic_ctx* ctx, char c, const ic_layer_io& io, const ic_stack_d
     const bool pdl = !prefill && static_cast<long long>(dims->B) * 8 <= ctx->num_sms;
     struct PdlScope {
         ic_ctx* c;
-        ~PdlScope() { c->pdl = 0; }
+        ~PdlScope() {
+            c->pdl = 0;
+            c->pf_K = c->pf_V = nullptr;
+        }
     } pdl_scope{ctx};
     int rc;
     if (c == 'F') {
@@ -588,6 +591,15 @@ int run_stack_layer(ic_ctx* ctx, char c, const ic_layer_io& io, const ic_stack_d
     if (prefill)
         return ic_sparse_attn(ctx, io.Q, io.K, io.V, idx, rows, dims->Hq, dims->d, k, 0, 0, dims->L,
                               dims->scale, io.out, stream);
+    // Decode: the next S layer gathers its own K/V at these same slots.  Its
+    // cached rows are already in HBM, so this layer's CTAs warm L2 with them
+    // after their own gather, overlapping that traffic with this layer's merge
+    // and the launch in between.  (Small batches already do this in the S
+    // layer itself, before its programmatic wait.)
+    if (next && !pdl) {
+        ctx->pf_K = next->K;
+        ctx->pf_V = next->V;
+    }
     return ic_sparse_attn(ctx, io.Q, io.K, io.V, idx, rows, dims->Hq, dims->d, k, 1,
                           static_cast<int64_t>(dims->S_max) * dims->d, dims->S_max, dims->scale,
                           io.out, stream);
@@ -611,7 +623,8 @@ extern "C" int ic_run_stack(ic_ctx* ctx, const ic_pattern* pattern, const ic_lay
     cudaSetDevice(ctx->device);
     const int N = static_cast<int>(pattern->c.size());
     for (int l = 0; l < N; ++l) {
-        rc = run_stack_layer(ctx, pattern->c[l], layers[l], dims, idx_cache, stream);
+        const ic_layer_io* next = l + 1 < N && pattern->c[l + 1] == 'S' ? &layers[l + 1] : nullptr;
+        rc = run_stack_layer(ctx, pattern->c[l], layers[l], next, dims, idx_cache, stream);
         if (rc) return rc;
     }
     return IC_OK;

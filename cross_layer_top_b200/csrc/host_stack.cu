@@ -161,7 +161,7 @@ extern "C" int ic_run_stack_host(ic_ctx* ctx, const ic_pattern* pattern,
         d.V = dV;
         d.out = dout;
         d.idx_snapshot = h.idx_snapshot;  // device memory, as in ic_run_stack
-        rc = run_stack_layer(ctx, pattern->c[l], d, dims, idx_cache, stream);
+        rc = run_stack_layer(ctx, pattern->c[l], d, nullptr, dims, idx_cache, stream);
         if (rc) return rc;
         e = cudaEventRecord(hs.computed[sl], s);
         if (e == cudaSuccess) e = cudaStreamWaitEvent(hs.out, hs.computed[sl], 0);

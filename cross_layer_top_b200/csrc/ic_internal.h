@@ -36,6 +36,11 @@ struct ic_ctx {
     // of an S layer) it may also read the index cache and warm L2 with the
     // K/V rows it will gather before that wait.
     int pdl = 0;
+    // set by the decode stack for one attention launch: the next layer's K/V
+    // (an S layer, which reuses this layer's index slots), whose rows at those
+    // slots the attention kernel prefetches into L2 once its own gather is done
+    const void* pf_K = nullptr;
+    const void* pf_V = nullptr;
     // ic_run_stack_host: kHostSlots device staging slots, a copy-in and a
     // copy-out stream, and per-slot events (created on first use)
     static constexpr int kHostSlots = 4;
@@ -99,8 +104,10 @@ int make_tmap_u8_2d(ic_ctx* ctx, CUtensorMap* map, const void* base, uint64_t ro
 
 // ----------------------------------------------------------------- launchers
 // One layer of the F/S stack (shared by ic_run_stack and ic_run_stack_host).
-int run_stack_layer(ic_ctx* ctx, char c, const ic_layer_io& io, const ic_stack_dims* dims,
-                    int32_t* idx_cache, void* stream);
+// `next` is the following layer when it is an S layer whose K/V are in device
+// memory (it reuses this layer's index slots), else null.
+int run_stack_layer(ic_ctx* ctx, char c, const ic_layer_io& io, const ic_layer_io* next,
+                    const ic_stack_dims* dims, int32_t* idx_cache, void* stream);
 int check_stack_args(ic_ctx* ctx, const ic_pattern* pattern, const void* layers,
                      const ic_stack_dims* dims, const int32_t* idx_cache);
 

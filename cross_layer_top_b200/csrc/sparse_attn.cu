@@ -192,6 +192,7 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS,
                   const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ idx, int Hq,
                   int k, int rows_per_seq, long long kv_seq_stride, int kv_len, float scale_log2,
                   int nsplit, int kps, int pf_ahead, int vec_idx, int pdl,
+                  const __nv_bfloat16* __restrict__ nK, const __nv_bfloat16* __restrict__ nV,
                   __nv_bfloat16* __restrict__ out,
                   int* __restrict__ err) {
     using S = AttnShape<D>;
@@ -272,22 +273,27 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS,
     if (bad) atomicCAS(err, 0, kDevBadIndex);
     last = __reduce_max_sync(0xffffffffu, last);
     if (lane == 0 && last >= 0) atomicMax(s_last, last);
+    // warm L2 with the K and V rows of a layer (base pointers kb, vb of this
+    // row's sequence) at this split's first n staged slots
+    auto prefetch_rows = [&](const __nv_bfloat16* kb, const __nv_bfloat16* vb, int n) {
+        constexpr int LPR = (D * 2 + 127) / 128;  // 128-byte lines per row
+        for (int t = tid; t < n * 2 * LPR; t += S::THREADS) {
+            const int slot = t / (2 * LPR), part = t - slot * (2 * LPR);
+            const int v = sIdx[slot];
+            if (v >= 0) {
+                const char* row = reinterpret_cast<const char*>(part < LPR ? kb : vb) +
+                                  static_cast<long long>(v) * D * 2 + (part % LPR) * 128;
+                asm volatile("prefetch.global.L2 [%0];" ::"l"(row));
+            }
+        }
+    };
     if (pdl == 2) {
         // An S layer's index slots and its cached K/V rows are not written by
         // the previous kernel: warm L2 with the rows this split will gather,
         // then wait for that kernel before reading the query heads (and, in
         // the main loop, the rows themselves, the newest one included).
         __syncthreads();  // every slot is staged
-        constexpr int LPR = (D * 2 + 127) / 128;  // 128-byte lines per row
-        for (int t = tid; t < nk * 2 * LPR; t += S::THREADS) {
-            const int slot = t / (2 * LPR), part = t - slot * (2 * LPR);
-            const int v = sIdx[slot];
-            if (v >= 0) {
-                const char* row = reinterpret_cast<const char*>(part < LPR ? Kb : Vb) +
-                                  static_cast<long long>(v) * D * 2 + (part % LPR) * 128;
-                asm volatile("prefetch.global.L2 [%0];" ::"l"(row));
-            }
-        }
+        prefetch_rows(Kb, Vb, nk);
         griddep_wait();
         stage_q();
     }
@@ -383,6 +389,9 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS,
         issue_with(j + S::STAGES, nsv);  // refill it
     }
     cp_async_wait<0>();
+    // the next layer (an S layer) gathers its own K/V at these same slots:
+    // its rows are fetched into L2 while this row merges
+    if (nK != nullptr) prefetch_rows(nK + seq * kv_seq_stride, nV + seq * kv_seq_stride, nk_eff);
     l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
     l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
     l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
@@ -569,6 +578,9 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
     const auto* Kp = static_cast<const __nv_bfloat16*>(K);
     const auto* Vp = static_cast<const __nv_bfloat16*>(V);
     auto* op = static_cast<__nv_bfloat16*>(out);
+    // the next layer's K/V, to prefetch at these slots (both or neither)
+    const auto* pfK = ctx->pf_V ? static_cast<const __nv_bfloat16*>(ctx->pf_K) : nullptr;
+    const auto* pfV = pfK ? static_cast<const __nv_bfloat16*>(ctx->pf_V) : nullptr;
     const long long kvs = static_cast<long long>(kv_seq_stride);
     if (nsplit == 1) {
         cudaLaunchConfig_t cfg = {};
@@ -583,7 +595,7 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
         cfg.numAttrs = na;
         cudaLaunchKernelEx(&cfg, k_sparse_attn<D, false>, Qp, Kp, Vp, idx, Hq, k, rows_per_seq, kvs,
                            kv_len, scale_log2, 1, kps, S::CTAS_PER_SM * ctx->num_sms, vec_idx,
-                           ctx->pdl, op, ctx->dev_err);
+                           ctx->pdl, pfK, pfV, op, ctx->dev_err);
     } else {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(rows, nsplit, 1);
@@ -600,7 +612,8 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
         cfg.attrs = attr;
         cfg.numAttrs = na;
         cudaLaunchKernelEx(&cfg, k_sparse_attn<D, true>, Qp, Kp, Vp, idx, Hq, k, rows_per_seq, kvs, kv_len,
-                           scale_log2, nsplit, kps, 0, vec_idx, ctx->pdl, op, ctx->dev_err);
+                           scale_log2, nsplit, kps, 0, vec_idx, ctx->pdl, pfK, pfV, op,
+                           ctx->dev_err);
     }
     cudaError_t e = ls.done();
     if (e != cudaSuccess) return cuda_fail(ctx, e, "sparse_attn launch");
