@@ -20,7 +20,10 @@
 // merge through shared memory; one split writes bf16 output; with several
 // splits (decode) the row's CTAs form a thread-block cluster and merge
 // through distributed shared memory (each CTA owns a share of the heads and
-// receives the other CTAs' partials of them).
+// receives the other CTAs' partials of them in a receive area of its own,
+// which leaves room for two such CTAs per SM).  A decode stack may pass the
+// next layer's K/V (an S layer gathers at the same slots): its rows are then
+// prefetched into L2 once this CTA's own gather is done.
 #include "ic_device.cuh"
 #include "ic_internal.h"
 

@@ -263,3 +263,41 @@ def test_decode_stack_programmatic_launch_matches(ic, ctx):
     ref_out = oracle.sparse_attn(f32(lay["Q"]), f32(lay["K"]), f32(lay["V"]), s_idx, rows_per_seq=1)
     got = lay["out"].float().cpu().numpy().astype(np.float64)
     assert np.all(np.abs(got - ref_out) <= 2e-2 + 1e-2 * np.abs(ref_out))
+
+
+def test_decode_stack_cross_layer_prefetch_matches(ic, ctx):
+    """A decode stack of a batch too large for programmatic launches
+    (B * 8 > SMs): an attention layer followed by an S layer warms L2 with
+    that layer's K/V rows at the shared index slots.  A prefetch changes no
+    value, so every layer's output must equal a standalone ic_sparse_attn call
+    on the same indices bit for bit, and an S layer must match the oracle."""
+    cfg = synth.DecodeConfig("wide_decode", 24, 3000, "FSSSFS", 64, 128, 512, 16, 128, 37)
+    B, S, k = cfg.B, cfg.S, cfg.k
+    assert B * 8 > 148  # no programmatic launches: the cross-layer prefetch runs
+    layers = []
+    for l in range(cfg.n_layers):
+        lay = synth.decode_layer(cfg, l, "cuda")
+        lay["out"] = torch.empty((B, cfg.Hq, cfg.d), dtype=torch.bfloat16, device="cuda")
+        layers.append(lay)
+    seq_len = layers[0]["seq_len"]
+    pat = ic.ic_create_pattern(cfg.pattern)
+    dims = ic.stack_dims(ic.IC_DECODE, cfg.H_I, cfg.d_I, k, cfg.Hq, cfg.d, B=B, S_max=S,
+                         seq_len=seq_len)
+    cache = torch.empty((B, k), dtype=torch.int32, device="cuda")
+    snaps = [torch.empty((B, k), dtype=torch.int32, device="cuda") for _ in range(cfg.n_layers)]
+    for lay, sn in zip(layers, snaps):
+        lay["idx_snapshot"] = sn
+    ic.ic_run_stack(ctx, pat, layers, dims, cache)
+    ctx.sync_status()
+    for l in range(cfg.n_layers):
+        lay = layers[l]
+        alone = torch.empty_like(lay["out"])
+        ic.ic_sparse_attn(ctx, lay["Q"], lay["K"], lay["V"], snaps[l], alone, rows_per_seq=1,
+                          kv_seq_stride=S * cfg.d, kv_len=S)
+        ctx.sync_status()
+        assert torch.equal(lay["out"], alone), l
+    lay = layers[3]  # an S layer after an S layer: both had their rows prefetched
+    ref_out = oracle.sparse_attn(f32(lay["Q"]), f32(lay["K"]), f32(lay["V"]),
+                                 snaps[3].cpu().numpy(), rows_per_seq=1)
+    got = lay["out"].float().cpu().numpy().astype(np.float64)
+    assert np.all(np.abs(got - ref_out) <= 2e-2 + 1e-2 * np.abs(ref_out))
