@@ -31,9 +31,9 @@
  *  - Positions are 0-based; causal means s <= t (the query sees itself).
  *  - Index rows hold min(k, n) selected positions in ascending order
  *    followed by -1 padding; ties in score go to the lower position.
- *  - A context (ic_ctx) owns scratch memory (score rows, split-attention
- *    partials) and the device error flag.  It is not thread-safe: use one
- *    context per host thread / stream.
+ *  - A context (ic_ctx) owns scratch memory (fp32 score rows; the staging
+ *    slots of ic_run_stack_host), timing events and the device error flag.
+ *    It is not thread-safe: use one context per host thread / stream.
  */
 #ifndef INDEXCACHE_H
 #define INDEXCACHE_H
