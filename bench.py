@@ -318,8 +318,8 @@ def run_ours(args, rank, world, local_rank):
 
 
 # DRAM traffic per launch (dram__bytes_read.sum + dram__bytes_write.sum) of
-# the prefill kernels, from one ncu capture of the current kernel each
-# (profiles/sparse_attn_prefill_L16384.md, profiles/indexer_prefill_L16384.md);
+# the prefill kernels, from one ncu capture of the current kernel each (the
+# summaries under profiles/ for the L=16384 prefill attention and indexer);
 # None once a kernel changes until it is captured again.
 ATTN_PREFILL_DRAM_BYTES = 209.84e6 + 51.81e6
 INDEX_SCORE_PREFILL_DRAM_BYTES = 248.2e6 + 487.7e6

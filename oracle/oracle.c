@@ -21,7 +21,7 @@
  *          overwritten at the next F); §3 sparse attention
  *          o_t = sum_{s in T_t} softmax(Q_t.K_s / sqrt(d)) V_s.
  *
- * Readings where the pages are silent (each is listed in the design doc):
+ * Readings taken where the pages are silent:
  *   causal range s <= t; ties in top-k go to the lower index; the selected
  *   set is returned in ascending index order, padded with -1 when the row
  *   has fewer than k candidates; -1 entries are skipped by attention.
