@@ -462,7 +462,10 @@ __global__ void __launch_bounds__(kTopkThreads)
     // each thread sums 4 consecutive bins (2048 = 4 x 512) over the cluster's
     // CTAs with one 16-byte remote load per CTA, all issued before any is used
     static_assert(2048 == 4 * kTopkThreads, "four bins per thread");
-    auto cluster_hist = [&]() {
+    // rewrite_next: the caller rewrites its histogram right after (another
+    // radix pass over the row), so a second barrier keeps every CTA's reads
+    // of it ahead of that; otherwise a later cluster barrier does
+    auto cluster_hist = [&](bool rewrite_next) {
         cluster_sync_all();  // every segment histogram is complete
         uint4 hv[kClusterCtas];
 #pragma unroll
@@ -476,10 +479,10 @@ __global__ void __launch_bounds__(kTopkThreads)
             t.w += hv[q].w;
         }
         *reinterpret_cast<uint4*>(&CS.hist_all[4 * tid]) = t;
-        cluster_sync_all();  // nobody rewrites a histogram another CTA still reads
+        if (rewrite_next) cluster_sync_all();  // nobody rewrites a histogram another CTA still reads
     };
     for (int i = tid; i < m; i += kTopkThreads) atomicAdd(&S.hist[bin_of(srow[i])], 1u);
-    cluster_hist();
+    cluster_hist(false);
     find_bin<2048>(S, static_cast<uint32_t>(k), CS.hist_all);
     const uint32_t b1 = S.bin;
     uint32_t krem = static_cast<uint32_t>(k) - S.above;
@@ -488,7 +491,11 @@ __global__ void __launch_bounds__(kTopkThreads)
 
     // ---- B: candidates of bin b1 from every segment, or (massive ties)
     // cluster-wide radix passes over the bin's keys
-    const bool use_cand = in_bin <= static_cast<uint32_t>(kCandCap);
+    const bool use_cand = in_bin <= static_cast<uint32_t>(kCandCap);  // the same in every CTA
+    // The radix passes rewrite S.hist.  With candidates, the barrier after
+    // they are collected keeps every CTA's reads of the histograms above
+    // ahead of that; without, this one does.
+    if (!use_cand) cluster_sync_all();
     int ncand = 0;
     if (use_cand) {
         for (int i = tid; i < m; i += kTopkThreads) {
@@ -520,7 +527,9 @@ __global__ void __launch_bounds__(kTopkThreads)
                     if (i4 + e < nq[q]) cand_all[off[q] + i4 + e] = c4[e];
             }
         }
-        cluster_sync_all();
+        // No CTA rewrites its S.ncand or S.cand after this, so other CTAs may
+        // still be reading them: only this CTA's merged list must be complete.
+        __syncthreads();
     }
     uint32_t prefix = 0, mask = 0;
 #pragma unroll 1
@@ -541,7 +550,7 @@ __global__ void __launch_bounds__(kTopkThreads)
                 if ((u & mask) == prefix && bin_of(u) == b1)
                     atomicAdd(&S.hist[(u >> shift) & dmask], 1u);
             }
-            cluster_hist();
+            cluster_hist(true);
         }
         const uint32_t* h = use_cand ? S.hist : CS.hist_all;
         if (pass < 2)
