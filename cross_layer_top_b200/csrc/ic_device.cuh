@@ -265,6 +265,9 @@ __device__ __forceinline__ void dsmem_st_f4(uint32_t addr, float4 v) {
                  "f"(v.z), "f"(v.w)
                  : "memory");
 }
+__device__ __forceinline__ void dsmem_st_u32(uint32_t addr, uint32_t v) {
+    asm volatile("st.shared::cluster.u32 [%0], %1;" ::"r"(addr), "r"(v) : "memory");
+}
 __device__ __forceinline__ void dsmem_st_f32(uint32_t addr, float v) {
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }

@@ -364,7 +364,10 @@ constexpr int kClusterCtas = 8;
 struct alignas(16) TopkClusterShared {
     TopkShared S;
     alignas(16) uint32_t hist_all[2048];
-    uint32_t seg_kmin, seg_kmax, seg_cg, seg_ce;
+    // pushed by each CTA q into the others' copies (slot q): its segment's
+    // key range, and (for the later segments) its counts of keys > T and == T
+    uint32_t rng_min[kClusterCtas], rng_max[kClusterCtas];
+    uint32_t cnt_g[kClusterCtas], cnt_e[kClusterCtas];
 };
 static_assert(offsetof(TopkShared, hist) % 16 == 0 && offsetof(TopkShared, cand) % 16 == 0,
               "16-byte loads of the histogram and candidates");
@@ -392,6 +395,9 @@ __global__ void __launch_bounds__(kTopkThreads)
             for (int i = tid; i < k; i += kTopkThreads) o[i] = i < n ? i : -1;
         return;
     }
+    // every CTA arrives on the cluster barrier now and waits on it before its
+    // first remote store, by when the whole cluster is known to be running
+    cluster_arrive_relaxed();
     const int seg = ((n + kClusterCtas - 1) / kClusterCtas + 3) / 4 * 4;
     const int s0 = min(n, static_cast<int>(rank) * seg), s1 = min(n, s0 + seg);
     const int m = s1 - s0;  // this CTA's segment length
@@ -426,29 +432,24 @@ __global__ void __launch_bounds__(kTopkThreads)
     for (int i = tid; i < 2048; i += kTopkThreads) S.hist[i] = 0;
     if (tid == 0) S.ncand = 0;
     __syncthreads();
-    if (tid == 0) {
+    cluster_wait_acquire();  // every CTA of the cluster is running
+    // thread q stores this segment's range into CTA q's slot `rank`
+    if (tid < kClusterCtas) {
         uint32_t a = 0xFFFFFFFFu, b = 0u;
         for (int w = 0; w < kTopkWarps; ++w) {
             a = min(a, S.wcnt[0][w]);
             b = max(b, S.wcnt[1][w]);
         }
-        CS.seg_kmin = a;
-        CS.seg_kmax = b;
+        dsmem_st_u32(dsmem_addr(&CS.rng_min[rank], tid), a);
+        dsmem_st_u32(dsmem_addr(&CS.rng_max[rank], tid), b);
     }
-    cluster_sync_all();
-    // every CTA's range: all remote loads issued before any is used
-    uint32_t qmin[kClusterCtas], qmax[kClusterCtas];
-#pragma unroll
-    for (uint32_t q = 0; q < kClusterCtas; ++q) {
-        qmin[q] = dsmem_ld(dsmem_addr(&CS.seg_kmin, q));
-        qmax[q] = dsmem_ld(dsmem_addr(&CS.seg_kmax, q));
-    }
+    cluster_sync_all();  // every segment's range is in every CTA
     kmin = 0xFFFFFFFFu;
     kmax = 0u;
 #pragma unroll
-    for (uint32_t q = 0; q < kClusterCtas; ++q) {
-        kmin = min(kmin, qmin[q]);
-        kmax = max(kmax, qmax[q]);
+    for (int q = 0; q < kClusterCtas; ++q) {
+        kmin = min(kmin, CS.rng_min[q]);
+        kmax = max(kmax, CS.rng_max[q]);
     }
     const float xmin = key_float(kmin), xmax = key_float(kmax);
     const float span = xmax - xmin;
@@ -580,20 +581,25 @@ __global__ void __launch_bounds__(kTopkThreads)
         S.wcnt[1][warp] = ce;
     }
     __syncthreads();
-    if (tid == 0) {
+    // thread q > rank stores this segment's counts into CTA q's slot `rank`
+    // (only the later segments offset by them)
+    if (tid < kClusterCtas && tid > static_cast<int>(rank)) {
         uint32_t a = 0, b = 0;
         for (int w = 0; w < kTopkWarps; ++w) {
             a += S.wcnt[0][w];
             b += S.wcnt[1][w];
         }
-        CS.seg_cg = a;
-        CS.seg_ce = b;
+        dsmem_st_u32(dsmem_addr(&CS.cnt_g[rank], tid), a);
+        dsmem_st_u32(dsmem_addr(&CS.cnt_e[rank], tid), b);
     }
+    // The last cluster barrier: every count is where it is needed, and every
+    // remote load of this CTA's histograms and candidates came before it, so
+    // from here each CTA touches only its own shared memory and may exit.
     cluster_sync_all();
     uint32_t G = 0, E = 0;
     for (uint32_t q = 0; q < rank; ++q) {
-        G += dsmem_ld(dsmem_addr(&CS.seg_cg, q));
-        E += dsmem_ld(dsmem_addr(&CS.seg_ce, q));
+        G += CS.cnt_g[q];
+        E += CS.cnt_e[q];
     }
 #pragma unroll
     for (int w = 0; w < kTopkWarps; ++w)
@@ -618,7 +624,6 @@ __global__ void __launch_bounds__(kTopkThreads)
         G += __popc(bg);
         E += __popc(be);
     }
-    cluster_sync_all();  // no CTA leaves while another may still read its shared memory
 }
 
 static int launch_topk_cluster(ic_ctx* ctx, const float* scores, int64_t ld, int rows, int k,
