@@ -395,18 +395,21 @@ def test_argument_errors(ic, ctx):
     ctx.sync_status()
 
 
+@pytest.mark.parametrize("B", [5, 24])
 @pytest.mark.parametrize("integer", [True, False])
-def test_topk_cluster_rows(ic, ctx, integer):
+def test_topk_cluster_rows(ic, ctx, integer, B):
     """Few long rows with explicit lengths take the cluster kernel (8 CTAs
     per row sharing histograms and candidates through distributed shared
-    memory); integer scores force the massive-tie fallback."""
-    gen = torch.Generator().manual_seed(11 + integer)
-    B, ld = 5, 100032
+    memory), for a small and a larger batch; integer scores force the
+    massive-tie fallback."""
+    gen = torch.Generator().manual_seed(11 + integer + 2 * B)
+    ld = 100032
     if integer:
         sc = torch.randint(-4, 5, (B, ld), generator=gen).float() * 0.5
     else:
         sc = torch.randn((B, ld), generator=gen)
-    lens = torch.tensor([100000, 16385, 2049, 99999, 77777], dtype=torch.int32)
+    lens = [100000, 16385, 2049, 99999, 77777]
+    lens = torch.tensor((lens * ((B + 4) // 5))[:B], dtype=torch.int32)
     idx = torch.empty((B, 2048), dtype=torch.int32, device="cuda")
     ic.ic_topk(ctx, sc.cuda(), 2048, idx, row_len=lens.cuda(), ld=ld)
     ctx.sync_status()
