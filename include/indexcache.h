@@ -283,10 +283,9 @@ typedef struct ic_stack_dims {
  * layer's attention reads the index cache and prefetches (into L2 only) the
  * K/V rows at those slots first.  Larger decode batches launch normally;
  * there an attention layer followed by an S layer prefetches (into L2 only)
- * that layer's K/V rows at the shared slots after its own gather, so the
- * caller must not change a later layer's K/V while the stack runs.  A
- * caller's own kernel before the stack is always complete before the stack
- * reads anything. */
+ * that layer's K/V rows at the shared slots after its own gather (a
+ * prefetch changes no result).  A caller's own kernel before the stack is
+ * always complete before the stack reads anything. */
 int ic_run_stack(ic_ctx *ctx, const ic_pattern *pattern, const ic_layer_io *layers,
                  const ic_stack_dims *dims, int32_t *idx_cache, void *stream);
 
