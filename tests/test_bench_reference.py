@@ -40,3 +40,14 @@ def test_reference_arm_other_ranks_silent():
     p = _run({"RANK": "1", "WORLD_SIZE": "2", "LOCAL_RANK": "1"})
     assert p.returncode == 0, p.stderr[-2000:]
     assert not [l for l in p.stdout.splitlines() if l.startswith("{")]
+
+
+def test_scored_pairs_counts_causal_rows_past_k():
+    """The headline unit: an F layer scores the causal pairs (t, s <= t) of
+    rows t >= k (rows t < k keep 0..t without a score), counted here by
+    brute force."""
+    sys.path.insert(0, ROOT)
+    import bench
+    for L, k, n_f in [(512, 64, 1), (100, 7, 3), (64, 64, 2), (50, 64, 1), (16384, 2048, 2)]:
+        brute = n_f * sum(t + 1 for t in range(k, L))
+        assert bench.scored_pairs(L, k, n_f) == brute
