@@ -62,6 +62,9 @@ def lib():
         L.oracle_sparse_attn_rows.argtypes = [_f32p, _f32p, _f32p, _i32p, _i32p, ctypes.c_int,
                                               ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                               ctypes.c_int, ctypes.c_int64, ctypes.c_double, _f64p]
+        L.oracle_attn_weight_spread_rows.argtypes = [
+            _f32p, _f32p, _f32p, _i32p, _i32p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+            ctypes.c_int, ctypes.c_int, ctypes.c_int64, ctypes.c_double, _f64p]
         L.oracle_overlap_row.argtypes = [_i32p, _i32p, ctypes.c_int]
         L.oracle_overlap_row.restype = ctypes.c_double
         _lib = L
@@ -237,6 +240,37 @@ def sparse_attn(Q, K, V, idx, rows=None, scale=None, rows_per_seq=0, q_is_rows=F
     lib().oracle_sparse_attn_rows(_p(Q, _f32p), _p(K, _f32p), _p(V, _f32p), _p(idx, _i32p),
                                   _p(rows, _i32p), len(rows), k, Hq, d, rows_per_seq,
                                   kv_stride, float(scale), _p(out, _f64p))
+    return out
+
+
+def attn_weight_spread(Q, K, V, idx, rows=None, scale=None, rows_per_seq=0, q_is_rows=False):
+    """sqrt(sum_s p_s^2 V[s]^2) per output element, with the softmax weights
+    p_s of ``sparse_attn`` (same arguments): how far o moves when every
+    weight carries a small independent relative error (the tolerance of the
+    attention tests, not a step of the method).  float64 [nrows, Hq, d]."""
+    if q_is_rows:
+        Q = _c(Q, np.float32)
+        out = np.empty((Q.shape[0],) + Q.shape[1:], dtype=np.float64)
+        seqs = np.zeros(len(rows), np.int64) if rows_per_seq <= 0 else np.asarray(rows) // rows_per_seq
+        for r in range(Q.shape[0]):
+            Kr = K if K.ndim == 2 else K[seqs[r]]
+            Vr = V if V.ndim == 2 else V[seqs[r]]
+            out[r] = attn_weight_spread(Q[r:r + 1], Kr, Vr, np.asarray(idx)[r:r + 1], scale=scale)[0]
+        return out
+    Q = _c(Q, np.float32)
+    K = _c(K, np.float32)
+    V = _c(V, np.float32)
+    idx = _c(idx, np.int32)
+    R, Hq, d = Q.shape
+    rows = np.arange(R, dtype=np.int32) if rows is None else _c(rows, np.int32)
+    k = idx.shape[1]
+    if scale is None:
+        scale = 1.0 / np.sqrt(d)
+    kv_stride = K.shape[-2] * d if K.ndim == 3 else 0
+    out = np.empty((len(rows), Hq, d), dtype=np.float64)
+    lib().oracle_attn_weight_spread_rows(_p(Q, _f32p), _p(K, _f32p), _p(V, _f32p), _p(idx, _i32p),
+                                         _p(rows, _i32p), len(rows), k, Hq, d, rows_per_seq,
+                                         kv_stride, float(scale), _p(out, _f64p))
     return out
 
 

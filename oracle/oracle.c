@@ -347,6 +347,62 @@ void oracle_sparse_attn_rows(const float *Q, const float *K, const float *V, con
     }
 }
 
+/* The spread of one attention output under small relative errors in the
+ * softmax weights, for the tolerance of the attention tests (not a step of
+ * the method).  With the normalised weights p_s of [RN] §3 (the same logits
+ * and skipping rule as oracle_sparse_attn_row),
+ *   spread[h,e] = sqrt( sum_{s in T} p_s^2 V[s,e]^2 ).
+ * If every weight carries an independent relative error of standard
+ * deviation u, o[h,e] moves by a random amount of standard deviation
+ * u * spread[h,e].  Same argument layout as oracle_sparse_attn_rows. */
+void oracle_attn_weight_spread_rows(const float *Q, const float *K, const float *V,
+                                    const int32_t *idx, const int32_t *rows, int nrows, int k,
+                                    int Hq, int d, int rows_per_seq, int64_t kv_stride,
+                                    double scale, double *out)
+{
+    int r;
+#pragma omp parallel for schedule(dynamic, 4)
+    for (r = 0; r < nrows; ++r) {
+        int t = rows[r];
+        int64_t seq = rows_per_seq > 0 ? (int64_t)(t / rows_per_seq) : 0;
+        const float *Qt = Q + (size_t)t * Hq * d;
+        const float *Kb = K + seq * kv_stride;
+        const float *Vb = V + seq * kv_stride;
+        const int32_t *ix = idx + (size_t)r * k;
+        double *z = (double *)malloc(sizeof(double) * (size_t)(k > 0 ? k : 1));
+        for (int h = 0; h < Hq; ++h) {
+            double zmax = -INFINITY;
+            for (int j = 0; j < k; ++j) {
+                if (ix[j] < 0)
+                    continue;
+                double dot = 0.0;
+                for (int e = 0; e < d; ++e)
+                    dot += (double)Qt[(size_t)h * d + e] * (double)Kb[(size_t)ix[j] * d + e];
+                z[j] = dot * scale;
+                if (z[j] > zmax)
+                    zmax = z[j];
+            }
+            double denom = 0.0;
+            for (int j = 0; j < k; ++j)
+                if (ix[j] >= 0)
+                    denom += exp(z[j] - zmax);
+            double *oh = out + ((size_t)r * Hq + h) * d;
+            for (int e = 0; e < d; ++e) {
+                double acc = 0.0;
+                for (int j = 0; j < k; ++j) {
+                    if (ix[j] < 0)
+                        continue;
+                    double p = exp(z[j] - zmax) / denom;
+                    double pv = p * (double)Vb[(size_t)ix[j] * d + e];
+                    acc += pv * pv;
+                }
+                oh[e] = sqrt(acc);
+            }
+        }
+        free(z);
+    }
+}
+
 /* Cross-layer overlap |T_i ∩ T_j| / k of two index rows ([IC] Appendix A);
  * -1 padding never counts. Both rows must be free of repeated indices. */
 double oracle_overlap_row(const int32_t *a, const int32_t *b, int k)

@@ -160,6 +160,44 @@ def test_scores_orthogonal_and_negative_weights():
     assert oracle.topk_row(row, len(zeros)).tolist() == zeros
 
 
+def test_scores_at_equals_scores_of_full_tensors():
+    """index_scores_at (sampled rows given compactly) against index_scores on
+    the whole tensors, bit for bit: Gaussian and integer inputs, unsorted
+    and repeated positions.  A wrong row stride or pos[r] mixed up with r
+    fails here."""
+    rng = np.random.default_rng(17)
+    L, H, d = 90, 3, 5
+    for integer in (False, True):
+        if integer:
+            q = rng.integers(-3, 4, (L, H, d)).astype(np.float32)
+            k = rng.integers(-3, 4, (L, d)).astype(np.float32)
+            w = rng.choice([-1.0, -0.5, 0.5, 1.0], (L, H)).astype(np.float32)
+        else:
+            q = rng.standard_normal((L, H, d)).astype(np.float32)
+            k = rng.standard_normal((L, d)).astype(np.float32)
+            w = rng.standard_normal((L, H)).astype(np.float32)
+        pos = np.array([57, 3, 89, 0, 57, 12, 44, 3], np.int32)  # unsorted, repeated
+        full = oracle.index_scores(q, k, w, rows=pos)
+        at = oracle.index_scores_at(q[pos], w[pos], k, pos)
+        assert at.shape == (len(pos), 90)
+        for r, t in enumerate(pos):
+            assert np.array_equal(at[r, :t + 1], full[r, :t + 1])
+            assert np.all(np.isnan(at[r, t + 1:]))
+
+
+def test_scores_at_hand_case():
+    """Two compact rows at positions 2 and 0 (H = 1, d = 2, w = [2] and
+    [-1]) over keys k0 = (1, 0), k1 = (0, 1), k2 = (1, 1):
+      row at t = 2, q = (1, -2): dots 1, -2, -1 -> 2*ReLU = 2, 0, 0
+      row at t = 0, q = (3, 1):  dot 3            -> -1*3 = -3."""
+    q_rows = np.array([[[1.0, -2.0]], [[3.0, 1.0]]], np.float32)
+    w_rows = np.array([[2.0], [-1.0]], np.float32)
+    k = np.array([[1.0, 0.0], [0.0, 1.0], [1.0, 1.0]], np.float32)
+    out = oracle.index_scores_at(q_rows, w_rows, k, np.array([2, 0], np.int32))
+    assert out[0].tolist() == [2.0, 0.0, 0.0]
+    assert out[1, 0] == -3.0 and np.all(np.isnan(out[1, 1:]))
+
+
 def test_integer_scores_are_exact_multiples_of_half():
     rng = np.random.default_rng(5)
     L, H, d = 64, 4, 32
@@ -396,6 +434,33 @@ def test_attention_batched_sequences():
 
 
 # ------------------------------------------------------------ stack / misc
+def test_attn_weight_spread_closed_forms():
+    """sqrt(sum_s p_s^2 V[s]^2) with the softmax weights of sparse_attn:
+      * equal logits (Q = 0) give p_s = 1/n: sqrt(sum_s V[s]^2) / n;
+      * one key gives |V[s]|;
+      * two keys with logits 0 and -g (scale 1): p = (1, e^-g)/(1 + e^-g),
+        so sqrt(V_a^2 + e^-2g V_b^2) / (1 + e^-g)."""
+    rng = np.random.default_rng(3)
+    K = rng.standard_normal((20, 4)).astype(np.float32)
+    V = rng.standard_normal((20, 4)).astype(np.float32)
+    sel = np.array([[4, 9, -1, 13, 2, -1]], np.int32)
+    sp = oracle.attn_weight_spread(np.zeros((1, 2, 4), np.float32), K, V, sel)
+    want = np.sqrt((V[[4, 9, 13, 2]].astype(np.float64) ** 2).sum(0)) / 4
+    assert np.allclose(sp[0, 0], want, rtol=1e-12) and np.allclose(sp[0, 1], want, rtol=1e-12)
+    one = oracle.attn_weight_spread(rng.standard_normal((1, 3, 4)).astype(np.float32), K, V,
+                                    np.array([[-1, 7, -1]], np.int32))
+    assert np.allclose(one[0], np.abs(V[7].astype(np.float64))[None, :], rtol=1e-12)
+    # two keys: K rows e0 and e1, Q = (0, -g): logits 0 and -g
+    g = 1.5
+    K2 = np.eye(4, dtype=np.float32)
+    Q2 = np.array([[[0.0, -g, 0.0, 0.0]]], np.float32)
+    V2 = rng.standard_normal((4, 4)).astype(np.float32)
+    sp2 = oracle.attn_weight_spread(Q2, K2, V2, np.array([[0, 1]], np.int32), scale=1.0)
+    e = math.exp(-g)
+    want2 = np.sqrt(V2[0].astype(np.float64) ** 2 + e * e * V2[1].astype(np.float64) ** 2) / (1 + e)
+    assert np.allclose(sp2[0, 0], want2, rtol=1e-12)
+
+
 def test_overlap_page_toy(golden):
     g = golden["overlap_toy"]
     assert oracle.overlap(g["a"], g["b"]) == g["overlap"]
