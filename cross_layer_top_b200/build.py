@@ -2,7 +2,9 @@
 
 Each csrc/*.cu is compiled to an object file under _build/ (in parallel) and
 linked into cross_layer_top_b200/libindexcache.so with the static CUDA
-runtime.  ``python -m cross_layer_top_b200.build`` or ``build()``.
+runtime.  The measurement and test aids in csrc/probe/ become a separate
+library, libindexcache_probe.so, linked against libindexcache.so.
+``python -m cross_layer_top_b200.build`` or ``build()``.
 """
 import concurrent.futures
 import os
@@ -15,6 +17,8 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 OBJ = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libindexcache.so")
+PROBE_DIR = os.path.join(CSRC, "probe")
+PROBE_LIB = os.path.join(HERE, "libindexcache_probe.so")
 INCLUDE = os.path.join(ROOT, "include")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -29,8 +33,8 @@ def nvcc() -> str:
     return exe
 
 
-def sources():
-    return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith(".cu"))
+def sources(folder=CSRC):
+    return sorted(os.path.join(folder, f) for f in os.listdir(folder) if f.endswith(".cu"))
 
 
 def headers():
@@ -38,8 +42,13 @@ def headers():
     return hs + [os.path.join(INCLUDE, f) for f in os.listdir(INCLUDE) if f.endswith(".h")]
 
 
+def _obj(src: str) -> str:
+    sub = "probe_" if os.path.dirname(src) == PROBE_DIR else ""
+    return os.path.join(OBJ, sub + os.path.basename(src)[:-3] + ".o")
+
+
 def _compile(src: str, verbose_ptxas: bool) -> str:
-    obj = os.path.join(OBJ, os.path.basename(src)[:-3] + ".o")
+    obj = _obj(src)
     newest_dep = max(os.path.getmtime(p) for p in headers() + [src])
     if os.path.exists(obj) and os.path.getmtime(obj) >= newest_dep and not verbose_ptxas:
         return obj
@@ -53,23 +62,32 @@ def _compile(src: str, verbose_ptxas: bool) -> str:
     return obj
 
 
+def _link(lib: str, objs, extra=()) -> None:
+    deps = list(objs) + [p for p in extra if p.endswith(".so")]
+    if os.path.exists(lib) and max(os.path.getmtime(o) for o in deps) <= os.path.getmtime(lib):
+        return
+    tmp = lib + ".tmp%d" % os.getpid()
+    cmd = [nvcc()] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + list(objs)
+    if extra:
+        cmd += ["-L", HERE, "-lindexcache", "-Xlinker", "-rpath,$ORIGIN"]
+    r = subprocess.run(cmd, capture_output=True, text=True)
+    if r.returncode != 0:
+        raise RuntimeError("link failed:\n%s%s" % (r.stdout, r.stderr))
+    os.replace(tmp, lib)
+
+
 def build(force: bool = False, verbose_ptxas: bool = False) -> str:
     os.makedirs(OBJ, exist_ok=True)
     srcs = sources()
+    probe_srcs = sources(PROBE_DIR)
     if force:
-        for s in srcs:
-            o = os.path.join(OBJ, os.path.basename(s)[:-3] + ".o")
-            if os.path.exists(o):
-                os.remove(o)
+        for s in srcs + probe_srcs:
+            if os.path.exists(_obj(s)):
+                os.remove(_obj(s))
     with concurrent.futures.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose_ptxas), srcs))
-    if (not os.path.exists(LIB)) or max(os.path.getmtime(o) for o in objs) > os.path.getmtime(LIB):
-        tmp = LIB + ".tmp%d" % os.getpid()
-        cmd = [nvcc()] + ARCH + ["-shared", "-cudart", "static", "-o", tmp] + objs
-        r = subprocess.run(cmd, capture_output=True, text=True)
-        if r.returncode != 0:
-            raise RuntimeError("link failed:\n%s%s" % (r.stdout, r.stderr))
-        os.replace(tmp, LIB)
+        objs = list(ex.map(lambda s: _compile(s, verbose_ptxas), srcs + probe_srcs))
+    _link(LIB, objs[:len(srcs)])
+    _link(PROBE_LIB, objs[len(srcs):], extra=[LIB])
     return LIB
 
 

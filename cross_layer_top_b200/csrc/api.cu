@@ -36,6 +36,14 @@ int cuda_fail(ic_ctx* ctx, cudaError_t e, const char* what) {
     return fail(ctx, IC_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
+int device_error(ic_ctx* ctx, int h) {
+    if (h == kDevBadIndex)
+        return fail(ctx, IC_ERR_DEVICE, "device: an index was outside [-1, kv_len)");
+    if (h == kDevSmemMisaligned)
+        return fail(ctx, IC_ERR_DEVICE, "device: dynamic shared memory not 1024-byte aligned");
+    return fail(ctx, IC_ERR_TIMEOUT, "device: a bounded wait ran out (code %d)", h);
+}
+
 LaunchScope::LaunchScope(ic_ctx* c, int k, cudaStream_t s) : ctx(c), kernel(k), stream(s), slot(0) {
     if (!ctx->timing) return;
     if (ctx->pending == ctx->pool.size()) {
@@ -202,11 +210,7 @@ extern "C" int ic_sync_status(ic_ctx* ctx, void* stream) {
     if (e != cudaSuccess) return cuda_fail(ctx, e, "ic_sync_status: read error word");
     if (h == 0) return IC_OK;
     cudaMemset(ctx->dev_err, 0, sizeof(int));
-    if (h == kDevBadIndex)
-        return fail(ctx, IC_ERR_DEVICE, "device: an index was outside [-1, kv_len)");
-    if (h == kDevSmemMisaligned)
-        return fail(ctx, IC_ERR_DEVICE, "device: dynamic shared memory not 1024-byte aligned");
-    return fail(ctx, IC_ERR_TIMEOUT, "device: a bounded wait ran out (code %d)", h);
+    return device_error(ctx, h);
 }
 
 extern "C" int ic_ctx_set_timing(ic_ctx* ctx, int enable) {

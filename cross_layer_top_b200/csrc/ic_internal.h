@@ -5,6 +5,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+#include <mutex>
 #include <string>
 #include <vector>
 
@@ -60,9 +62,37 @@ struct ic_pattern {
 
 namespace ic {
 
+constexpr int kMaxDevices = 64;
+
+// Once-per-device set-up for host state that CUDA keeps per device, such as
+// a kernel's maximum dynamic shared memory (cudaFuncSetAttribute acts on the
+// current device only).  run(device, f) calls f() the first time it is asked
+// for `device`, and again after f() failed; it is safe to call from several
+// host threads at once.  Devices past kMaxDevices run f() on every call.
+class PerDeviceOnce {
+  public:
+    template <class F>
+    cudaError_t run(int device, F&& f) {
+        if (device < 0 || device >= kMaxDevices) return f();
+        const uint64_t bit = 1ull << device;
+        if (done_.load(std::memory_order_acquire) & bit) return cudaSuccess;
+        std::lock_guard<std::mutex> lock(m_);
+        if (done_.load(std::memory_order_relaxed) & bit) return cudaSuccess;
+        const cudaError_t e = f();
+        if (e == cudaSuccess) done_.fetch_or(bit, std::memory_order_release);
+        return e;
+    }
+
+  private:
+    std::atomic<uint64_t> done_{0};
+    std::mutex m_;
+};
+
 // Records the message on ctx (or the global slot) and returns code.
 int fail(ic_ctx* ctx, int code, const char* fmt, ...);
 int cuda_fail(ic_ctx* ctx, cudaError_t e, const char* what);
+// Maps a nonzero device error word to its IC_ERR_* code and message.
+int device_error(ic_ctx* ctx, int h);
 
 // Brackets one kernel launch with timing events when timing is enabled and
 // counts it.  Usage: LaunchScope ls(ctx, IC_K_TOPK, stream); kernel<<<>>>; ls.done();

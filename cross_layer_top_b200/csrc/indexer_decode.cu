@@ -488,13 +488,12 @@ static int launch_decode_t(ic_ctx* ctx, const void* q, const void* w, const uint
                            const float* kI_scale, const int32_t* seq_len, int B, int S_max,
                            float* scores, int64_t ld, cudaStream_t stream) {
     using S = DecodeShape<H_I>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_index_score_decode<H_I>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
-        if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaFuncSetAttribute(index_decode)");
-        attr_set = true;
-    }
+    static PerDeviceOnce attr_once;
+    cudaError_t ea = attr_once.run(ctx->device, [] {
+        return cudaFuncSetAttribute(k_index_score_decode<H_I>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
+    });
+    if (ea != cudaSuccess) return cuda_fail(ctx, ea, "cudaFuncSetAttribute(index_decode)");
     // tile row coordinates are 32-bit
     if (static_cast<long long>(B) * S_max + S::BM > 0x7FFFFFFFll)
         return fail(ctx, IC_ERR_SHAPE, "decode index: B*S_max=%lld too large",

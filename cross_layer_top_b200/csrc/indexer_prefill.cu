@@ -350,13 +350,11 @@ static int launch_prefill_t(ic_ctx* ctx, const void* qI, const void* kI, const v
                             cudaStream_t stream) {
     using S = PrefillShape<H_I, NATOM, F8>;
     auto kern = k_index_score_prefill<H_I, NATOM, F8>;
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e =
-            cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
-        if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaFuncSetAttribute(index_score)");
-        attr_set = true;
-    }
+    static PerDeviceOnce attr_once;
+    cudaError_t ea = attr_once.run(ctx->device, [&] {
+        return cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
+    });
+    if (ea != cudaSuccess) return cuda_fail(ctx, ea, "cudaFuncSetAttribute(index_score)");
     CUtensorMap tm_q, tm_k;
     int rc;
     if (F8) {

@@ -12,11 +12,19 @@
 // This variant keeps its fp32 score rows in a fixed array in device global
 // memory, defined below, and needs no context.  The array is part of the
 // library's module, so every GPU that loads the library holds it
-// (kNoAllocScoreBytes) until the process exits.  Every call shares it:
-// calls whose kernels overlap on the GPU (different streams, no ordering)
-// race on it.  No entry of the array needs to start at any particular
-// value: the scan writes every score the top-k reads.
+// (kNoAllocScoreFloats fp32 scores) until the process exits.  Every call
+// shares it: calls whose kernels overlap on the GPU (different streams, no
+// ordering) race on it.  No entry of the array needs to start at any
+// particular value: the scan writes every score the top-k reads.
+//
+// Errors found on the device (a bounded wait that ran out, a misaligned
+// shared-memory window) are latched in a device word of the same kind;
+// ic_noalloc_sync_status reads and clears it without allocating.  The host
+// side of each call holds a per-device lock, so calls from several host
+// threads are safe on the host (their kernels still share the array).
 #include <string.h>
+
+#include <mutex>
 
 #include "ic_internal.h"
 
@@ -24,7 +32,7 @@ namespace {
 
 // 4 Mi fp32 scores = 16 MiB: B * round_up(S_max, 64) must not exceed this.
 constexpr size_t kNoAllocScoreFloats = size_t(4) << 20;
-constexpr int kMaxDevices = 64;
+using ic::kMaxDevices;
 
 }  // namespace
 
@@ -37,13 +45,15 @@ static __device__ __align__(256) int g_noalloc_err[64];
 namespace {
 
 struct NoAllocDevice {
+    std::mutex lock;  // held for the host side of every call on this device
     bool ready = false;
     ic_ctx ctx;  // host-side view; its pointers alias the static arrays above
 };
 NoAllocDevice g_dev[kMaxDevices];
 
-// Once per device, with that device current: resolve the device addresses of
-// the static arrays and fill a context that points at them.
+// Once per device, with that device current and its lock held: resolve the
+// device addresses of the static arrays and fill a context that points at
+// them.
 int setup_device(int device, ic_ctx** out) {
     NoAllocDevice& d = g_dev[device];
     if (!d.ready) {
@@ -99,6 +109,7 @@ extern "C" int ic_index_fp_decode_noalloc(const void* q, const void* w, const ui
     cudaError_t e = cudaGetDevice(&device);
     if (e != cudaSuccess || device < 0 || device >= kMaxDevices)
         return ic::fail(nullptr, IC_ERR_CUDA, "decode noalloc: no current device");
+    std::lock_guard<std::mutex> lock(g_dev[device].lock);
     ic_ctx* ctx = nullptr;
     int rc = setup_device(device, &ctx);
     if (rc) return rc;
@@ -109,4 +120,22 @@ extern "C" int ic_index_fp_decode_noalloc(const void* q, const void* w, const ui
         rc = ic::launch_topk(ctx, ctx->scores, ld, B, k, 0, seq_len, S_max, idx_out, k, s);
     if (rc) ic::fail(nullptr, rc, "%s", ctx->last_error.c_str());
     return rc;
+}
+
+extern "C" int ic_noalloc_sync_status(void* stream) {
+    int device = 0;
+    cudaError_t e = cudaGetDevice(&device);
+    if (e != cudaSuccess || device < 0 || device >= kMaxDevices)
+        return ic::fail(nullptr, IC_ERR_CUDA, "noalloc status: no current device");
+    e = cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return ic::cuda_fail(nullptr, e, "noalloc status: stream");
+    // copies between the symbol and a host int: no device allocation
+    int h = 0;
+    e = cudaMemcpyFromSymbol(&h, g_noalloc_err, sizeof(int));
+    if (e != cudaSuccess) return ic::cuda_fail(nullptr, e, "noalloc status: read error word");
+    if (h == 0) return IC_OK;
+    const int zero = 0;
+    e = cudaMemcpyToSymbol(g_noalloc_err, &zero, sizeof(int));
+    if (e != cudaSuccess) return ic::cuda_fail(nullptr, e, "noalloc status: clear error word");
+    return ic::device_error(nullptr, h);
 }

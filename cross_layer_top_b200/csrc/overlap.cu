@@ -88,12 +88,16 @@ int launch_index_overlap(ic_ctx* ctx, const int32_t* a, const int32_t* b, int ro
                     kOverlapMaxKeys);
     const bool byte_map = n_keys <= kOverlapByteMapKeys;
     const int smem = byte_map ? ((n_keys + 3) >> 2) * 4 : ((n_keys + 31) >> 5) * 4;
-    static int attr_bytes = 48 * 1024;
-    if (!byte_map && smem > attr_bytes) {
-        cudaError_t e = cudaFuncSetAttribute(k_index_overlap<false>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    // the bit-map form's shared memory grows with n_keys: its limit is raised
+    // once per device to the largest map this kernel can need
+    static PerDeviceOnce attr_once;
+    if (!byte_map) {
+        cudaError_t e = attr_once.run(ctx->device, [] {
+            return cudaFuncSetAttribute(k_index_overlap<false>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        ((kOverlapMaxKeys + 31) >> 5) * 4);
+        });
         if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaFuncSetAttribute(index_overlap)");
-        attr_bytes = smem;
     }
     LaunchScope ls(ctx, IC_K_OVERLAP, stream);
     if (byte_map)

@@ -1,9 +1,12 @@
-// Measurement aid (include/indexcache_probe.h): the K/V row gather of the
+// libindexcache_probe.so (include/indexcache_probe.h): measurement and test
+// aids kept out of the method's library.  The K/V row gather of the
 // sparse-attention kernel alone, to measure the random-row gather ceiling
-// that bounds attention when K/V sit in L2.  Not part of the method.
-#include "../../include/indexcache_probe.h"
-#include "ic_device.cuh"
-#include "ic_internal.h"
+// that bounds attention when K/V sit in L2; and one bounded device wait that
+// runs out, for the failure-detection test.  Not part of the method.  Links
+// against libindexcache.so (error messages, the context's error word).
+#include "../../../include/indexcache_probe.h"
+#include "../ic_device.cuh"
+#include "../ic_internal.h"
 
 namespace ic {
 

@@ -523,25 +523,28 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
                          int64_t kv_seq_stride, int kv_len, float scale, void* out,
                          cudaStream_t stream) {
     using S = AttnShape<D>;
-    static bool attr_set = false;
-    if (!attr_set) {
+    static PerDeviceOnce attr_once;
+    cudaError_t ea = attr_once.run(ctx->device, [] {
         cudaError_t e = cudaFuncSetAttribute(k_sparse_attn<D, false>,
                                              cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(k_sparse_attn<D, true>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_SPLIT);
-        if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaFuncSetAttribute(sparse_attn)");
-        attr_set = true;
-    }
+        return e;
+    });
+    if (ea != cudaSuccess) return cuda_fail(ctx, ea, "cudaFuncSetAttribute(sparse_attn)");
     // Split the index slots across CTAs when there are too few rows to fill
     // the GPU (decode): about one wave of resident CTAs, whole chunks per
     // split, at most kMaxClusterSplits.  A split row's CTAs form one cluster
     // (they merge through distributed shared memory); the split count is
     // lowered until every row's cluster can be resident at once (a cluster
     // waiting for a second wave would double the kernel's time).
-    static int active[kMaxClusterSplits + 1] = {};  // resident clusters per cluster size (0: unknown)
+    // resident clusters per device and cluster size (0: not yet asked)
+    static std::atomic<int> active[kMaxDevices][kMaxClusterSplits + 1] = {};
+    const int dev = ctx->device >= 0 && ctx->device < kMaxDevices ? ctx->device : 0;
     auto resident_clusters = [&](int cs) -> int {
-        if (active[cs] == 0) {
+        int n = active[dev][cs].load(std::memory_order_relaxed);
+        if (n == 0) {
             cudaLaunchConfig_t q = {};
             q.gridDim = dim3(1, cs, 1);
             q.blockDim = dim3(S::THREADS, 1, 1);
@@ -553,12 +556,11 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
             qa[0].val.clusterDim.z = 1;
             q.attrs = qa;
             q.numAttrs = 1;
-            int n = 0;
             if (cudaOccupancyMaxActiveClusters(&n, k_sparse_attn<D, true>, &q) != cudaSuccess) n = -1;
             cudaGetLastError();  // a refused query leaves no error behind
-            active[cs] = n;
+            active[dev][cs].store(n, std::memory_order_relaxed);
         }
-        return active[cs];
+        return n;
     };
     int nsplit = 1;
     const int target = S::CTAS_PER_SM * ctx->num_sms;

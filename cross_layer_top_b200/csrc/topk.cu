@@ -665,13 +665,12 @@ int launch_topk(ic_ctx* ctx, const float* scores, int64_t ld, int rows, int k, i
         max_len > 16384 && max_len <= kClusterCtas * 45000)
         return launch_topk_cluster(ctx, scores, ld, rows, k, causal_base, row_len, max_len, idx_out,
                                    ld_out, stream);
-    static bool attr_set = false;
-    if (!attr_set) {
-        cudaError_t e = cudaFuncSetAttribute(k_topk, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             kCandCap * 4 + kBitmapCap / 8);
-        if (e != cudaSuccess) return cuda_fail(ctx, e, "cudaFuncSetAttribute(topk)");
-        attr_set = true;
-    }
+    static PerDeviceOnce attr_once;
+    cudaError_t ea = attr_once.run(ctx->device, [] {
+        return cudaFuncSetAttribute(k_topk, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    kCandCap * 4 + kBitmapCap / 8);
+    });
+    if (ea != cudaSuccess) return cuda_fail(ctx, ea, "cudaFuncSetAttribute(topk)");
     // causal row r has n = causal_base + r + 1 keys; rows longer than the
     // bitmap holds take the general path
     const long long nmax = row_len ? max_len : static_cast<long long>(causal_base) + rows;

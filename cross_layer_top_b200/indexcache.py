@@ -80,12 +80,11 @@ _SIGS = {
     "ic_index_score_decode": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _i64, _vp], _i),
     "ic_index_fp_decode": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp], _i),
     "ic_index_fp_decode_noalloc": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _vp], _i),
-    "ic_probe_gather": ([_vp, _vp, _vp, _i, _i, _i, _i, _vp], _i),
     "ic_sparse_attn": ([_vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i64, _i, _f, _vp, _vp], _i),
     "ic_index_overlap": ([_vp, _vp, _vp, _i, _i, _i, _vp, _vp], _i),
     "ic_index_score_fp8": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _i64, _vp], _i),
     "ic_index_fp_fp8": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _vp, _vp], _i),
-    "ic_probe_wait_timeout": ([_vp, _vp], _i),
+    "ic_noalloc_sync_status": ([_vp], _i),
     "ic_run_stack": ([_vp, _vp, ctypes.POINTER(ic_layer_io), ctypes.POINTER(ic_stack_dims), _vp,
                       _vp], _i),
     "ic_run_stack_host": ([_vp, _vp, ctypes.POINTER(ic_layer_io), ctypes.POINTER(ic_stack_dims),
@@ -300,6 +299,12 @@ def ic_index_fp_decode_noalloc(q, w, kI8, kI_scale, seq_len, k: int, idx_out, st
                                            _stream(stream)))
 
 
+def ic_noalloc_sync_status(stream=None):
+    """Synchronize `stream`, then report (and clear) the device error word of
+    the allocation-free path on the current device; raises ICError."""
+    _check(_lib.ic_noalloc_sync_status(_stream(stream)))
+
+
 def ic_sparse_attn(ctx: Context, Q, K, V, idx, out, rows_per_seq: int = 0, kv_seq_stride: int = 0,
                    kv_len=None, scale: float = 0.0, stream=None):
     rows, Hq, d = Q.shape
@@ -345,19 +350,6 @@ def ic_index_overlap(ctx: Context, idx_a, idx_b, hits, n_keys: int, stream=None)
         raise ValueError("idx_a and idx_b must have the same shape")
     _check(_lib.ic_index_overlap(ctx.handle, _ptr(idx_a), _ptr(idx_b), rows, k, n_keys, _ptr(hits),
                                  _stream(stream)), ctx)
-
-
-def ic_probe_wait_timeout(ctx: Context, stream=None):
-    """Test aid: one bounded device wait that runs out (about a second); the
-    next ctx.sync_status() raises IC_ERR_TIMEOUT."""
-    _check(_lib.ic_probe_wait_timeout(ctx.handle, _stream(stream)), ctx)
-
-
-def ic_probe_gather(K, V, idx, ctas_per_sm: int = 2, stream=None):
-    """Measurement aid: the attention's K/V row gather alone (no compute)."""
-    rows, k = idx.shape
-    _check(_lib.ic_probe_gather(_ptr(K), _ptr(V), _ptr(idx), rows, k, K.shape[-1], ctas_per_sm,
-                                _stream(stream)))
 
 
 def make_stack_layers(layers, mode=IC_PREFILL):

@@ -203,12 +203,24 @@ int ic_index_fp_decode(ic_ctx *ctx, const void *q, const void *w, const uint8_t 
  * exit): B * round_up(S_max, 64) must be <= 4194304, else IC_ERR_UNSUPPORTED
  * with a message.  The first call on a device resolves that array's address
  * (cudaGetSymbolAddress) and should come before any stream capture.  All
- * calls share the array: calls whose kernels overlap on the GPU race.
- * Device-side wait timeouts are not reported (the call never
- * synchronizes).  Error messages: ic_last_error(NULL). */
+ * calls share the array: calls whose kernels overlap on the GPU race.  The
+ * host side of a call holds a per-device lock, so host threads may call it
+ * concurrently.  The call never synchronizes: errors found on the device (a
+ * bounded wait that ran out, a misaligned shared-memory window) are latched
+ * in a device word of the library, which ic_noalloc_sync_status reports;
+ * after such an error the indices of the calls before that report are not
+ * valid.  Error messages: ic_last_error(NULL). */
 int ic_index_fp_decode_noalloc(const void *q, const void *w, const uint8_t *kI8,
                                const float *kI_scale, const int32_t *seq_len, int B, int S_max,
                                int H_I, int d_I, int k, int32_t *idx_out, void *stream);
+
+/* Status of ic_index_fp_decode_noalloc on the current device, also without
+ * allocating: synchronizes `stream`, then reads and clears the device error
+ * word that the allocation-free path's kernels latch (copies between a host
+ * int and the library's device symbol).  Returns IC_OK, IC_ERR_TIMEOUT,
+ * IC_ERR_DEVICE or IC_ERR_CUDA; message in ic_last_error(NULL).  Like the
+ * entry point it reports on, it has no counterpart on the pages. */
+int ic_noalloc_sync_status(void *stream);
 
 /* ------------------------------------------------------ sparse attention */
 

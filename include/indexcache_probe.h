@@ -1,6 +1,8 @@
 /*
- * indexcache_probe.h — measurement aid of libindexcache.so (not part of the
- * IndexCache method; the pages have no counterpart).
+ * indexcache_probe.h — libindexcache_probe.so, a separate measurement and
+ * test library beside libindexcache.so (not part of the IndexCache method;
+ * the pages have no counterpart).  It links against libindexcache.so, whose
+ * contexts ic_probe_wait_timeout takes.
  *
  * ic_probe_gather enqueues a kernel that performs exactly the K/V row
  * gather of sparse attention and nothing else: for each of `rows` query

@@ -1,7 +1,9 @@
-"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
-every symbol include/indexcache.h declares, and its host-only logic
-(patterns, argument checks) behaves; the pattern resolution is checked
-against the oracle's."""
+"""Host-side checks of the C ABI (no GPU needed): each library loads and
+exports every symbol its header declares (include/indexcache.h for
+libindexcache.so, include/indexcache_probe.h for the separate
+libindexcache_probe.so, whose symbols the method's library must not carry),
+and its host-only logic (patterns, argument checks) behaves; the pattern
+resolution is checked against the oracle's."""
 import ctypes
 import os
 import re
@@ -11,6 +13,8 @@ import pytest
 import oracle
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+MAIN_HEADER = os.path.join(ROOT, "include", "indexcache.h")
+PROBE_HEADER = os.path.join(ROOT, "include", "indexcache_probe.h")
 HEADERS = [os.path.join(ROOT, "include", f) for f in sorted(os.listdir(os.path.join(ROOT, "include")))
            if f.endswith(".h")]
 
@@ -27,9 +31,13 @@ def ic():
     return indexcache
 
 
-def declared_symbols():
-    text = "\n".join(open(h).read() for h in HEADERS)
+def declared_symbols(headers=(MAIN_HEADER,)):
+    text = "\n".join(open(h).read() for h in headers)
     return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(ic_\w+)\s*\(", text, re.M)))
+
+
+def test_every_header_belongs_to_a_library():
+    assert sorted(HEADERS) == sorted([MAIN_HEADER, PROBE_HEADER])
 
 
 def test_header_declares_the_boundary():
@@ -45,6 +53,25 @@ def test_library_exports_every_declared_symbol(ic):
     assert not missing, missing
     # and the binding covers the same set
     assert set(declared_symbols()) <= set(ic.EXPORTED)
+
+
+def test_probe_library_is_separate(ic):
+    from cross_layer_top_b200 import probe
+    probe_syms = declared_symbols((PROBE_HEADER,))
+    assert probe_syms == ["ic_probe_gather", "ic_probe_wait_timeout"]
+    plib = ctypes.CDLL(probe.LIB_PATH)
+    assert all(hasattr(plib, s) for s in probe_syms)
+    assert set(probe_syms) <= set(probe.EXPORTED)
+    # the method's library exports none of the aids
+    names = subprocess_nm(ic.LIB_PATH)
+    assert not [s for s in probe_syms if s in names]
+
+
+def subprocess_nm(path):
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True,
+                         check=True).stdout
+    return {line.split()[-1] for line in out.splitlines() if line.strip()}
 
 
 def test_version(ic):

@@ -18,8 +18,9 @@ def ic():
 
 
 def test_bounded_wait_reports_timeout_and_context_survives(ic):
+    from cross_layer_top_b200 import probe
     ctx = ic.Context(0)
-    ic.ic_probe_wait_timeout(ctx)
+    probe.ic_probe_wait_timeout(ctx)
     with pytest.raises(ic.ICError) as e:
         ctx.sync_status()
     assert e.value.code == ic.IC_ERR_TIMEOUT
