@@ -32,8 +32,10 @@ def test_reference_arm_json_line():
     assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "pairs/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
-    # the step time is the stack's scored pairs at the measured rate
+    # the step time is the stack's scored pairs at the measured rate, and the
+    # line says it is extrapolated from bounded samples, with their seconds
     assert d["ms_per_step"] > 0
+    assert d["extrapolated"] is True and d["measured_s"] > 0
 
 
 def test_reference_arm_other_ranks_silent():
