@@ -9,7 +9,7 @@ Acceptance bars:
   * attention (on the GPU's own indices) within 2e-2 max abs and 1e-2
     relative (|g - o| <= 2e-2 + 1e-2 |o|) of the fp64 oracle, and within the
     bound of bf16 arithmetic that scales with the output
-    (|g - o| <= 2^-8 |o| + 6 * 2^-9 * spread + 1e-6, tests/attn_check.py).
+    (|g - o| <= 2^-7 |o| + 6 * 2^-8 * spread + 1e-6, tests/attn_check.py).
 """
 import math
 
