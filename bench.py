@@ -389,6 +389,77 @@ def measure_overlap(ctx, layers, cfg, stream):
             "bytes_per_launch": 2 * L * k * 4}
 
 
+def run_split(args, rank, world, local_rank):
+    """--prefill-split: ONE prefill sequence split over the ranks by query rows
+    (strong scaling).  Each rank holds its rows of every layer (the
+    causal-balanced partition of ic_prefill_partition); a step is one NCCL
+    all-gather per k_I / K / V tensor of the ranks' rows, then
+    ic_run_stack_rows on the rank's rows.  value = the sequence's scored
+    pairs per step / the max-over-ranks step time."""
+    from cross_layer_top_b200 import indexcache as ic
+    from cross_layer_top_b200 import sharding, synth
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    cfg = synth.CONFIGS[WORKLOAD]
+    L, k = cfg.L, cfg.k
+    parts = sharding.partition(L, world)
+    mine = parts[rank]
+    n = sum(b - a for a, b in mine)
+    ctx = ic.Context(local_rank)
+    pat = ic.ic_create_pattern(cfg.pattern)
+    dims = ic.stack_dims(ic.IC_PREFILL, cfg.H_I, cfg.d_I, k, cfg.Hq, cfg.d, L=L)
+    local, gathered = [], []
+    for l in range(cfg.n_layers):
+        full = synth.prefill_layer(cfg, l, dev)  # same seed on every rank: take my rows
+        loc = {m: sharding.rows_of(t, mine) for m, t in full.items()}
+        loc["out"] = torch.empty((n, cfg.Hq, cfg.d), dtype=torch.bfloat16, device=dev)
+        local.append(loc)
+        del full
+    cache = torch.empty((n, k), dtype=torch.int32, device=dev)
+
+    def step():
+        lays = []
+        for loc in local:
+            lay = dict(loc)
+            for m in ("kI", "K", "V"):
+                if m in loc:
+                    lay[m] = sharding.allgather_rows(loc[m], parts, L)
+            lays.append(lay)
+        ic.ic_run_stack_rows(ctx, pat, lays, dims, mine, cache)
+        return lays
+
+    for _ in range(args.warmup):
+        step()
+    ctx.sync_status()
+    dist_barrier(world)
+    torch.cuda.synchronize()
+    stream = torch.cuda.current_stream()
+    launches0 = ctx.launch_count()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(args.steps):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize()
+    dist_barrier(world)
+    ms = dist_max(a.elapsed_time(b), world)
+    launches = ctx.launch_count() - launches0
+    pairs_step = scored_pairs(L, k, cfg.pattern.count("F"))
+    line = {"metric": METRIC, "value": pairs_step * args.steps / (ms / 1e3), "unit": "pairs/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "strong",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "prefill stack split by query rows: 1 sequence over %d GPUs, "
+                                   "L=16384, FSSSFSSS, H_I=64, d_I=128, k=2048, 16 query heads, "
+                                   "d=128; per step one all-gather per k_I/K/V tensor" % world,
+                       "global_batch": 1, "seq_len": L, "parallelism": "rows%d" % world,
+                       "rows_per_rank": n},
+            "gpu_launches": launches}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    ctx.close()
+
+
 def run_e2e(args, ctx, pat, dims, cfg, layers, cache, world, pairs_step, stream):
     """Same metric through the library's host-memory entry point
     (ic_run_stack_host): every step copies all layer inputs host->device from
@@ -874,6 +945,10 @@ def main():
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the decode workload (not the contract line)")
     ap.add_argument("--decode-layers", type=int, default=0)
+    ap.add_argument("--prefill-split", action="store_true",
+                    help="one prefill sequence split over the ranks by query rows (strong "
+                         "scaling, an all-gather of k_I/K/V per step) instead of one sequence "
+                         "per rank")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours":
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -899,7 +974,10 @@ def main():
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
                                              device_id=torch.device("cuda", local_rank))
     try:
-        run_ours(args, rank, world, local_rank)
+        if args.prefill_split:
+            run_split(args, rank, world, local_rank)
+        else:
+            run_ours(args, rank, world, local_rank)
     finally:
         if world > 1:
             torch.distributed.destroy_process_group()

@@ -358,35 +358,42 @@ extern "C" int ic_topk(ic_ctx* ctx, const float* scores, int64_t ld, int rows, i
                        as_stream(stream));
 }
 
-// F layer: rows t < k select {0..t} without scores; the other rows are
-// scored in chunks whose fp32 rows fit in the scratch limit, each chunk
-// followed by its top-k.  `score(rb, re, scores, ld)` scores rows [rb, re).
+// F layer over query rows [r0, r1) (idx_out row 0 is row r0): rows t < k
+// select {0..t} without scores; the other rows are scored in chunks whose
+// fp32 rows fit in the scratch limit, each chunk followed by its top-k.
+// `score(rb, re, scores, ld)` scores rows [rb, re).
 template <class ScoreFn>
-static int index_fp_rows(ic_ctx* ctx, int L, int k, int32_t* idx_out, cudaStream_t s,
-                         ScoreFn score) {
-    const int first = k < L ? k : L;
-    if (first > 0) {
-        int rc = launch_topk(ctx, nullptr, 0, first, k, 0, nullptr, 0, idx_out, k, s);
+static int index_fp_range(ic_ctx* ctx, int r0, int r1, int k, int32_t* idx_out, cudaStream_t s,
+                          ScoreFn score) {
+    const int first = r0 > k ? r0 : (k < r1 ? k : r1);  // rows [r0, first) need no score
+    if (first > r0) {
+        int rc = launch_topk(ctx, nullptr, 0, first - r0, k, r0, nullptr, 0, idx_out, k, s);
         if (rc) return rc;
     }
-    if (first >= L) return IC_OK;
-    const int64_t ld = (static_cast<int64_t>(L) + 63) / 64 * 64;
+    if (first >= r1) return IC_OK;
+    const int64_t ld = (static_cast<int64_t>(r1) + 63) / 64 * 64;
     int64_t chunk = static_cast<int64_t>(ctx->scratch_limit / (static_cast<size_t>(ld) * 4));
     if (chunk < 1) return fail(ctx, IC_ERR_NOMEM, "index_fp: scratch too small for one row");
-    if (chunk > L - first) chunk = L - first;
+    if (chunk > r1 - first) chunk = r1 - first;
     int rc = ensure_buffer(ctx, reinterpret_cast<void**>(&ctx->scores), &ctx->scores_cap,
                            static_cast<size_t>(chunk) * ld * 4);
     if (rc) return rc;
-    for (int rb = first; rb < L; rb += static_cast<int>(chunk)) {
-        const int re = static_cast<int>(rb + chunk < L ? rb + chunk : L);
+    for (int rb = first; rb < r1; rb += static_cast<int>(chunk)) {
+        const int re = static_cast<int>(rb + chunk < r1 ? rb + chunk : r1);
         const int64_t ldc = (static_cast<int64_t>(re) + 63) / 64 * 64;
         rc = score(rb, re, ctx->scores, ldc);
         if (rc) return rc;
         rc = launch_topk(ctx, ctx->scores, ldc, re - rb, k, rb,
-                         nullptr, 0, idx_out + static_cast<int64_t>(rb) * k, k, s);
+                         nullptr, 0, idx_out + static_cast<int64_t>(rb - r0) * k, k, s);
         if (rc) return rc;
     }
     return IC_OK;
+}
+
+template <class ScoreFn>
+static int index_fp_rows(ic_ctx* ctx, int L, int k, int32_t* idx_out, cudaStream_t s,
+                         ScoreFn score) {
+    return index_fp_range(ctx, 0, L, k, idx_out, s, score);
 }
 
 extern "C" int ic_index_fp(ic_ctx* ctx, const void* qI, const void* kI, const void* w, int L,
@@ -400,6 +407,53 @@ extern "C" int ic_index_fp(ic_ctx* ctx, const void* qI, const void* kI, const vo
     return index_fp_rows(ctx, L, k, idx_out, s, [&](int rb, int re, float* sc, int64_t ldc) {
         return launch_index_score_prefill(ctx, qI, kI, w, L, H_I, d_I, rb, re, sc, ldc, s);
     });
+}
+
+// The F layer of one range of query rows whose q_I / w rows are held
+// compactly (a rank's share of a prefill split across GPUs).
+extern "C" int ic_index_fp_rows(ic_ctx* ctx, const void* qI_rows, const void* w_rows,
+                                const void* kI, int L, int H_I, int d_I, int row_begin,
+                                int row_end, int k, int32_t* idx_out, void* stream) {
+    if (!ctx) return fail(nullptr, IC_ERR_INVALID_ARG, "context is NULL");
+    if (k < 1 || k > 2048) return fail(ctx, IC_ERR_SHAPE, "index_fp_rows: k=%d not in [1,2048]", k);
+    if (row_begin < 0 || row_end > L || row_begin > row_end)
+        return fail(ctx, IC_ERR_SHAPE, "index_fp_rows: rows [%d,%d) outside [0,%d)", row_begin,
+                    row_end, L);
+    if (row_end == row_begin) return IC_OK;  // no rows: nothing is read or written
+    int rc = check_index_args(ctx, qI_rows, kI, w_rows, L, H_I, d_I);
+    if (rc) return rc;
+    if (!idx_out) return fail(ctx, IC_ERR_INVALID_ARG, "index_fp_rows: idx_out is NULL");
+    cudaSetDevice(ctx->device);
+    cudaStream_t s = as_stream(stream);
+    const int n = row_end - row_begin;
+    return index_fp_range(ctx, row_begin, row_end, k, idx_out, s,
+                          [&](int rb, int re, float* sc, int64_t ldc) {
+                              return launch_index_score_prefill(ctx, qI_rows, kI, w_rows, L, H_I,
+                                                                d_I, rb, re, sc, ldc, s, row_begin,
+                                                                n);
+                          });
+}
+
+// Causal-balanced split of L query rows over `world` ranks: 2*world chunks
+// of near-equal size (the first L % (2*world) one row longer); rank r takes
+// chunks r and 2*world - 1 - r, so an early (cheap) and a late (costly)
+// chunk pair up.
+extern "C" int ic_prefill_partition(int L, int world, int rank, int32_t* ranges, int* n_ranges) {
+    if (!ranges || !n_ranges || L < 0 || world < 1 || rank < 0 || rank >= world)
+        return fail(nullptr, IC_ERR_INVALID_ARG, "prefill_partition: L=%d world=%d rank=%d", L,
+                    world, rank);
+    const int64_t nch = 2ll * world;
+    auto start = [&](int64_t c) {  // first row of chunk c
+        const int64_t base = L / nch, extra = L % nch;
+        return c * base + (c < extra ? c : extra);
+    };
+    const int64_t ca = rank, cb = nch - 1 - rank;
+    ranges[0] = static_cast<int32_t>(start(ca));
+    ranges[1] = static_cast<int32_t>(start(ca + 1));
+    ranges[2] = static_cast<int32_t>(start(cb));
+    ranges[3] = static_cast<int32_t>(start(cb + 1));
+    *n_ranges = 2;
+    return IC_OK;
 }
 
 // ------------------------------------------------ FP8 prefill indexer
@@ -619,6 +673,54 @@ int check_stack_args(ic_ctx* ctx, const ic_pattern* pattern, const void* layers,
     return IC_OK;
 }
 }  // namespace ic
+
+extern "C" int ic_run_stack_rows(ic_ctx* ctx, const ic_pattern* pattern, const ic_layer_io* layers,
+                                 const ic_stack_dims* dims, const int32_t* ranges, int n_ranges,
+                                 int32_t* idx_cache, void* stream) {
+    int rc = check_stack_args(ctx, pattern, layers, dims, idx_cache);
+    if (rc) return rc;
+    if (dims->mode != IC_PREFILL)
+        return fail(ctx, IC_ERR_INVALID_ARG, "run_stack_rows: prefill stacks only");
+    if (!ranges || n_ranges < 1) return fail(ctx, IC_ERR_INVALID_ARG, "run_stack_rows: no ranges");
+    int64_t rows = 0;
+    for (int i = 0; i < n_ranges; ++i) {
+        const int a = ranges[2 * i], b = ranges[2 * i + 1];
+        if (a < 0 || b > dims->L || a > b)
+            return fail(ctx, IC_ERR_SHAPE, "run_stack_rows: range [%d,%d) outside [0,%d)", a, b,
+                        dims->L);
+        rows += b - a;
+    }
+    cudaSetDevice(ctx->device);
+    const int N = static_cast<int>(pattern->c.size());
+    const int k = dims->k;
+    for (int l = 0; l < N; ++l) {
+        const ic_layer_io& io = layers[l];
+        if (pattern->c[l] == 'F') {
+            int64_t off = 0;
+            for (int i = 0; i < n_ranges; ++i) {
+                const int a = ranges[2 * i], b = ranges[2 * i + 1];
+                const char* q = static_cast<const char*>(io.qI) + off * dims->H_I * dims->d_I * 2;
+                const char* w = static_cast<const char*>(io.w) + off * dims->H_I * 2;
+                rc = ic_index_fp_rows(ctx, q, w, io.kI, dims->L, dims->H_I, dims->d_I, a, b, k,
+                                      idx_cache + off * k, stream);
+                if (rc) return rc;
+                off += b - a;
+            }
+        }
+        const int32_t* idx = nullptr;
+        ic_index_reuse(idx_cache, &idx);
+        if (io.idx_snapshot) {
+            cudaError_t e = cudaMemcpyAsync(io.idx_snapshot, idx,
+                                            static_cast<size_t>(rows) * k * sizeof(int32_t),
+                                            cudaMemcpyDeviceToDevice, as_stream(stream));
+            if (e != cudaSuccess) return cuda_fail(ctx, e, "run_stack_rows: snapshot copy");
+        }
+        rc = ic_sparse_attn(ctx, io.Q, io.K, io.V, idx, static_cast<int>(rows), dims->Hq, dims->d,
+                            k, 0, 0, dims->L, dims->scale, io.out, stream);
+        if (rc) return rc;
+    }
+    return IC_OK;
+}
 
 extern "C" int ic_run_stack(ic_ctx* ctx, const ic_pattern* pattern, const ic_layer_io* layers,
                             const ic_stack_dims* dims, int32_t* idx_cache, void* stream) {

@@ -141,9 +141,10 @@ int run_stack_layer(ic_ctx* ctx, char c, const ic_layer_io& io, const ic_layer_i
 int check_stack_args(ic_ctx* ctx, const ic_pattern* pattern, const void* layers,
                      const ic_stack_dims* dims, const int32_t* idx_cache);
 
+// q_I and w hold rows [q_row0, q_row0 + q_rows) (q_rows < 0: every row of L)
 int launch_index_score_prefill(ic_ctx* ctx, const void* qI, const void* kI, const void* w, int L,
                                int H_I, int d_I, int row_begin, int row_end, float* scores,
-                               int64_t ld, cudaStream_t stream);
+                               int64_t ld, cudaStream_t stream, int q_row0 = 0, int q_rows = -1);
 int launch_index_score_decode(ic_ctx* ctx, const void* q, const void* w, const uint8_t* kI8,
                               const float* kI_scale, const int32_t* seq_len, int B, int S_max,
                               int H_I, int d_I, float* scores, int64_t ld, cudaStream_t stream);

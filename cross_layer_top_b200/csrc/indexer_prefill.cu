@@ -2,6 +2,8 @@
 //
 // Computes, for query rows t in [row_begin, row_end) and keys s <= t,
 //   I[t,s] = sum_j w[t,j] * ReLU(q_I[t,j,:] . k_I[s,:])
+// The q_I and w tensors may hold a window of rows only: row t of them is at
+// t - q_row0 (q_row0 = 0 when they hold every row).
 // ("IndexCache：跨层复用稀疏索引，以及它为什么能被训练", §2.1, the DSA
 // lightning-indexer score; "IndexCache: Accelerating Sparse Attention via
 // Cross-Layer Index Reuse", §2.1: the indexer scores all preceding tokens).
@@ -75,7 +77,7 @@ __global__ void __launch_bounds__(PrefillShape<H_I, NATOM, F8>::THREADS, 1)
                           const __nv_bfloat16* __restrict__ w, const float* __restrict__ q_scale,
                           const float* __restrict__ k_scale, float* __restrict__ scores,
                           long long ld, int L, int row_begin, int row_end, int n_items,
-                          int* __restrict__ err) {
+                          int q_row0, int q_rows, int* __restrict__ err) {
     using S = PrefillShape<H_I, NATOM, F8>;
     constexpr int KST = S::KSTAGES;
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -150,7 +152,7 @@ __global__ void __launch_bounds__(PrefillShape<H_I, NATOM, F8>::THREADS, 1)
 #pragma unroll
                 for (int k = 0; k < NATOM; ++k)
                     tma_load_2d(sB + a * S::B_ACC + k * S::B_ATOM, &tm_q, q_full, k * 64,
-                                (t0 + a * S::TOK_PER_ACC) * H_I);
+                                (t0 - q_row0 + a * S::TOK_PER_ACC) * H_I);
             q_last = q_it & 1;
             ++q_it;
             for (int kt = 0; kt < n_tiles; ++kt) {
@@ -262,10 +264,10 @@ __global__ void __launch_bounds__(PrefillShape<H_I, NATOM, F8>::THREADS, 1)
 #pragma unroll
                 for (int q = 0; q < CPL; ++q) {
                     const int c = lane * CPL + q;  // column within the group
-                    const int t = tok0 + c / H_I;
-                    const size_t wi = static_cast<size_t>(t) * H_I + (c % H_I);
-                    float wv = t < L ? __bfloat162float(w[wi]) : 0.f;
-                    if (F8 && t < L) wv *= q_scale[wi];
+                    const int tq = tok0 + c / H_I - q_row0;  // row in the q_I / w window
+                    const size_t wi = static_cast<size_t>(tq) * H_I + (c % H_I);
+                    float wv = tq < q_rows ? __bfloat162float(w[wi]) : 0.f;
+                    if (F8 && tq < q_rows) wv *= q_scale[wi];
                     wW[a * COLS + c] = wv;
                 }
             }
@@ -346,8 +348,8 @@ __global__ void __launch_bounds__(PrefillShape<H_I, NATOM, F8>::THREADS, 1)
 template <int H_I, int NATOM, bool F8>
 static int launch_prefill_t(ic_ctx* ctx, const void* qI, const void* kI, const void* w,
                             const float* q_scale, const float* k_scale, int L, int d_I,
-                            int row_begin, int row_end, float* scores, int64_t ld,
-                            cudaStream_t stream) {
+                            int row_begin, int row_end, float* scores, int64_t ld, int q_row0,
+                            int q_rows, cudaStream_t stream) {
     using S = PrefillShape<H_I, NATOM, F8>;
     auto kern = k_index_score_prefill<H_I, NATOM, F8>;
     static PerDeviceOnce attr_once;
@@ -358,11 +360,12 @@ static int launch_prefill_t(ic_ctx* ctx, const void* qI, const void* kI, const v
     CUtensorMap tm_q, tm_k;
     int rc;
     if (F8) {
-        rc = make_tmap_u8_2d(ctx, &tm_q, qI, static_cast<uint64_t>(L) * H_I, d_I, 128, S::BN, true);
+        rc = make_tmap_u8_2d(ctx, &tm_q, qI, static_cast<uint64_t>(q_rows) * H_I, d_I, 128, S::BN,
+                             true);
         if (rc) return rc;
         rc = make_tmap_u8_2d(ctx, &tm_k, kI, static_cast<uint64_t>(L), d_I, 128, S::BM, true);
     } else {
-        rc = make_tmap_bf16_2d(ctx, &tm_q, qI, static_cast<uint64_t>(L) * H_I, d_I, S::BN);
+        rc = make_tmap_bf16_2d(ctx, &tm_q, qI, static_cast<uint64_t>(q_rows) * H_I, d_I, S::BN);
         if (rc) return rc;
         rc = make_tmap_bf16_2d(ctx, &tm_k, kI, static_cast<uint64_t>(L), d_I, S::BM);
     }
@@ -372,7 +375,7 @@ static int launch_prefill_t(ic_ctx* ctx, const void* qI, const void* kI, const v
     LaunchScope ls(ctx, IC_K_INDEX_SCORE, stream);
     kern<<<grid, S::THREADS, S::SMEM, stream>>>(tm_q, tm_k, static_cast<const __nv_bfloat16*>(w), q_scale,
                                          k_scale, scores, static_cast<long long>(ld), L, row_begin,
-                                         row_end, n_items, ctx->dev_err);
+                                         row_end, n_items, q_row0, q_rows, ctx->dev_err);
     cudaError_t e = ls.done();
     if (e != cudaSuccess) return cuda_fail(ctx, e, "index_score launch");
     return IC_OK;
@@ -380,17 +383,18 @@ static int launch_prefill_t(ic_ctx* ctx, const void* qI, const void* kI, const v
 
 int launch_index_score_prefill(ic_ctx* ctx, const void* qI, const void* kI, const void* w, int L,
                                int H_I, int d_I, int row_begin, int row_end, float* scores,
-                               int64_t ld, cudaStream_t stream) {
+                               int64_t ld, cudaStream_t stream, int q_row0, int q_rows) {
     if (row_end <= row_begin) return IC_OK;
+    if (q_rows < 0) q_rows = L;  // q_I and w hold every row
     const bool one_atom = d_I <= 64;
 #define IC_PREFILL_CASE(H)                                                                      \
     case H:                                                                                     \
         return one_atom ? launch_prefill_t<H, 1, false>(ctx, qI, kI, w, nullptr, nullptr, L,    \
                                                         d_I, row_begin, row_end, scores, ld,    \
-                                                        stream)                                 \
+                                                        q_row0, q_rows, stream)                 \
                         : launch_prefill_t<H, 2, false>(ctx, qI, kI, w, nullptr, nullptr, L,    \
                                                         d_I, row_begin, row_end, scores, ld,    \
-                                                        stream);
+                                                        q_row0, q_rows, stream);
     switch (H_I) {
         IC_PREFILL_CASE(4)
         IC_PREFILL_CASE(8)
@@ -413,13 +417,13 @@ int launch_index_score_prefill_fp8(ic_ctx* ctx, const uint8_t* qI8, const float*
     switch (H_I) {
         case 16:
             return launch_prefill_t<16, 1, true>(ctx, qI8, kI8, w, q_scale, k_scale, L, d_I,
-                                                 row_begin, row_end, scores, ld, stream);
+                                                 row_begin, row_end, scores, ld, 0, L, stream);
         case 32:
             return launch_prefill_t<32, 1, true>(ctx, qI8, kI8, w, q_scale, k_scale, L, d_I,
-                                                 row_begin, row_end, scores, ld, stream);
+                                                 row_begin, row_end, scores, ld, 0, L, stream);
         case 64:
             return launch_prefill_t<64, 1, true>(ctx, qI8, kI8, w, q_scale, k_scale, L, d_I,
-                                                 row_begin, row_end, scores, ld, stream);
+                                                 row_begin, row_end, scores, ld, 0, L, stream);
         default:
             return fail(ctx, IC_ERR_UNSUPPORTED, "index_score_fp8: H_I=%d not in {16,32,64}", H_I);
     }

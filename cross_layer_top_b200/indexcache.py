@@ -89,6 +89,10 @@ _SIGS = {
                       _vp], _i),
     "ic_run_stack_host": ([_vp, _vp, ctypes.POINTER(ic_layer_io), ctypes.POINTER(ic_stack_dims),
                            _vp, _vp], _i),
+    "ic_run_stack_rows": ([_vp, _vp, ctypes.POINTER(ic_layer_io), ctypes.POINTER(ic_stack_dims),
+                           ctypes.POINTER(ctypes.c_int32), _i, _vp, _vp], _i),
+    "ic_prefill_partition": ([_i, _i, _i, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(_i)], _i),
+    "ic_index_fp_rows": ([_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp], _i),
     "ic_stack_graph_create": ([_vp, _vp, ctypes.POINTER(ic_layer_io),
                                ctypes.POINTER(ic_stack_dims), _vp, ctypes.POINTER(_vp)], _i),
     "ic_stack_graph_launch": ([_vp, _vp], _i),
@@ -391,6 +395,38 @@ def ic_run_stack_host(ctx: Context, pattern: Pattern, layers_host, dims: ic_stac
         layer_array = make_stack_layers(layers_host, dims.mode)
     _check(_lib.ic_run_stack_host(ctx.handle, pattern.handle, layer_array, ctypes.byref(dims),
                                   _ptr(idx_cache), _stream(stream)), ctx)
+
+
+def ic_prefill_partition(L: int, world: int, rank: int):
+    """The rank's query-row ranges [(a0, b0), (a1, b1)] of a causal-balanced
+    split of L rows over `world` ranks (host only)."""
+    r = (ctypes.c_int32 * 4)()
+    n = _i()
+    _check(_lib.ic_prefill_partition(L, world, rank, r, ctypes.byref(n)))
+    return [(int(r[2 * i]), int(r[2 * i + 1])) for i in range(n.value)]
+
+
+def ic_index_fp_rows(ctx: Context, qI_rows, w_rows, kI, row_begin: int, row_end: int, k: int,
+                     idx_out, stream=None):
+    """F layer of rows [row_begin, row_end) with compact q_I / w rows and the
+    whole k_I [L, d_I]; idx_out int32 [row_end - row_begin, k]."""
+    n, H_I, d_I = qI_rows.shape
+    if n != row_end - row_begin:
+        raise ValueError("qI_rows must hold row_end - row_begin rows")
+    _check(_lib.ic_index_fp_rows(ctx.handle, _ptr(qI_rows), _ptr(w_rows), _ptr(kI), kI.shape[0],
+                                 H_I, d_I, row_begin, row_end, k, _ptr(idx_out), _stream(stream)),
+           ctx)
+
+
+def ic_run_stack_rows(ctx: Context, pattern: Pattern, layers, dims: ic_stack_dims, ranges,
+                      idx_cache, stream=None, layer_array=None):
+    """One rank's share of a prefill stack split by rows: `ranges` are its
+    (begin, end) row ranges; qI/w/Q/out (and idx_snapshot) of each layer hold
+    those rows only, kI/K/V all L rows."""
+    arr = layer_array if layer_array is not None else make_stack_layers(layers, dims.mode)
+    flat = (ctypes.c_int32 * (2 * len(ranges)))(*[v for ab in ranges for v in ab])
+    _check(_lib.ic_run_stack_rows(ctx.handle, pattern.handle, arr, ctypes.byref(dims), flat,
+                                  len(ranges), _ptr(idx_cache), _stream(stream)), ctx)
 
 
 class StackGraph:

@@ -222,6 +222,38 @@ int ic_index_fp_decode_noalloc(const void *q, const void *w, const uint8_t *kI8,
  * entry point it reports on, it has no counterpart on the pages. */
 int ic_noalloc_sync_status(void *stream);
 
+/* ------------------------------------------ prefill split across ranks */
+
+/* The prefill path splits by query rows: given the whole k_I, K and V, every
+ * row's scores, top-k and attention need nothing from any other row ([RN]
+ * §2.1 and §3: each query row's score row and softmax are its own; [RN]
+ * §10.3 reports the pages' prefill with data-parallel attention over 8
+ * GPUs).  A rank owns some row ranges; one all-gather of its rows of k_I, K
+ * and V (done by the caller, e.g. torch.distributed over NCCL) gives every
+ * rank the whole key tensors, and from there everything is local. */
+
+/* Causal-balanced split of L query rows over `world` ranks.  The rows are cut
+ * into 2*world chunks of near-equal size (the first L % (2*world) chunks one
+ * row longer); rank `rank` owns chunks rank and 2*world-1-rank, so each rank
+ * pairs an early, cheap chunk with a late, costly one (an F-layer row t
+ * scores t+1 keys).  Writes ranges[0..3] = {a0, b0, a1, b1} (half-open row
+ * ranges, b0 <= a1; a range is empty when L < 2*world) and *n_ranges = 2.
+ * Host only.
+ * Errors: IC_ERR_INVALID_ARG (NULL, L < 0, world < 1, rank outside). */
+int ic_prefill_partition(int L, int world, int rank, int32_t *ranges, int *n_ranges);
+
+/* One prefill F layer for the query rows [row_begin, row_end) only, with
+ * their q_I and w rows held compactly:
+ *   qI_rows: bf16 [row_end - row_begin, H_I, d_I];  w_rows: bf16 [.., H_I];
+ *   kI: bf16 [L, d_I], the whole key tensor (rows >= row_end are not read);
+ *   idx_out: int32 [row_end - row_begin, k]: row i holds T_{row_begin + i}.
+ * Results are identical to the same rows of ic_index_fp.  An empty range
+ * returns IC_OK at once.  Supported and errors as ic_index_fp, plus
+ * IC_ERR_SHAPE for a range outside [0, L). */
+int ic_index_fp_rows(ic_ctx *ctx, const void *qI_rows, const void *w_rows, const void *kI, int L,
+                     int H_I, int d_I, int row_begin, int row_end, int k, int32_t *idx_out,
+                     void *stream);
+
 /* ------------------------------------------------------ sparse attention */
 
 /* [RN] §3 sparse MQA attention, every layer:
@@ -300,6 +332,18 @@ typedef struct ic_stack_dims {
  * always complete before the stack reads anything. */
 int ic_run_stack(ic_ctx *ctx, const ic_pattern *pattern, const ic_layer_io *layers,
                  const ic_stack_dims *dims, int32_t *idx_cache, void *stream);
+
+/* The prefill stack of one rank of a row split ([IC] Figure 2 over the
+ * rank's rows).  `ranges` (HOST int32 [2*n_ranges], half-open, disjoint,
+ * e.g. from ic_prefill_partition) are the rank's query rows.  In layers[l],
+ * qI, w, Q, out and idx_snapshot hold the rank's rows only, range after
+ * range in the order given (rows = the sum of the range lengths); kI, K and
+ * V hold all dims->L rows (after the caller's all-gather).  idx_cache is
+ * int32 [rows, k].  Every output row is identical to the same row of
+ * ic_run_stack on the whole sequence.  Prefill mode only. */
+int ic_run_stack_rows(ic_ctx *ctx, const ic_pattern *pattern, const ic_layer_io *layers,
+                      const ic_stack_dims *dims, const int32_t *ranges, int n_ranges,
+                      int32_t *idx_cache, void *stream);
 
 /* A stack captured once as a CUDA graph and replayed: a decode step of
  * many small dependent kernels then costs one graph launch.  Create runs
