@@ -339,8 +339,11 @@ int ic_run_stack(ic_ctx *ctx, const ic_pattern *pattern, const ic_layer_io *laye
  * qI, w, Q, out and idx_snapshot hold the rank's rows only, range after
  * range in the order given (rows = the sum of the range lengths); kI, K and
  * V hold all dims->L rows (after the caller's all-gather).  idx_cache is
- * int32 [rows, k].  Every output row is identical to the same row of
- * ic_run_stack on the whole sequence.  Prefill mode only. */
+ * int32 [rows, k].  Every index row is identical to the same row of
+ * ic_run_stack on the whole sequence, and so is every output row unless one
+ * of the two attention launches is short enough (fewer rows than about
+ * three CTAs per SM) to spread each row over a cluster of CTAs, which rounds
+ * differently within the attention tolerance.  Prefill mode only. */
 int ic_run_stack_rows(ic_ctx *ctx, const ic_pattern *pattern, const ic_layer_io *layers,
                       const ic_stack_dims *dims, const int32_t *ranges, int n_ranges,
                       int32_t *idx_cache, void *stream);

@@ -1,16 +1,25 @@
 """The prefill split across ranks on the GPU, with the ranks run one after
 another on one device (they never wait on one another: after the
-all-gather each rank's work is local).  Every rank's rows of the indices and
-of every layer's output must equal the same rows of the one-rank stack bit
-for bit: the kernels compute each row from the same inputs in the same
-order, whichever rows share the launch.  The all-gather itself is the
-host-side plumbing checked with gloo ranks in tests/test_prefill_split.py;
-here each rank's k_I/K/V are the whole tensors it would receive."""
+all-gather each rank's work is local).
+
+Every rank's rows of the index tensors must equal the same rows of the
+one-rank stack bit for bit: the indexer and the top-k compute each row from
+the same inputs in the same order, whichever rows share the launch.  The
+same holds for the attention outputs while both launches keep one CTA per
+row.  A launch of few rows (under about three CTAs per SM) spreads each
+row's key slots over a cluster of CTAs, which rounds differently.  A rank's
+output rows are then checked against the oracle with the attention bars
+instead.
+
+The all-gather itself is the host-side plumbing checked with gloo ranks in
+tests/test_prefill_split.py.  Here each rank's k_I/K/V are the whole
+tensors it would receive."""
 import numpy as np
 import pytest
 import torch
 
 from cross_layer_top_b200 import synth
+from tests import attn_check
 
 pytestmark = pytest.mark.gpu
 
@@ -33,7 +42,7 @@ def _full_stack(ic, ctx, cfg, layers):
     return dims
 
 
-@pytest.mark.parametrize("name,world", [("tiny", 2), ("tiny", 3), ("prefill", 4)])
+@pytest.mark.parametrize("name,world", [("tiny", 2), ("tiny", 3), ("prefill", 4), ("prefill", 8)])
 def test_split_ranks_equal_one_rank_stack(ic, name, world):
     from cross_layer_top_b200 import sharding
     cfg = synth.CONFIGS[name]
@@ -55,9 +64,19 @@ def test_split_ranks_equal_one_rank_stack(ic, name, world):
         cache = torch.empty((n, k), dtype=torch.int32, device="cuda")
         ic.ic_run_stack_rows(ctx, pat, local, dims, mine, cache)
         ctx.sync_status()
+        rows = np.concatenate([np.arange(a, b) for a, b in mine]).astype(np.int32)
         for l in range(cfg.n_layers):
-            assert torch.equal(local[l]["idx_snapshot"], sharding.rows_of(layers[l]["idx_snapshot"], mine)), (rank, l)
-            assert torch.equal(local[l]["out"], sharding.rows_of(layers[l]["out"], mine)), (rank, l)
+            idx_l = local[l]["idx_snapshot"]
+            assert torch.equal(idx_l, sharding.rows_of(layers[l]["idx_snapshot"], mine)), (rank, l)
+            if torch.equal(local[l]["out"], sharding.rows_of(layers[l]["out"], mine)):
+                continue
+            assert n < 3 * torch.cuda.get_device_properties(0).multi_processor_count, (rank, l)
+            sel = np.arange(n) if n <= 256 else np.linspace(0, n - 1, 64).astype(np.int64)
+            f = synth.bf16_to_f32_numpy
+            attn_check.check(local[l]["out"].float().cpu().numpy()[sel],
+                             f(layers[l]["Q"]), f(layers[l]["K"]), f(layers[l]["V"]),
+                             idx_l.cpu().numpy()[sel], rows=rows[sel],
+                             what="rank %d layer %d" % (rank, l))
         for a, b in mine:
             covered[a:b] = True
     assert covered.all()
