@@ -178,6 +178,7 @@ extern "C" int ic_ctx_destroy(ic_ctx* ctx) {
     cudaSetDevice(ctx->device);
     cudaDeviceSynchronize();
     cudaFree(ctx->scores);
+    cudaFree(ctx->hist);
     cudaFree(ctx->dev_err);
     if (ctx->hs.ready) {
         for (int i = 0; i < ic_ctx::kHostSlots; ++i) {
@@ -555,10 +556,31 @@ extern "C" int ic_index_fp_decode(ic_ctx* ctx, const void* q, const void* w, con
                        static_cast<size_t>(B) * ld * 4);
     if (rc) return rc;
     cudaStream_t s = as_stream(stream);
+    // When the top-k takes the cluster form, the scan also counts each
+    // sequence's scores by the top-k's first radix digit, so the top-k knows
+    // its threshold bin before it reads a score.
+    uint32_t* hist = nullptr;
+    if (topk_uses_cluster(ctx, B, true, S_max)) {
+        const size_t bytes = static_cast<size_t>(B) * 2048 * sizeof(uint32_t);
+        if (ctx->hist_cap < bytes || ctx->hist == nullptr) {
+            rc = ensure_buffer(ctx, reinterpret_cast<void**>(&ctx->hist), &ctx->hist_cap, bytes);
+            if (rc) return rc;
+            ctx->hist_dirty = true;
+        }
+        if (ctx->hist_dirty) {
+            cudaError_t e = cudaMemsetAsync(ctx->hist, 0, ctx->hist_cap, s);
+            if (e != cudaSuccess) return cuda_fail(ctx, e, "decode index: clear histograms");
+            ctx->hist_dirty = false;
+        }
+        hist = ctx->hist;
+    }
+    if (hist) ctx->hist_dirty = true;  // until the top-k that clears it is enqueued
     rc = launch_index_score_decode(ctx, q, w, kI8, kI_scale, seq_len, B, S_max, H_I, d_I,
-                                   ctx->scores, ld, s);
+                                   ctx->scores, ld, s, hist);
     if (rc) return rc;
-    return launch_topk(ctx, ctx->scores, ld, B, k, 0, seq_len, S_max, idx_out, k, s);
+    rc = launch_topk(ctx, ctx->scores, ld, B, k, 0, seq_len, S_max, idx_out, k, s, hist);
+    if (rc == IC_OK) ctx->hist_dirty = false;
+    return rc;
 }
 
 // ------------------------------------------------------ sparse attention

@@ -286,6 +286,19 @@ __device__ __forceinline__ void griddep_launch_dependents() {
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 }
 
+// ------------------------------------------------------- order keys
+// An fp32 score as an unsigned key with the same order (the top-k compares
+// and bins keys; the decode scan bins the scores it writes by the same key).
+__device__ __forceinline__ uint32_t order_key(float x) {
+    // x + (+0.0) turns -0.0 into +0.0 and leaves every other value as it is
+    const uint32_t b = __float_as_uint(__fadd_rn(x, 0.0f));
+    // negative: all bits flipped; non-negative: the sign bit set
+    return b ^ (static_cast<uint32_t>(static_cast<int32_t>(b) >> 31) | 0x80000000u);
+}
+// The top-k's first radix digit: the key's top 11 bits (2048 bins).
+constexpr int kKeyBins = 2048;
+constexpr int kKeyBinShift = 21;
+
 // ------------------------------------------------------- cp.async / ldmatrix
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, bool valid) {
     // src-size 0 fills the 16 bytes with zeros and reads nothing

@@ -19,6 +19,13 @@ struct ic_ctx {
     size_t scratch_limit = 0;       // bound on the prefill score scratch (bytes)
     float* scores = nullptr;        // score scratch (fp32 rows)
     size_t scores_cap = 0;          // bytes
+    // decode: per-sequence first-digit histograms of the scores ([B][2048]
+    // uint32), written by the scan and read (then cleared) by the cluster
+    // top-k; zero between uses, `hist_dirty` when a use may have stopped
+    // between the two launches
+    uint32_t* hist = nullptr;
+    size_t hist_cap = 0;            // bytes
+    bool hist_dirty = false;
     int* dev_err = nullptr;         // device error word (first error wins)
     std::string last_error;
     bool timing = false;
@@ -145,12 +152,20 @@ int check_stack_args(ic_ctx* ctx, const ic_pattern* pattern, const void* layers,
 int launch_index_score_prefill(ic_ctx* ctx, const void* qI, const void* kI, const void* w, int L,
                                int H_I, int d_I, int row_begin, int row_end, float* scores,
                                int64_t ld, cudaStream_t stream, int q_row0 = 0, int q_rows = -1);
+// hist (optional, zero on entry): [B][2048] counts of the written scores
+// by the top 11 bits of their order key, for launch_topk
 int launch_index_score_decode(ic_ctx* ctx, const void* q, const void* w, const uint8_t* kI8,
                               const float* kI_scale, const int32_t* seq_len, int B, int S_max,
-                              int H_I, int d_I, float* scores, int64_t ld, cudaStream_t stream);
+                              int H_I, int d_I, float* scores, int64_t ld, cudaStream_t stream,
+                              uint32_t* hist = nullptr);
+// Whether launch_topk takes the cluster form (a thread-block cluster per row)
+// for these rows; only that form uses a precomputed histogram.
+bool topk_uses_cluster(const ic_ctx* ctx, int rows, bool has_row_len, int max_len);
+// hist (optional, cluster form only): the rows' first-digit histograms from
+// launch_index_score_decode; read, then cleared to zero for the next use
 int launch_topk(ic_ctx* ctx, const float* scores, int64_t ld, int rows, int k, int causal_base,
                 const int32_t* row_len, int max_len, int32_t* idx_out, int64_t ld_out,
-                cudaStream_t stream);
+                cudaStream_t stream, uint32_t* hist = nullptr);
 int launch_index_score_prefill_fp8(ic_ctx* ctx, const uint8_t* qI8, const float* q_scale,
                                    const uint8_t* kI8, const float* k_scale, const void* w, int L,
                                    int H_I, int d_I, int row_begin, int row_end, float* scores,

@@ -34,6 +34,13 @@
 //    scale, and stores I[b,s].
 // Each CTA scans a contiguous range of (sequence, key tile) pairs.  All
 // waits are bounded.
+// When asked (hist != NULL) the epilogue also counts the scores it stores
+// per sequence into 2048 bins by the top 11 bits of their order key, the
+// first radix digit of the top-k that follows: hist[b][bin] += count.  The
+// counts of the CTA's first and last sequence gather in shared memory and
+// go out with one atomic add per nonzero bin at the end; a sequence in
+// between, which only this CTA touches, is counted straight into hist.
+// hist must be zero before the launch (the top-k clears it after use).
 #include "ic_device.cuh"
 #include "ic_internal.h"
 
@@ -58,13 +65,15 @@ struct DecodeShape {
     static constexpr int SC_RING = 8;       // scale prefetch depth (tiles)
     static constexpr int SC_BYTES = SC_RING * BM * 4;
     static constexpr int QRED_BYTES = 32;   // [2][4] warp maxima of |q|
+    static constexpr int HIST_BYTES = 2 * kKeyBins * 4;  // first / last sequence's counts
     static constexpr int BAR_BYTES = 512;
     static constexpr int OFF_A = 0;
     static constexpr int OFF_B = OFF_A + A_ST * A_BYTES;
     static constexpr int OFF_W = OFF_B + 2 * B_BUF;
     static constexpr int OFF_SC = OFF_W + W_BYTES;
     static constexpr int OFF_QRED = OFF_SC + SC_BYTES;
-    static constexpr int OFF_BAR = OFF_QRED + QRED_BYTES;
+    static constexpr int OFF_HIST = OFF_QRED + QRED_BYTES;
+    static constexpr int OFF_BAR = OFF_HIST + HIST_BYTES;
     static constexpr int SMEM = OFF_BAR + BAR_BYTES;
     static_assert(SMEM <= 232448, "shared memory budget");
     static_assert(NACC >= 2, "TMEM allocation");
@@ -142,7 +151,7 @@ __global__ void __launch_bounds__(512, 1)
                          const __nv_bfloat16* __restrict__ qg, const __nv_bfloat16* __restrict__ w,
                          const float* __restrict__ kscale, const int32_t* __restrict__ seq_len,
                          int B, int S_max, int tps, float* __restrict__ scores, long long ld,
-                         int* __restrict__ err) {
+                         uint32_t* __restrict__ hist, int* __restrict__ err) {
     using S = DecodeShape<H_I>;
     extern __shared__ __align__(1024) uint8_t smem[];
     uint8_t* sA = smem + S::OFF_A;
@@ -158,6 +167,7 @@ __global__ void __launch_bounds__(512, 1)
     uint64_t* done_bar = q_max + 1;
     uint32_t* qred = reinterpret_cast<uint32_t*>(smem + S::OFF_QRED);  // [2][4]
     uint8_t* seq_ring = smem + S::OFF_W;
+    uint32_t* sh_hist = reinterpret_cast<uint32_t*>(smem + S::OFF_HIST);  // [2][kKeyBins]
     uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
     volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -198,6 +208,8 @@ __global__ void __launch_bounds__(512, 1)
         tmem_alloc(tmem_slot, S::TMEM_COLS);
         tmem_relinquish();
     }
+    if (hist != nullptr)
+        for (int i = threadIdx.x; i < 2 * kKeyBins; i += blockDim.x) sh_hist[i] = 0;
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -385,6 +397,11 @@ __global__ void __launch_bounds__(512, 1)
         TileWalk<S::BM> tw, tp;
         tw.init(g_begin, g_end, tps, seq_len, S_max);
         tp.init(g_begin, g_end, tps, seq_len, S_max);
+        // the sequences of this CTA's first and last (sequence, tile) pair:
+        // their score counts gather in shared memory (the others are this
+        // CTA's alone and go straight to hist)
+        const int b_first = static_cast<int>(g_begin / tps);
+        const int b_last = g_end > g_begin ? static_cast<int>((g_end - 1) / tps) : b_first;
         auto prefetch_scale = [&](int slot) {
             if (!tp.done()) {
                 const int s = tp.j * S::BM + key;
@@ -465,14 +482,33 @@ __global__ void __launch_bounds__(512, 1)
             asm volatile("ld.shared.f32 %0, [%1];"
                          : "=f"(sc)
                          : "r"(sc_ring + (it % S::SC_RING) * S::BM * 4));
-            if (s < n)
-                scores[static_cast<long long>(b) * ld + s] =
-                    (sc * q_unscale) * ((p[0] + p[1]) + (p[2] + p[3]));
+            const float val = (sc * q_unscale) * ((p[0] + p[1]) + (p[2] + p[3]));
+            if (s < n) scores[static_cast<long long>(b) * ld + s] = val;
+            if (hist != nullptr && s < n) {
+                // b is the same for the whole tile: the slot is chosen once
+                const uint32_t bin = order_key(val) >> kKeyBinShift;
+                if (b == b_first || b == b_last)
+                    atomicAdd(&sh_hist[(b == b_first ? 0 : kKeyBins) + bin], 1u);
+                else
+                    atomicAdd(&hist[static_cast<long long>(b) * kKeyBins + bin], 1u);
+            }
             acc_ph ^= 1u << acc;
             if (++acc == S::NACC) acc = 0;
             ++it;
         }
         cp_async_wait<0>();  // no prefetch may still be landing at exit
+        if (hist != nullptr) {
+            // every epilogue warp leaves the tile loop (also on an abort) and
+            // meets here; then the shared counts go out, one add per bin
+            asm volatile("bar.sync 1, %0;" ::"n"(256) : "memory");
+            const int et = threadIdx.x - 256;  // 0..255
+            for (int i = et; i < 2 * kKeyBins; i += 256) {
+                const uint32_t c = sh_hist[i];
+                const int bb = i < kKeyBins ? b_first : b_last;
+                if (c != 0 && !(i >= kKeyBins && b_last == b_first))
+                    atomicAdd(&hist[static_cast<long long>(bb) * kKeyBins + (i % kKeyBins)], c);
+            }
+        }
     }
 
     tc_fence_before();
@@ -486,7 +522,7 @@ __global__ void __launch_bounds__(512, 1)
 template <int H_I>
 static int launch_decode_t(ic_ctx* ctx, const void* q, const void* w, const uint8_t* kI8,
                            const float* kI_scale, const int32_t* seq_len, int B, int S_max,
-                           float* scores, int64_t ld, cudaStream_t stream) {
+                           float* scores, int64_t ld, uint32_t* hist, cudaStream_t stream) {
     using S = DecodeShape<H_I>;
     static PerDeviceOnce attr_once;
     cudaError_t ea = attr_once.run(ctx->device, [] {
@@ -518,7 +554,7 @@ static int launch_decode_t(ic_ctx* ctx, const void* q, const void* w, const uint
     LaunchScope ls(ctx, IC_K_INDEX_SCORE_DECODE, stream);
     cudaLaunchKernelEx(&cfg, k_index_score_decode<H_I>, tm_k, static_cast<const __nv_bfloat16*>(q),
                        static_cast<const __nv_bfloat16*>(w), kI_scale, seq_len, B, S_max, tps,
-                       scores, static_cast<long long>(ld), ctx->dev_err);
+                       scores, static_cast<long long>(ld), hist, ctx->dev_err);
     cudaError_t e = ls.done();
     if (e != cudaSuccess) return cuda_fail(ctx, e, "index_score_decode launch");
     return IC_OK;
@@ -526,12 +562,15 @@ static int launch_decode_t(ic_ctx* ctx, const void* q, const void* w, const uint
 
 int launch_index_score_decode(ic_ctx* ctx, const void* q, const void* w, const uint8_t* kI8,
                               const float* kI_scale, const int32_t* seq_len, int B, int S_max,
-                              int H_I, int d_I, float* scores, int64_t ld, cudaStream_t stream) {
+                              int H_I, int d_I, float* scores, int64_t ld, cudaStream_t stream,
+                              uint32_t* hist) {
     if (d_I != 128) return fail(ctx, IC_ERR_UNSUPPORTED, "decode index: d_I=%d (need 128)", d_I);
     if (H_I == 64)
-        return launch_decode_t<64>(ctx, q, w, kI8, kI_scale, seq_len, B, S_max, scores, ld, stream);
+        return launch_decode_t<64>(ctx, q, w, kI8, kI_scale, seq_len, B, S_max, scores, ld, hist,
+                                   stream);
     if (H_I == 32)
-        return launch_decode_t<32>(ctx, q, w, kI8, kI_scale, seq_len, B, S_max, scores, ld, stream);
+        return launch_decode_t<32>(ctx, q, w, kI8, kI_scale, seq_len, B, S_max, scores, ld, hist,
+                                   stream);
     return fail(ctx, IC_ERR_UNSUPPORTED, "decode index: H_I=%d (need 32 or 64)", H_I);
 }
 

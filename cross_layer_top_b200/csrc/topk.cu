@@ -38,12 +38,6 @@ constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kCandCap = 4096;
 constexpr int kBitmapCap = 131072;  // longest row (keys) with a shared selection bitmap
 
-__device__ __forceinline__ uint32_t order_key(float x) {
-    // x + (+0.0) turns -0.0 into +0.0 and leaves every other value as it is
-    const uint32_t b = __float_as_uint(__fadd_rn(x, 0.0f));
-    // negative: all bits flipped; non-negative: the sign bit set
-    return b ^ (static_cast<uint32_t>(static_cast<int32_t>(b) >> 31) | 0x80000000u);
-}
 // inverse of order_key (up to the sign of zero)
 __device__ __forceinline__ float key_float(uint32_t u) {
     return __uint_as_float((u & 0x80000000u) ? (u & 0x7fffffffu) : ~u);
@@ -59,21 +53,22 @@ struct alignas(16) TopkShared {
     uint32_t wcand[kTopkWarps];  // bitmap path: candidates in each warp's slice
     uint32_t bin;
     uint32_t above;
+    uint32_t bin_count;  // keys in `bin`
 };
 
 // Find the bin b (of nbins, 512 threads owning nbins/512 consecutive bins
 // each) such that count(bins > b) < krem <= count(bins >= b).  Writes the
 // bin and count(bins > b) to S.bin / S.above.  Must be called by all threads.
+// The same with this thread's counts of bins tid*PER .. tid*PER+PER-1
+// already in registers; also writes the found bin's count to S.bin_count.
 template <int NB>
-__device__ __forceinline__ void find_bin(TopkShared& S, uint32_t krem, const uint32_t* hist) {
+__device__ __forceinline__ void find_bin_counts(TopkShared& S, uint32_t krem,
+                                                const uint32_t (&c)[NB / kTopkThreads]) {
     constexpr int PER = NB / kTopkThreads;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    uint32_t c[PER], tot = 0;
+    uint32_t tot = 0;
 #pragma unroll
-    for (int b = 0; b < PER; ++b) {
-        c[b] = hist[tid * PER + b];
-        tot += c[b];
-    }
+    for (int b = 0; b < PER; ++b) tot += c[b];
     // inclusive suffix sum within the warp (higher lanes hold higher bins)
     uint32_t suf = tot;
 #pragma unroll
@@ -102,12 +97,21 @@ __device__ __forceinline__ void find_bin(TopkShared& S, uint32_t krem, const uin
             if (acc + c[b] >= krem) {
                 S.bin = tid * PER + b;
                 S.above = acc;
+                S.bin_count = c[b];
                 break;
             }
             acc += c[b];
         }
     }
     __syncthreads();
+}
+template <int NB>
+__device__ __forceinline__ void find_bin(TopkShared& S, uint32_t krem, const uint32_t* hist) {
+    constexpr int PER = NB / kTopkThreads;
+    uint32_t c[PER];
+#pragma unroll
+    for (int b = 0; b < PER; ++b) c[b] = hist[threadIdx.x * PER + b];
+    find_bin_counts<NB>(S, krem, c);
 }
 template <int NB>
 __device__ __forceinline__ void find_bin(TopkShared& S, uint32_t krem) {
@@ -376,7 +380,8 @@ static_assert(offsetof(TopkClusterShared, hist_all) % 16 == 0, "16-byte stores o
 __global__ void __launch_bounds__(kTopkThreads)
     k_topk_cluster(const float* __restrict__ scores, long long ld, int k,
                    const int32_t* __restrict__ row_len, int max_len, int causal_base,
-                   int32_t* __restrict__ out, long long ld_out, int seg_cap) {
+                   int32_t* __restrict__ out, long long ld_out, int seg_cap,
+                   uint32_t* __restrict__ ghist) {
     // dynamic shared memory: the staged segment, then the merged candidates
     extern __shared__ uint32_t srow[];
     uint32_t* cand_all = srow + seg_cap;
@@ -390,22 +395,33 @@ __global__ void __launch_bounds__(kTopkThreads)
     griddep_launch_dependents();
     const int n = row_len ? min(row_len[r], max_len) : causal_base + r + 1;
     int32_t* o = out + static_cast<long long>(r) * ld_out;
+    // the row's first-digit histogram from the scan, if given; CTA 0 clears
+    // it once every CTA of the cluster is past reading it
+    uint32_t* gh = ghist ? ghist + static_cast<long long>(r) * kKeyBins : nullptr;
+    auto clear_hist = [&]() {
+        if (gh != nullptr && rank == 0)
+            for (int i = tid; i < kKeyBins; i += kTopkThreads) gh[i] = 0u;
+    };
     if (n <= k) {  // the same for every CTA of the cluster: no cluster barrier is reached
         if (rank == 0)
             for (int i = tid; i < k; i += kTopkThreads) o[i] = i < n ? i : -1;
+        clear_hist();
         return;
     }
-    // every CTA arrives on the cluster barrier now and waits on it before its
-    // first remote store, by when the whole cluster is known to be running
-    cluster_arrive_relaxed();
+    // With the histogram: the bin b1 of the k-th largest key and how many
+    // keys it holds are known before the row is read.  If they fit the
+    // candidate list (the same answer in every CTA), each CTA stages its
+    // segment and collects the keys of bin b1 in one pass, and the radix
+    // passes start at the second digit; otherwise the path below.
     const int seg = ((n + kClusterCtas - 1) / kClusterCtas + 3) / 4 * 4;
     const int s0 = min(n, static_cast<int>(rank) * seg), s1 = min(n, s0 + seg);
     const int m = s1 - s0;  // this CTA's segment length
     const float* row = scores + static_cast<long long>(r) * ld + s0;
-
-    // ---- A: stage the segment, cluster-wide key range
-    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
-    {
+    // this segment as order keys in shared memory; returns the segment's
+    // key range (the path without a histogram needs it)
+    auto stage = [&](uint32_t& kmin, uint32_t& kmax) {
+        kmin = 0xFFFFFFFFu;
+        kmax = 0u;
         const int m4 = m >> 2;
         const float4* row4 = reinterpret_cast<const float4*>(row);
         for (int i = tid; i < m4; i += kTopkThreads) {
@@ -422,39 +438,68 @@ __global__ void __launch_bounds__(kTopkThreads)
             kmin = min(kmin, u);
             kmax = max(kmax, u);
         }
-    }
-    kmin = __reduce_min_sync(0xffffffffu, kmin);
-    kmax = __reduce_max_sync(0xffffffffu, kmax);
-    if (lane == 0) {
-        S.wcnt[0][warp] = kmin;
-        S.wcnt[1][warp] = kmax;
-    }
-    for (int i = tid; i < 2048; i += kTopkThreads) S.hist[i] = 0;
-    if (tid == 0) S.ncand = 0;
-    __syncthreads();
-    cluster_wait_acquire();  // every CTA of the cluster is running
-    // thread q stores this segment's range into CTA q's slot `rank`
-    if (tid < kClusterCtas) {
-        uint32_t a = 0xFFFFFFFFu, b = 0u;
-        for (int w = 0; w < kTopkWarps; ++w) {
-            a = min(a, S.wcnt[0][w]);
-            b = max(b, S.wcnt[1][w]);
-        }
-        dsmem_st_u32(dsmem_addr(&CS.rng_min[rank], tid), a);
-        dsmem_st_u32(dsmem_addr(&CS.rng_max[rank], tid), b);
-    }
-    cluster_sync_all();  // every segment's range is in every CTA
-    kmin = 0xFFFFFFFFu;
-    kmax = 0u;
+    };
+    // The histogram's counts are loaded before the segment, so that their
+    // round trip overlaps the staging reads.
+    bool fast = false;
+    uint32_t fb1 = 0, fkrem = 0;
+    uint32_t kmin = 0xFFFFFFFFu, kmax = 0u;
+    if (gh != nullptr) {
+        uint32_t c[4];
 #pragma unroll
-    for (int q = 0; q < kClusterCtas; ++q) {
-        kmin = min(kmin, CS.rng_min[q]);
-        kmax = max(kmax, CS.rng_max[q]);
+        for (int b = 0; b < 4; ++b) c[b] = gh[tid * 4 + b];
+        stage(kmin, kmax);
+        if (tid == 0) {  // defined even if the counts were not the row's (find_bin orders this)
+            S.bin = 0;
+            S.above = 0;
+            S.bin_count = 0xFFFFFFFFu;
+        }
+        find_bin_counts<2048>(S, static_cast<uint32_t>(k), c);
+        fb1 = S.bin;
+        fkrem = static_cast<uint32_t>(k) - S.above;
+        fast = S.bin_count <= static_cast<uint32_t>(kCandCap);  // the same in every CTA
+        __syncthreads();  // S.bin / S.above are rewritten below
     }
-    const float xmin = key_float(kmin), xmax = key_float(kmax);
-    const float span = xmax - xmin;
-    const float inv = 2047.0f / span;
-    const bool by_value = span > 0.f && isfinite(span) && isfinite(inv) && inv > 0.f;
+    // every CTA's candidate count, then its candidates at the running offset:
+    // 4 per 16-byte remote load, each round's loads (one per CTA) issued
+    // before any is stored; returns the merged count
+    auto merge_candidates = [&]() {
+        int nq[kClusterCtas], off[kClusterCtas], total = 0;
+#pragma unroll
+        for (uint32_t q = 0; q < kClusterCtas; ++q) nq[q] = static_cast<int>(dsmem_ld(dsmem_addr(&S.ncand, q)));
+#pragma unroll
+        for (uint32_t q = 0; q < kClusterCtas; ++q) {
+            nq[q] = min(nq[q], kCandCap - total);  // never past the merged list
+            off[q] = total;
+            total += nq[q];
+        }
+        for (int i4 = 4 * tid; i4 < kCandCap; i4 += 4 * kTopkThreads) {
+            uint4 cv[kClusterCtas];
+#pragma unroll
+            for (uint32_t q = 0; q < kClusterCtas; ++q)
+                if (i4 < nq[q]) cv[q] = dsmem_ld_u4(dsmem_addr(&S.cand[i4], q));
+#pragma unroll
+            for (uint32_t q = 0; q < kClusterCtas; ++q) {
+                const uint32_t c4[4] = {cv[q].x, cv[q].y, cv[q].z, cv[q].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                    if (i4 + e < nq[q]) cand_all[off[q] + i4 + e] = c4[e];
+            }
+        }
+        // No CTA rewrites its S.ncand or S.cand after this, so other CTAs may
+        // still be reading them: only this CTA's merged list must be complete.
+        __syncthreads();
+        return total;
+    };
+    uint32_t prefix = 0, mask = 0, krem = 0;
+    bool use_cand = true;
+    int ncand = 0, first_pass = 0;
+    // The path without a histogram bins keys uniformly in value between the
+    // row's minimum and maximum (monotone in the key, so exact), or by their
+    // top 11 bits when that range is degenerate.
+    float xmin = 0.f, inv = 0.f;
+    bool by_value = false;
+    uint32_t b1 = 0;
     auto bin_of = [&](uint32_t u) -> uint32_t {
         if (!by_value) return u >> 21;
         return static_cast<uint32_t>(fminf((key_float(u) - xmin) * inv, 2047.0f));
@@ -482,59 +527,93 @@ __global__ void __launch_bounds__(kTopkThreads)
         *reinterpret_cast<uint4*>(&CS.hist_all[4 * tid]) = t;
         if (rewrite_next) cluster_sync_all();  // nobody rewrites a histogram another CTA still reads
     };
+    if (fast) {
+        if (tid == 0) S.ncand = 0;
+        __syncthreads();
+        for (int i = tid; i < m; i += kTopkThreads) {
+            const uint32_t u = srow[i];
+            if ((u >> kKeyBinShift) == fb1) {
+                // the counts bound the list; the check only keeps counts that
+                // do not belong to these scores from writing past it
+                const uint32_t slot = atomicAdd(&S.ncand, 1u);
+                if (slot < static_cast<uint32_t>(kCandCap)) S.cand[slot] = u;
+            }
+        }
+        // every CTA of the cluster is running and has its candidates, and
+        // has read the histogram
+        cluster_sync_all();
+        clear_hist();
+        ncand = merge_candidates();
+        prefix = fb1 << kKeyBinShift;
+        mask = 0x7FFu << kKeyBinShift;
+        krem = fkrem;
+        first_pass = 1;
+    } else {
+    // every CTA arrives on the cluster barrier now and waits on it before its
+    // first remote store, by when the whole cluster is known to be running
+    cluster_arrive_relaxed();
+
+    // ---- A: stage the segment (unless done above), cluster-wide key range
+    if (gh == nullptr) stage(kmin, kmax);
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    if (lane == 0) {
+        S.wcnt[0][warp] = kmin;
+        S.wcnt[1][warp] = kmax;
+    }
+    for (int i = tid; i < 2048; i += kTopkThreads) S.hist[i] = 0;
+    if (tid == 0) S.ncand = 0;
+    __syncthreads();
+    cluster_wait_acquire();  // every CTA of the cluster is running
+    clear_hist();            // ... and past reading the histogram
+    // thread q stores this segment's range into CTA q's slot `rank`
+    if (tid < kClusterCtas) {
+        uint32_t a = 0xFFFFFFFFu, b = 0u;
+        for (int w = 0; w < kTopkWarps; ++w) {
+            a = min(a, S.wcnt[0][w]);
+            b = max(b, S.wcnt[1][w]);
+        }
+        dsmem_st_u32(dsmem_addr(&CS.rng_min[rank], tid), a);
+        dsmem_st_u32(dsmem_addr(&CS.rng_max[rank], tid), b);
+    }
+    cluster_sync_all();  // every segment's range is in every CTA
+    kmin = 0xFFFFFFFFu;
+    kmax = 0u;
+#pragma unroll
+    for (int q = 0; q < kClusterCtas; ++q) {
+        kmin = min(kmin, CS.rng_min[q]);
+        kmax = max(kmax, CS.rng_max[q]);
+    }
+    xmin = key_float(kmin);
+    const float span = key_float(kmax) - xmin;
+    inv = 2047.0f / span;
+    by_value = span > 0.f && isfinite(span) && isfinite(inv) && inv > 0.f;
     for (int i = tid; i < m; i += kTopkThreads) atomicAdd(&S.hist[bin_of(srow[i])], 1u);
     cluster_hist(false);
     find_bin<2048>(S, static_cast<uint32_t>(k), CS.hist_all);
-    const uint32_t b1 = S.bin;
-    uint32_t krem = static_cast<uint32_t>(k) - S.above;
+    b1 = S.bin;
+    krem = static_cast<uint32_t>(k) - S.above;
     const uint32_t in_bin = CS.hist_all[b1];
     __syncthreads();
 
     // ---- B: candidates of bin b1 from every segment, or (massive ties)
     // cluster-wide radix passes over the bin's keys
-    const bool use_cand = in_bin <= static_cast<uint32_t>(kCandCap);  // the same in every CTA
+    use_cand = in_bin <= static_cast<uint32_t>(kCandCap);  // the same in every CTA
     // The radix passes rewrite S.hist.  With candidates, the barrier after
     // they are collected keeps every CTA's reads of the histograms above
     // ahead of that; without, this one does.
     if (!use_cand) cluster_sync_all();
-    int ncand = 0;
     if (use_cand) {
         for (int i = tid; i < m; i += kTopkThreads) {
             const uint32_t u = srow[i];
             if (bin_of(u) == b1) S.cand[atomicAdd(&S.ncand, 1u)] = u;
         }
         cluster_sync_all();
-        // every CTA's candidate count, then its candidates at the running
-        // offset: 4 per 16-byte remote load, each round's loads (one per CTA)
-        // issued before any is stored
-        int nq[kClusterCtas], off[kClusterCtas];
-#pragma unroll
-        for (uint32_t q = 0; q < kClusterCtas; ++q) nq[q] = static_cast<int>(dsmem_ld(dsmem_addr(&S.ncand, q)));
-#pragma unroll
-        for (uint32_t q = 0; q < kClusterCtas; ++q) {
-            off[q] = ncand;
-            ncand += nq[q];
-        }
-        for (int i4 = 4 * tid; i4 < kCandCap; i4 += 4 * kTopkThreads) {
-            uint4 cv[kClusterCtas];
-#pragma unroll
-            for (uint32_t q = 0; q < kClusterCtas; ++q)
-                if (i4 < nq[q]) cv[q] = dsmem_ld_u4(dsmem_addr(&S.cand[i4], q));
-#pragma unroll
-            for (uint32_t q = 0; q < kClusterCtas; ++q) {
-                const uint32_t c4[4] = {cv[q].x, cv[q].y, cv[q].z, cv[q].w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    if (i4 + e < nq[q]) cand_all[off[q] + i4 + e] = c4[e];
-            }
-        }
-        // No CTA rewrites its S.ncand or S.cand after this, so other CTAs may
-        // still be reading them: only this CTA's merged list must be complete.
-        __syncthreads();
+        ncand = merge_candidates();
     }
-    uint32_t prefix = 0, mask = 0;
+    }  // the path without a histogram (or with too many keys in its bin)
 #pragma unroll 1
-    for (int pass = 0; pass < 3; ++pass) {
+    for (int pass = first_pass; pass < 3; ++pass) {
         const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
         const uint32_t dmask = pass == 2 ? 0x3FFu : 0x7FFu;
         for (int i = tid; i < 2048; i += kTopkThreads) S.hist[i] = 0;
@@ -617,10 +696,10 @@ __global__ void __launch_bounds__(kTopkThreads)
         const unsigned be = __ballot_sync(0xffffffffu, eq);
         const uint32_t g_before = G + __popc(bg & lt);
         const uint32_t e_before = E + __popc(be & lt);
-        if (gt)
-            o[g_before + (e_before < krem ? e_before : krem)] = s0 + i;
-        else if (eq && e_before < krem)
-            o[g_before + e_before] = s0 + i;
+        // positions stay below k whenever T and krem are the row's; the
+        // bound only guards the output against counts that were not
+        const uint32_t pos = gt ? g_before + (e_before < krem ? e_before : krem) : g_before + e_before;
+        if ((gt || (eq && e_before < krem)) && pos < static_cast<uint32_t>(k)) o[pos] = s0 + i;
         G += __popc(bg);
         E += __popc(be);
     }
@@ -628,7 +707,8 @@ __global__ void __launch_bounds__(kTopkThreads)
 
 static int launch_topk_cluster(ic_ctx* ctx, const float* scores, int64_t ld, int rows, int k,
                                int causal_base, const int32_t* row_len, int max_len,
-                               int32_t* idx_out, int64_t ld_out, cudaStream_t stream) {
+                               int32_t* idx_out, int64_t ld_out, cudaStream_t stream,
+                               uint32_t* hist) {
     const int seg_cap = ((max_len + kClusterCtas - 1) / kClusterCtas + 3) / 4 * 4;
     const int smem = (seg_cap + kCandCap) * 4;
     cudaError_t e = cudaFuncSetAttribute(k_topk_cluster, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -650,21 +730,29 @@ static int launch_topk_cluster(ic_ctx* ctx, const float* scores, int64_t ld, int
     cfg.numAttrs = na;
     LaunchScope ls(ctx, IC_K_TOPK, stream);
     cudaLaunchKernelEx(&cfg, k_topk_cluster, scores, static_cast<long long>(ld), k, row_len,
-                       max_len, causal_base, idx_out, static_cast<long long>(ld_out), seg_cap);
+                       max_len, causal_base, idx_out, static_cast<long long>(ld_out), seg_cap,
+                       hist);
     e = ls.done();
     if (e != cudaSuccess) return cuda_fail(ctx, e, "topk_cluster launch");
     return IC_OK;
 }
 
+bool topk_uses_cluster(const ic_ctx* ctx, int rows, bool has_row_len, int max_len) {
+    // few long rows (decode): a cluster of CTAs per row keeps many SMs busy
+    return has_row_len && rows > 0 &&
+           static_cast<long long>(rows) * kClusterCtas <= 4LL * ctx->num_sms && max_len > 16384 &&
+           max_len <= kClusterCtas * 45000;
+}
+
 int launch_topk(ic_ctx* ctx, const float* scores, int64_t ld, int rows, int k, int causal_base,
                 const int32_t* row_len, int max_len, int32_t* idx_out, int64_t ld_out,
-                cudaStream_t stream) {
+                cudaStream_t stream, uint32_t* hist) {
     if (rows <= 0) return IC_OK;
-    // Few long rows (decode): a cluster of CTAs per row keeps many SMs busy.
-    if (row_len != nullptr && static_cast<long long>(rows) * kClusterCtas <= 4LL * ctx->num_sms &&
-        max_len > 16384 && max_len <= kClusterCtas * 45000)
+    if (topk_uses_cluster(ctx, rows, row_len != nullptr, max_len))
         return launch_topk_cluster(ctx, scores, ld, rows, k, causal_base, row_len, max_len, idx_out,
-                                   ld_out, stream);
+                                   ld_out, stream, hist);
+    if (hist != nullptr)
+        return fail(ctx, IC_ERR_INVALID_ARG, "topk: a histogram is only used by the cluster form");
     static PerDeviceOnce attr_once;
     cudaError_t ea = attr_once.run(ctx->device, [] {
         return cudaFuncSetAttribute(k_topk, cudaFuncAttributeMaxDynamicSharedMemorySize,

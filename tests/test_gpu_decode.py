@@ -138,6 +138,49 @@ def test_decode_index_selected_set(ic, ctx):
             assert ref[sel].min() >= kth - SEL_RTOL * abs(kth)
 
 
+def _first_digit_bin_count(score64, k):
+    """How many of a row's fp32 scores share the top 11 bits of the order key
+    (sign-adjusted bits, -0.0 as +0.0) with its k-th largest score: the
+    size of the top-k's threshold bin on the first radix digit."""
+    x = (score64.astype(np.float32) + np.float32(0.0)).view(np.uint32)
+    key = np.where(x >> 31 == 1, ~x, x | np.uint32(0x80000000)).astype(np.uint32)
+    kth = np.sort(key)[::-1][k - 1]
+    return int(np.sum((key >> 21) == (kth >> 21)))
+
+
+def test_decode_index_histogram_paths_bit_exact(ic, ctx):
+    """The decode F layer with the scan's first-digit histograms (cluster
+    top-k): rows whose threshold bin fits the candidate list, rows whose bin
+    overflows it (massive ties: a zero query gives all-zero scores), rows of
+    at most k candidates, in one launch and again in a second call with the
+    roles swapped (the histograms must be clear between calls).  Integer
+    inputs make the scores exact, so every row must equal the oracle's
+    top-k bit for bit (ties to the lower index)."""
+    B, S_max, k = 6, 70001, 2048
+    lens = [70001, 2048, 60000, 70001, 1, 50001]
+    q, w, k8, sc, lens_t = _decode_inputs(B, S_max, 64, 21, lens=lens, integer=True)
+    calls = []
+    q1 = q.clone()
+    q1[3] = 0  # row 3: every score 0
+    calls.append(q1)
+    q2 = q.clone()
+    q2[0] = 0  # second call: row 0 tied instead, row 3 spread out
+    calls.append(q2)
+    kinds = set()
+    for qc in calls:
+        idx = torch.full((B, k), -7, dtype=torch.int32, device="cuda")
+        ic.ic_index_fp_decode(ctx, qc.cuda(), w.cuda(), k8.cuda(), sc.cuda(), lens_t.cuda(), k, idx)
+        ctx.sync_status()
+        got = idx.cpu().numpy()
+        for b in range(B):
+            n = lens[b]
+            ref = oracle.decode_scores(f32(qc[b]), f32(w[b]), k8[b].numpy(), sc[b].numpy(), S=n)
+            assert got[b].tolist() == oracle.topk_row(ref, k).tolist(), b
+            if n > k:
+                kinds.add("fits" if _first_digit_bin_count(ref, k) <= 4096 else "overflows")
+    assert kinds == {"fits", "overflows"}
+
+
 def test_decode_workload_sampled(ic, ctx):
     """Decode workload shapes (32 sequences x 65537 candidates, H_I=64,
     k=2048): one F layer, 6 sequences checked against the oracle."""
