@@ -460,6 +460,82 @@ def run_split(args, rank, world, local_rank):
     ctx.close()
 
 
+PROFILE_KERNELS = ("index_score", "topk", "sparse_attn", "fp_decode", "sparse_attn_decode")
+
+
+def run_profile_kernel(args, local_rank):
+    """--profile-kernel NAME: a small harness for ncu captures.  It allocates
+    only what one kernel of the stack needs, at the workload's size (a few
+    GB at most), runs --warmup launches, then --steps launches, and exits:
+      index_score         prefill indexer scores, rows [k, L) of one F layer
+      topk                prefill top-k of those rows (scores made once first)
+      sparse_attn         prefill attention of one layer (indices made once first)
+      fp_decode           decode F layer (FP8 scan with its first-digit
+                          histograms, then the cluster top-k), 32 x 65537
+      sparse_attn_decode  decode attention of one layer, 32 x 65537
+    Prints one JSON line with the average time per launch (CUDA events)."""
+    from cross_layer_top_b200 import indexcache as ic
+    from cross_layer_top_b200 import synth
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    ctx = ic.Context(local_rank)
+    name = args.profile_kernel
+    if name in ("index_score", "topk", "sparse_attn"):
+        cfg = synth.CONFIGS[WORKLOAD]
+        L, k = cfg.L, cfg.k
+        lay = synth.prefill_layer(cfg, 0, dev)
+        ld = (L + 63) // 64 * 64
+        if name == "sparse_attn":
+            idx = torch.empty((L, k), dtype=torch.int32, device=dev)
+            ic.ic_index_fp(ctx, lay["qI"], lay["kI"], lay["w"], k, idx)
+            out = torch.empty((L, cfg.Hq, cfg.d), dtype=torch.bfloat16, device=dev)
+            for m in ("qI", "kI", "w"):
+                del lay[m]
+            run = lambda: ic.ic_sparse_attn(ctx, lay["Q"], lay["K"], lay["V"], idx, out)
+        else:
+            scores = torch.empty((L - k, ld), dtype=torch.float32, device=dev)
+            score = lambda: ic.ic_index_score(ctx, lay["qI"], lay["kI"], lay["w"], k, L, scores, ld)
+            if name == "index_score":
+                run = score
+            else:
+                score()
+                for m in ("qI", "kI", "w", "Q", "K", "V"):
+                    del lay[m]
+                idx = torch.empty((L - k, k), dtype=torch.int32, device=dev)
+                run = lambda: ic.ic_topk(ctx, scores, k, idx, causal_base=k, ld=ld)
+    elif name in ("fp_decode", "sparse_attn_decode"):
+        cfg = synth.CONFIGS["decode"]
+        B, S, k = cfg.B, cfg.S, cfg.k
+        lay = synth.decode_layer(cfg, 0, dev)
+        idx = torch.empty((B, k), dtype=torch.int32, device=dev)
+        fp = lambda: ic.ic_index_fp_decode(ctx, lay["q"], lay["w"], lay["kI8"], lay["kI_scale"],
+                                           lay["seq_len"], k, idx)
+        if name == "fp_decode":
+            run = fp
+        else:
+            fp()
+            out = torch.empty((B, cfg.Hq, cfg.d), dtype=torch.bfloat16, device=dev)
+            run = lambda: ic.ic_sparse_attn(ctx, lay["Q"], lay["K"], lay["V"], idx, out,
+                                            rows_per_seq=1, kv_seq_stride=S * cfg.d, kv_len=S)
+    else:
+        raise SystemExit("--profile-kernel: one of %s" % ", ".join(PROFILE_KERNELS))
+    ctx.sync_status()
+    for _ in range(args.warmup):
+        run()
+    ctx.sync_status()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record()
+    for _ in range(args.steps):
+        run()
+    b.record()
+    b.synchronize()
+    ctx.sync_status()
+    print(json.dumps({"profile_kernel": name, "launches": args.steps,
+                      "ms_per_call": a.elapsed_time(b) / max(1, args.steps),
+                      "gpu_mem_gb": round(torch.cuda.max_memory_allocated() / 1e9, 2)}), flush=True)
+    ctx.close()
+
+
 def run_e2e(args, ctx, pat, dims, cfg, layers, cache, world, pairs_step, stream):
     """Same metric through the library's host-memory entry point
     (ic_run_stack_host): every step copies all layer inputs host->device from
@@ -945,18 +1021,23 @@ def main():
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the decode workload (not the contract line)")
     ap.add_argument("--decode-layers", type=int, default=0)
+    ap.add_argument("--profile-kernel", default=None, choices=PROFILE_KERNELS,
+                    help="harness for ncu captures: only this kernel's inputs, then exit")
     ap.add_argument("--prefill-split", action="store_true",
                     help="one prefill sequence split over the ranks by query rows (strong "
                          "scaling, an all-gather of k_I/K/V per step) instead of one sequence "
                          "per rank")
     args = ap.parse_args()
-    if args.warmup < 3 and args.impl == "ours":
+    if args.warmup < 3 and args.impl == "ours" and not args.profile_kernel:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))
     local_rank = int(os.environ.get("LOCAL_RANK", 0))
     if args.impl == "reference":
         run_reference(args, rank, world)
+        return
+    if args.profile_kernel:
+        run_profile_kernel(args, local_rank)
         return
     if args.decode_only:
         torch.cuda.set_device(local_rank)
