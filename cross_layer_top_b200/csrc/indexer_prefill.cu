@@ -66,10 +66,9 @@ struct PrefillShape {
     static_assert(!F8 || NATOM == 1, "e4m3 rows of d_I = 128 are one 128-byte atom");
 };
 
-// Score 64 consecutive accumulator columns held in va (cols 0..31) and vb
-// (cols 32..63); wcol points at the fp32 weights of those 64 columns
-// (token-major, head-minor, same order as the columns).  Produces one score
-// per token covered (64 / H_I tokens).
+// The scoring kernel (one persistent CTA per SM, warp roles as above):
+// scores of query rows [row_begin, row_end) against keys s <= t, written to
+// scores[(t - row_begin) * ld + s].
 template <int H_I, int NATOM, bool F8>
 __global__ void __launch_bounds__(PrefillShape<H_I, NATOM, F8>::THREADS, 1)
     k_index_score_prefill(const __grid_constant__ CUtensorMap tm_q,
