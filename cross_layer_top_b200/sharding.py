@@ -38,6 +38,13 @@ def allgather_rows(local: torch.Tensor, ranges_all, L: int, group=None) -> torch
     local: this rank's rows (ranges_all[rank], range after range).  All ranks
     call this with the same ranges_all, in the same order.  Returns the whole
     [L, ...] tensor on local's device."""
+    if len(ranges_all) == 1:  # one rank: its rows are every row, in order
+        full = local.new_empty((L,) + tuple(local.shape[1:]))
+        off = 0
+        for a, b in ranges_all[0]:
+            full[a:b] = local[off:off + b - a]
+            off += b - a
+        return full
     counts = [sum(b - a for a, b in rr) for rr in ranges_all]
     cmax = max(counts)
     send = local
