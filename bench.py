@@ -56,57 +56,115 @@ def scored_pairs(L, k, n_f):
 
 # ----------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi sampling (200 ms) while the timed region runs."""
+    """SM clock and clock-event reasons of one GPU, sampled every 20 ms by
+    NVML in a thread (read-only queries), kept only while the timed region
+    runs (mark_start / mark_stop); falls back to nvidia-smi at 200 ms when
+    NVML is unavailable."""
 
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, device_index):
         self.dev = device_index
+        self.samples = []  # (sm_mhz, set of reasons)
+        self.smax = None
+        self.in_region = False
+        self.stop_flag = False
         self.proc = None
-        self.lines = []
+        self.nvml = None
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:  # the CUDA device's own board, when torch reports its PCI bus id
+            bus = torch.cuda.get_device_properties(self.dev).pci_bus_id
+            h = pynvml.nvmlDeviceGetHandleByPciBusId(
+                "%08x:%02x:%02x.0" % (torch.cuda.get_device_properties(self.dev).pci_domain_id,
+                                      bus, torch.cuda.get_device_properties(self.dev).pci_device_id))
+        except Exception:
+            vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+            idx = int(vis.split(",")[self.dev]) if vis and vis.split(",")[0].isdigit() else self.dev
+            h = pynvml.nvmlDeviceGetHandleByIndex(idx)
+        return pynvml, h
 
     def start(self):
+        try:
+            pynvml, h = self._nvml_handle()
+            self.smax = float(pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM))
+            masks = [(n, getattr(pynvml, a)) for n, a in self.REASONS]
+
+            def run():
+                while not self.stop_flag:
+                    if self.in_region:
+                        try:
+                            mhz = float(pynvml.nvmlDeviceGetClockInfo(h, pynvml.NVML_CLOCK_SM))
+                            r = pynvml.nvmlDeviceGetCurrentClocksEventReasons(h)
+                            self.samples.append((mhz, {n for n, m in masks if r & m}))
+                        except Exception:
+                            pass
+                    time.sleep(0.02)
+
+            self.thread = threading.Thread(target=run, daemon=True)
+            self.thread.start()
+            self.nvml = pynvml
+            self.source = "nvml, 20 ms"
+            return
+        except Exception:
+            self.nvml = None
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.dev), "--query-gpu=" + self.FIELDS,
                  "--format=csv,noheader,nounits", "-lms", "200"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread = threading.Thread(target=self._read_smi, daemon=True)
             self.thread.start()
+            self.source = "nvidia-smi, 200 ms"
         except Exception:
             self.proc = None
 
-    def _read(self):
+    def _read_smi(self):
+        names = [n for n, _ in self.REASONS]
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
-
-    def stop(self):
-        if self.proc is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
-        self.proc.terminate()
-        try:
-            self.proc.wait(timeout=5)
-        except Exception:
-            self.proc.kill()
-        self.thread.join(timeout=2)
-        sm, smax, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) < 9:
+            parts = [p.strip() for p in line.strip().split(",")]
+            if len(parts) < 9 or not self.in_region:
                 continue
             try:
-                sm.append(float(parts[1]))
-                smax = float(parts[2])
+                mhz, self.smax = float(parts[1]), float(parts[2])
             except ValueError:
                 continue
-            for n, v in zip(names, parts[5:9]):
-                if v.lower().startswith("active"):
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+            self.samples.append((mhz, {n for n, v in zip(names, parts[5:9])
+                                       if v.lower().startswith("active")}))
+
+    def mark_start(self):
+        self.in_region = True
+
+    def mark_stop(self):
+        self.in_region = False
+
+    def stop(self):
+        self.in_region = False
+        self.stop_flag = True
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+        if self.nvml is None and self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["clock sampling unavailable"]}
+        self.thread.join(timeout=2)
+        sm = [m for m, _ in self.samples]
+        reasons = set()
+        for _, r in self.samples:
+            reasons |= r
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.smax,
+                "reasons": sorted(reasons), "samples": len(sm), "source": self.source}
 
 
 # ------------------------------------------------------------- our arm
@@ -144,11 +202,10 @@ def run_ours(args, rank, world, local_rank):
     def step():
         ic.ic_run_stack(ctx, pat, None, dims, cache, layer_array=arr)
 
-    # the clock sampler starts before the warm-up so that it is producing
-    # samples (under load) by the time the timed region begins
+    # the clock sampler starts before the warm-up; it keeps only the samples
+    # taken while the timed steps run
     clocks = ClockSampler(local_rank)
     clocks.start()
-    time.sleep(0.3)
     for _ in range(args.warmup):
         step()
     ctx.sync_status()
@@ -163,12 +220,14 @@ def run_ours(args, rank, world, local_rank):
           for _ in range(args.steps)]
     dist_barrier(world)
     torch.cuda.synchronize()
+    clocks.mark_start()
     for i in range(args.steps):
         flush.fill_(float(i))  # L2 flush, outside the timed events
         ev[i][0].record(stream)
         step()
         ev[i][1].record(stream)
     torch.cuda.synchronize()
+    clocks.mark_stop()
     dist_barrier(world)
     clk = clocks.stop()
     ctx.set_timing(False)
