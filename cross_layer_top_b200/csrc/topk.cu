@@ -549,68 +549,68 @@ __global__ void __launch_bounds__(kTopkThreads)
         krem = fkrem;
         first_pass = 1;
     } else {
-    // every CTA arrives on the cluster barrier now and waits on it before its
-    // first remote store, by when the whole cluster is known to be running
-    cluster_arrive_relaxed();
+        // every CTA arrives on the cluster barrier now and waits on it before its
+        // first remote store, by when the whole cluster is known to be running
+        cluster_arrive_relaxed();
 
-    // ---- A: stage the segment (unless done above), cluster-wide key range
-    if (gh == nullptr) stage(kmin, kmax);
-    kmin = __reduce_min_sync(0xffffffffu, kmin);
-    kmax = __reduce_max_sync(0xffffffffu, kmax);
-    if (lane == 0) {
-        S.wcnt[0][warp] = kmin;
-        S.wcnt[1][warp] = kmax;
-    }
-    for (int i = tid; i < 2048; i += kTopkThreads) S.hist[i] = 0;
-    if (tid == 0) S.ncand = 0;
-    __syncthreads();
-    cluster_wait_acquire();  // every CTA of the cluster is running
-    clear_hist();            // ... and past reading the histogram
-    // thread q stores this segment's range into CTA q's slot `rank`
-    if (tid < kClusterCtas) {
-        uint32_t a = 0xFFFFFFFFu, b = 0u;
-        for (int w = 0; w < kTopkWarps; ++w) {
-            a = min(a, S.wcnt[0][w]);
-            b = max(b, S.wcnt[1][w]);
+        // ---- A: stage the segment (unless done above), cluster-wide key range
+        if (gh == nullptr) stage(kmin, kmax);
+        kmin = __reduce_min_sync(0xffffffffu, kmin);
+        kmax = __reduce_max_sync(0xffffffffu, kmax);
+        if (lane == 0) {
+            S.wcnt[0][warp] = kmin;
+            S.wcnt[1][warp] = kmax;
         }
-        dsmem_st_u32(dsmem_addr(&CS.rng_min[rank], tid), a);
-        dsmem_st_u32(dsmem_addr(&CS.rng_max[rank], tid), b);
-    }
-    cluster_sync_all();  // every segment's range is in every CTA
-    kmin = 0xFFFFFFFFu;
-    kmax = 0u;
+        for (int i = tid; i < 2048; i += kTopkThreads) S.hist[i] = 0;
+        if (tid == 0) S.ncand = 0;
+        __syncthreads();
+        cluster_wait_acquire();  // every CTA of the cluster is running
+        clear_hist();            // ... and past reading the histogram
+        // thread q stores this segment's range into CTA q's slot `rank`
+        if (tid < kClusterCtas) {
+            uint32_t a = 0xFFFFFFFFu, b = 0u;
+            for (int w = 0; w < kTopkWarps; ++w) {
+                a = min(a, S.wcnt[0][w]);
+                b = max(b, S.wcnt[1][w]);
+            }
+            dsmem_st_u32(dsmem_addr(&CS.rng_min[rank], tid), a);
+            dsmem_st_u32(dsmem_addr(&CS.rng_max[rank], tid), b);
+        }
+        cluster_sync_all();  // every segment's range is in every CTA
+        kmin = 0xFFFFFFFFu;
+        kmax = 0u;
 #pragma unroll
-    for (int q = 0; q < kClusterCtas; ++q) {
-        kmin = min(kmin, CS.rng_min[q]);
-        kmax = max(kmax, CS.rng_max[q]);
-    }
-    xmin = key_float(kmin);
-    const float span = key_float(kmax) - xmin;
-    inv = 2047.0f / span;
-    by_value = span > 0.f && isfinite(span) && isfinite(inv) && inv > 0.f;
-    for (int i = tid; i < m; i += kTopkThreads) atomicAdd(&S.hist[bin_of(srow[i])], 1u);
-    cluster_hist(false);
-    find_bin<2048>(S, static_cast<uint32_t>(k), CS.hist_all);
-    b1 = S.bin;
-    krem = static_cast<uint32_t>(k) - S.above;
-    const uint32_t in_bin = CS.hist_all[b1];
-    __syncthreads();
-
-    // ---- B: candidates of bin b1 from every segment, or (massive ties)
-    // cluster-wide radix passes over the bin's keys
-    use_cand = in_bin <= static_cast<uint32_t>(kCandCap);  // the same in every CTA
-    // The radix passes rewrite S.hist.  With candidates, the barrier after
-    // they are collected keeps every CTA's reads of the histograms above
-    // ahead of that; without, this one does.
-    if (!use_cand) cluster_sync_all();
-    if (use_cand) {
-        for (int i = tid; i < m; i += kTopkThreads) {
-            const uint32_t u = srow[i];
-            if (bin_of(u) == b1) S.cand[atomicAdd(&S.ncand, 1u)] = u;
+        for (int q = 0; q < kClusterCtas; ++q) {
+            kmin = min(kmin, CS.rng_min[q]);
+            kmax = max(kmax, CS.rng_max[q]);
         }
-        cluster_sync_all();
-        ncand = merge_candidates();
-    }
+        xmin = key_float(kmin);
+        const float span = key_float(kmax) - xmin;
+        inv = 2047.0f / span;
+        by_value = span > 0.f && isfinite(span) && isfinite(inv) && inv > 0.f;
+        for (int i = tid; i < m; i += kTopkThreads) atomicAdd(&S.hist[bin_of(srow[i])], 1u);
+        cluster_hist(false);
+        find_bin<2048>(S, static_cast<uint32_t>(k), CS.hist_all);
+        b1 = S.bin;
+        krem = static_cast<uint32_t>(k) - S.above;
+        const uint32_t in_bin = CS.hist_all[b1];
+        __syncthreads();
+
+        // ---- B: candidates of bin b1 from every segment, or (massive ties)
+        // cluster-wide radix passes over the bin's keys
+        use_cand = in_bin <= static_cast<uint32_t>(kCandCap);  // the same in every CTA
+        // The radix passes rewrite S.hist.  With candidates, the barrier after
+        // they are collected keeps every CTA's reads of the histograms above
+        // ahead of that; without, this one does.
+        if (!use_cand) cluster_sync_all();
+        if (use_cand) {
+            for (int i = tid; i < m; i += kTopkThreads) {
+                const uint32_t u = srow[i];
+                if (bin_of(u) == b1) S.cand[atomicAdd(&S.ncand, 1u)] = u;
+            }
+            cluster_sync_all();
+            ncand = merge_candidates();
+        }
     }  // the path without a histogram (or with too many keys in its bin)
 #pragma unroll 1
     for (int pass = first_pass; pass < 3; ++pass) {
