@@ -424,14 +424,23 @@ __global__ void __launch_bounds__(kTopkThreads)
         kmax = 0u;
         const int m4 = m >> 2;
         const float4* row4 = reinterpret_cast<const float4*>(row);
-        for (int i = tid; i < m4; i += kTopkThreads) {
-            const float4 v = __ldg(row4 + i);
+        auto put = [&](int i, const float4& v) {
             const uint32_t u0 = order_key(v.x), u1 = order_key(v.y);
             const uint32_t u2 = order_key(v.z), u3 = order_key(v.w);
             *reinterpret_cast<uint4*>(srow + 4 * i) = make_uint4(u0, u1, u2, u3);
             kmin = min(kmin, min(min(u0, u1), min(u2, u3)));
             kmax = max(kmax, max(max(u0, u1), max(u2, u3)));
+        };
+        // four 16-byte loads in flight per thread before any is used
+        int i = tid;
+        for (; i + 3 * kTopkThreads < m4; i += 4 * kTopkThreads) {
+            float4 v[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) v[q] = __ldg(row4 + i + q * kTopkThreads);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) put(i + q * kTopkThreads, v[q]);
         }
+        for (; i < m4; i += kTopkThreads) put(i, __ldg(row4 + i));
         for (int i = 4 * m4 + tid; i < m; i += kTopkThreads) {
             const uint32_t u = order_key(__ldg(row + i));
             srow[i] = u;
@@ -530,13 +539,19 @@ __global__ void __launch_bounds__(kTopkThreads)
     if (fast) {
         if (tid == 0) S.ncand = 0;
         __syncthreads();
-        for (int i = tid; i < m; i += kTopkThreads) {
-            const uint32_t u = srow[i];
-            if ((u >> kKeyBinShift) == fb1) {
-                // the counts bound the list; the check only keeps counts that
-                // do not belong to these scores from writing past it
-                const uint32_t slot = atomicAdd(&S.ncand, 1u);
-                if (slot < static_cast<uint32_t>(kCandCap)) S.cand[slot] = u;
+        // four staged keys per 16-byte load (the staged segment's storage is
+        // a multiple of 4 keys; keys past m are not the row's)
+        for (int i4 = tid; 4 * i4 < m; i4 += kTopkThreads) {
+            const uint4 v = *reinterpret_cast<const uint4*>(srow + 4 * i4);
+            const uint32_t u4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                if (4 * i4 + j < m && (u4[j] >> kKeyBinShift) == fb1) {
+                    // the counts bound the list; the check only keeps counts
+                    // that do not belong to these scores from writing past it
+                    const uint32_t slot = atomicAdd(&S.ncand, 1u);
+                    if (slot < static_cast<uint32_t>(kCandCap)) S.cand[slot] = u4[j];
+                }
             }
         }
         // every CTA of the cluster is running and has its candidates, and
@@ -644,17 +659,34 @@ __global__ void __launch_bounds__(kTopkThreads)
     }
     const uint32_t T = prefix;
 
-    // ---- C: counts of this segment, offsets from the segments before it
-    const int wseg = ((m + kTopkWarps - 1) / kTopkWarps + 31) / 32 * 32;
+    // ---- C: counts of this segment, offsets from the segments before it.
+    // Each warp walks a contiguous part of the segment in blocks of 128 keys,
+    // lane l taking keys 4l .. 4l+3 of a block with one 16-byte load (the
+    // staged segment's storage is a multiple of 4 keys).
+    const int wseg = ((m + kTopkWarps - 1) / kTopkWarps + 127) / 128 * 128;
     const int sb = warp * wseg, se = min(m, sb + wseg);
+    auto load4 = [&](int i0, uint32_t (&u4)[4]) {
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (i0 < se) v = *reinterpret_cast<const uint4*>(srow + i0);
+        u4[0] = v.x;
+        u4[1] = v.y;
+        u4[2] = v.z;
+        u4[3] = v.w;
+    };
     uint32_t cg = 0, ce = 0;
-    for (int base = sb; base < se; base += 32) {
-        const int i = base + lane;
-        const bool in = i < se;
-        const uint32_t u = in ? srow[i] : 0u;
-        cg += __popc(__ballot_sync(0xffffffffu, in && u > T));
-        ce += __popc(__ballot_sync(0xffffffffu, in && u == T));
+    for (int base = sb; base < se; base += 128) {
+        const int i0 = base + 4 * lane;
+        uint32_t u4[4];
+        load4(i0, u4);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const bool in = i0 + j < se;
+            cg += (in && u4[j] > T) ? 1u : 0u;
+            ce += (in && u4[j] == T) ? 1u : 0u;
+        }
     }
+    cg = __reduce_add_sync(0xffffffffu, cg);
+    ce = __reduce_add_sync(0xffffffffu, ce);
     if (lane == 0) {
         S.wcnt[0][warp] = cg;
         S.wcnt[1][warp] = ce;
@@ -687,21 +719,37 @@ __global__ void __launch_bounds__(kTopkThreads)
             E += S.wcnt[1][w];
         }
     const unsigned lt = (1u << lane) - 1u;
-    for (int base = sb; base < se; base += 32) {
-        const int i = base + lane;
-        const bool in = i < se;
-        const uint32_t u = in ? srow[i] : 0u;
-        const bool gt = in && u > T, eq = in && u == T;
-        const unsigned bg = __ballot_sync(0xffffffffu, gt);
-        const unsigned be = __ballot_sync(0xffffffffu, eq);
-        const uint32_t g_before = G + __popc(bg & lt);
-        const uint32_t e_before = E + __popc(be & lt);
-        // positions stay below k whenever T and krem are the row's; the
-        // bound only guards the output against counts that were not
-        const uint32_t pos = gt ? g_before + (e_before < krem ? e_before : krem) : g_before + e_before;
-        if ((gt || (eq && e_before < krem)) && pos < static_cast<uint32_t>(k)) o[pos] = s0 + i;
-        G += __popc(bg);
-        E += __popc(be);
+    for (int base = sb; base < se; base += 128) {
+        const int i0 = base + 4 * lane;
+        uint32_t u4[4];
+        load4(i0, u4);
+        bool gt[4], eq[4];
+        unsigned bg[4], be[4];
+        uint32_t g_before = G, e_before = E;  // keys > T and == T before this lane's first
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const bool in = i0 + j < se;
+            gt[j] = in && u4[j] > T;
+            eq[j] = in && u4[j] == T;
+            bg[j] = __ballot_sync(0xffffffffu, gt[j]);
+            be[j] = __ballot_sync(0xffffffffu, eq[j]);
+            g_before += __popc(bg[j] & lt);
+            e_before += __popc(be[j] & lt);
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const uint32_t pos =
+                gt[j] ? g_before + (e_before < krem ? e_before : krem) : g_before + e_before;
+            if ((gt[j] || (eq[j] && e_before < krem)) && pos < static_cast<uint32_t>(k))
+                o[pos] = s0 + i0 + j;
+            g_before += gt[j] ? 1u : 0u;
+            e_before += eq[j] ? 1u : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            G += __popc(bg[j]);
+            E += __popc(be[j]);
+        }
     }
 }
 
