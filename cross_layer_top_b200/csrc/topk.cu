@@ -6,7 +6,8 @@
 // in ascending position order, ties going to the lower position, followed
 // by -1 padding.  -0.0 and +0.0 compare equal.
 //
-// Algorithm (one 512-thread CTA per row), on order-preserving uint32 keys:
+// Algorithm (one CTA per row: 8 warps for rows up to 32768 keys, 16 warps
+// beyond), on order-preserving uint32 keys:
 //  A. one pass over the row: a 2048-bin histogram of the keys' top 11 bits;
 //     the bin b1 holding the k-th largest key is found by a block suffix
 //     scan;
@@ -33,9 +34,19 @@
 
 namespace ic {
 
+// cluster variant: 16 warps per CTA, 4096 candidate slots
 constexpr int kTopkThreads = 512;
 constexpr int kTopkWarps = kTopkThreads / 32;
 constexpr int kCandCap = 4096;
+// single-CTA row kernel, two shapes:
+//  - rows up to kShortRow keys: 8 warps per CTA and 2048 candidate slots, so
+//    eight CTAs share an SM at 16K keys (measured on one prefill F layer's
+//    14336 rows: 0.379 ms against 0.411 ms with the long-row shape; 8 warps
+//    with 4096 slots and four CTAs per SM gained nothing);
+//  - longer rows: 16 warps and 4096 slots.  On Gaussian scores the bin of
+//    the k-th largest key holds about 2170 keys at 131072 keys, which the
+//    short-row list would send to the general path.
+constexpr int kShortRow = 32768;
 constexpr int kBitmapCap = 131072;  // longest row (keys) with a shared selection bitmap
 
 // inverse of order_key (up to the sign of zero)
@@ -44,27 +55,32 @@ __device__ __forceinline__ float key_float(uint32_t u) {
 }
 
 // hist and cand are read with 16-byte (remote) loads in the cluster variant
-struct alignas(16) TopkShared {
+template <int WARPS, int CAND>
+struct alignas(16) TopkSharedT {
+    static constexpr int kWarps = WARPS;
     alignas(16) uint32_t hist[2048];
-    alignas(16) uint32_t cand[kCandCap];
-    uint32_t wsum[kTopkWarps];
-    uint32_t wcnt[2][kTopkWarps];
+    alignas(16) uint32_t cand[CAND];
+    uint32_t wsum[WARPS];
+    uint32_t wcnt[2][WARPS];
     uint32_t ncand;
-    uint32_t wcand[kTopkWarps];  // bitmap path: candidates in each warp's slice
+    uint32_t wcand[WARPS];  // bitmap path: candidates in each warp's slice
     uint32_t bin;
     uint32_t above;
     uint32_t bin_count;  // keys in `bin`
 };
+using TopkShared = TopkSharedT<kTopkWarps, kCandCap>;
 
-// Find the bin b (of nbins, 512 threads owning nbins/512 consecutive bins
-// each) such that count(bins > b) < krem <= count(bins >= b).  Writes the
-// bin and count(bins > b) to S.bin / S.above.  Must be called by all threads.
-// The same with this thread's counts of bins tid*PER .. tid*PER+PER-1
-// already in registers; also writes the found bin's count to S.bin_count.
-template <int NB>
-__device__ __forceinline__ void find_bin_counts(TopkShared& S, uint32_t krem,
-                                                const uint32_t (&c)[NB / kTopkThreads]) {
-    constexpr int PER = NB / kTopkThreads;
+// Find the bin b (of NB, the CTA's threads owning NB / threads consecutive
+// bins each) such that count(bins > b) < krem <= count(bins >= b).  Writes
+// the bin and count(bins > b) to S.bin / S.above.  Must be called by all
+// threads.  This form takes the thread's counts of bins tid*PER ..
+// tid*PER+PER-1 in registers and also writes the found bin's count to
+// S.bin_count.
+template <int NB, class SH>
+__device__ __forceinline__ void find_bin_counts(SH& S, uint32_t krem,
+                                                const uint32_t (&c)[NB / (SH::kWarps * 32)]) {
+    constexpr int WARPS = SH::kWarps;
+    constexpr int PER = NB / (WARPS * 32);
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     uint32_t tot = 0;
 #pragma unroll
@@ -81,11 +97,11 @@ __device__ __forceinline__ void find_bin_counts(TopkShared& S, uint32_t krem,
     // keys in the warps above this one: a suffix scan of the warp totals
     // across lanes (lane w ends with the keys in warps >= w; lanes past the
     // last warp hold 0)
-    uint32_t ws = lane < kTopkWarps ? S.wsum[lane] : 0u;
+    uint32_t ws = lane < WARPS ? S.wsum[lane] : 0u;
 #pragma unroll
-    for (int off = 1; off < kTopkWarps; off <<= 1) {
+    for (int off = 1; off < WARPS; off <<= 1) {
         const uint32_t v = __shfl_down_sync(0xffffffffu, ws, off);
-        if (lane + off < kTopkWarps) ws += v;
+        if (lane + off < WARPS) ws += v;
     }
     const uint32_t higher = __shfl_sync(0xffffffffu, ws, warp + 1);
     const uint32_t incl = suf + higher;       // keys in bins >= my first bin
@@ -105,27 +121,29 @@ __device__ __forceinline__ void find_bin_counts(TopkShared& S, uint32_t krem,
     }
     __syncthreads();
 }
-template <int NB>
-__device__ __forceinline__ void find_bin(TopkShared& S, uint32_t krem, const uint32_t* hist) {
-    constexpr int PER = NB / kTopkThreads;
+template <int NB, class SH>
+__device__ __forceinline__ void find_bin(SH& S, uint32_t krem, const uint32_t* hist) {
+    constexpr int PER = NB / (SH::kWarps * 32);
     uint32_t c[PER];
 #pragma unroll
     for (int b = 0; b < PER; ++b) c[b] = hist[threadIdx.x * PER + b];
     find_bin_counts<NB>(S, krem, c);
 }
-template <int NB>
-__device__ __forceinline__ void find_bin(TopkShared& S, uint32_t krem) {
+template <int NB, class SH>
+__device__ __forceinline__ void find_bin(SH& S, uint32_t krem) {
     find_bin<NB>(S, krem, S.hist);
 }
 
-__global__ void __launch_bounds__(kTopkThreads)
+template <int kRowThreads, int kRowCandCap, int kRowMinCtas>
+__global__ void __launch_bounds__(kRowThreads, kRowMinCtas)
     k_topk(const float* __restrict__ scores, long long ld, int k, int causal_base,
            const int32_t* __restrict__ row_len, int max_len, int32_t* __restrict__ out,
            long long ld_out, int bcap) {
-    // dynamic shared memory: the candidates' positions [kCandCap], then the
+    // dynamic shared memory: the candidates' positions [kRowCandCap], then the
     // selection bitmap of rows up to bcap keys [bcap / 32]
     extern __shared__ uint32_t dsm[];
-    __shared__ TopkShared S;
+    constexpr int kRowWarps = kRowThreads / 32;
+    __shared__ TopkSharedT<kRowWarps, kRowCandCap> S;
 
     const int r = blockIdx.x;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -136,19 +154,19 @@ __global__ void __launch_bounds__(kTopkThreads)
     const int n = row_len ? min(row_len[r], max_len) : causal_base + r + 1;
     int32_t* o = out + static_cast<long long>(r) * ld_out;
     if (n <= k) {
-        for (int i = tid; i < k; i += kTopkThreads) o[i] = i < n ? i : -1;
+        for (int i = tid; i < k; i += kRowThreads) o[i] = i < n ? i : -1;
         return;
     }
     const float* row = scores + static_cast<long long>(r) * ld;
     auto key_at = [&](int i) -> uint32_t { return order_key(__ldg(row + i)); };
     // ---- A: keys + histogram of the top 11 bits
-    for (int i = tid; i < 2048; i += kTopkThreads) S.hist[i] = 0;
+    for (int i = tid; i < 2048; i += kRowThreads) S.hist[i] = 0;
     if (tid == 0) S.ncand = 0;
     __syncthreads();
     {
         const int n4 = n >> 2;
         const float4* row4 = reinterpret_cast<const float4*>(row);
-        for (int i = tid; i < n4; i += kTopkThreads) {
+        for (int i = tid; i < n4; i += kRowThreads) {
             const float4 v = __ldg(row4 + i);
             const uint32_t u0 = order_key(v.x), u1 = order_key(v.y);
             const uint32_t u2 = order_key(v.z), u3 = order_key(v.w);
@@ -157,7 +175,7 @@ __global__ void __launch_bounds__(kTopkThreads)
             atomicAdd(&S.hist[u2 >> 21], 1u);
             atomicAdd(&S.hist[u3 >> 21], 1u);
         }
-        for (int i = 4 * n4 + tid; i < n; i += kTopkThreads) {
+        for (int i = 4 * n4 + tid; i < n; i += kRowThreads) {
             const uint32_t u = order_key(__ldg(row + i));
             atomicAdd(&S.hist[u >> 21], 1u);
         }
@@ -171,14 +189,14 @@ __global__ void __launch_bounds__(kTopkThreads)
 
     // ---- B: resolve bits 20..10 and 9..0 within bin b1
     uint32_t prefix = b1 << 21, mask = 0xFFE00000u;
-    const bool use_cand = in_bin <= static_cast<uint32_t>(kCandCap);
+    const bool use_cand = in_bin <= static_cast<uint32_t>(kRowCandCap);
     // warp segments, whole 128-key blocks (a warp's float4 load of 4 keys per lane)
-    const int seg = ((n + kTopkWarps - 1) / kTopkWarps + 127) / 128 * 128;
+    const int seg = ((n + kRowWarps - 1) / kRowWarps + 127) / 128 * 128;
     const int sb = warp * seg, se = min(n, sb + seg);
     const unsigned lt = (1u << lane) - 1u;
     uint32_t* cpos = dsm;
-    uint32_t* bits = cpos + kCandCap;
-    constexpr int kSlice = kCandCap / kTopkWarps;  // candidate slots per warp
+    uint32_t* bits = cpos + kRowCandCap;
+    constexpr int kSlice = kRowCandCap / kRowWarps;  // candidate slots per warp
     bool sliced = false;  // candidates in per-warp slices of the list, bitmap path
     if (use_cand && n <= bcap) {
         // one pass over the warp's segment: the keys above bin b1 (selected
@@ -234,11 +252,11 @@ __global__ void __launch_bounds__(kTopkThreads)
         __syncthreads();
         bool over = false;  // a slice overflowed: take the general path
 #pragma unroll
-        for (int w = 0; w < kTopkWarps; ++w) over |= S.wcand[w] > static_cast<uint32_t>(kSlice);
+        for (int w = 0; w < kRowWarps; ++w) over |= S.wcand[w] > static_cast<uint32_t>(kSlice);
         sliced = !over;
     }
     if (use_cand && !sliced) {
-        for (int i = tid; i < n; i += kTopkThreads) {
+        for (int i = tid; i < n; i += kRowThreads) {
             const uint32_t u = key_at(i);
             if ((u >> 21) == b1) S.cand[atomicAdd(&S.ncand, 1u)] = u;
         }
@@ -248,12 +266,12 @@ __global__ void __launch_bounds__(kTopkThreads)
     // sliced: each warp walks its own slice; otherwise the threads stride the list (or row)
     const int c0 = sliced ? warp * kSlice + lane : tid;
     const int c1 = sliced ? warp * kSlice + static_cast<int>(S.wcand[warp]) : ncand;
-    const int cstep = sliced ? 32 : kTopkThreads;
+    const int cstep = sliced ? 32 : kRowThreads;
 #pragma unroll 1
     for (int pass = 0; pass < 2; ++pass) {
         const int shift = pass == 0 ? 10 : 0;
         const uint32_t dmask = pass == 0 ? 0x7FFu : 0x3FFu;
-        for (int i = tid; i < 2048; i += kTopkThreads) S.hist[i] = 0;
+        for (int i = tid; i < 2048; i += kRowThreads) S.hist[i] = 0;
         __syncthreads();
         for (int i = c0; i < c1; i += cstep) {
             const uint32_t u = use_cand ? S.cand[i] : key_at(i);
@@ -281,7 +299,7 @@ __global__ void __launch_bounds__(kTopkThreads)
             }
         __syncthreads();
         const int nw = (n + 31) >> 5;
-        const int wpt = (nw + kTopkThreads - 1) / kTopkThreads;  // words per thread
+        const int wpt = (nw + kRowThreads - 1) / kRowThreads;  // words per thread
         const int w0 = min(nw, tid * wpt), w1 = min(nw, w0 + wpt);
         uint32_t cnt = 0;
         for (int w = w0; w < w1; ++w) cnt += __popc(bits[w]);
@@ -295,9 +313,9 @@ __global__ void __launch_bounds__(kTopkThreads)
         __syncthreads();
         // positions in the warps before this one: a prefix scan of the warp
         // totals across lanes (lane w ends with the positions in warps <= w)
-        uint32_t ws = lane < kTopkWarps ? S.wsum[lane] : 0u;
+        uint32_t ws = lane < kRowWarps ? S.wsum[lane] : 0u;
 #pragma unroll
-        for (int off = 1; off < kTopkWarps; off <<= 1) {
+        for (int off = 1; off < kRowWarps; off <<= 1) {
             const uint32_t v = __shfl_up_sync(0xffffffffu, ws, off);
             if (lane >= off) ws += v;
         }
@@ -325,7 +343,7 @@ __global__ void __launch_bounds__(kTopkThreads)
     __syncthreads();
     uint32_t G = 0, E = 0;
 #pragma unroll
-    for (int w = 0; w < kTopkWarps; ++w)
+    for (int w = 0; w < kRowWarps; ++w)
         if (w < warp) {
             G += S.wcnt[0][w];
             E += S.wcnt[1][w];
@@ -785,6 +803,38 @@ static int launch_topk_cluster(ic_ctx* ctx, const float* scores, int64_t ld, int
     return IC_OK;
 }
 
+// one launch of the row kernel in the given shape (threads, candidate slots,
+// and the CTAs per SM it is compiled for, 0 leaving the register count to
+// the compiler), bcap the bitmap's keys
+template <int THREADS, int CAND, int MINB>
+static int launch_topk_rows(ic_ctx* ctx, const float* scores, int64_t ld, int rows, int k,
+                            int causal_base, const int32_t* row_len, int max_len,
+                            int32_t* idx_out, int64_t ld_out, int bcap, cudaStream_t stream) {
+    static PerDeviceOnce attr_once;
+    cudaError_t ea = attr_once.run(ctx->device, [] {
+        return cudaFuncSetAttribute(k_topk<THREADS, CAND, MINB>,
+                                    cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                    CAND * 4 + kBitmapCap / 8);
+    });
+    if (ea != cudaSuccess) return cuda_fail(ctx, ea, "cudaFuncSetAttribute(topk)");
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(rows, 1, 1);
+    cfg.blockDim = dim3(THREADS, 1, 1);
+    cfg.dynamicSmemBytes = CAND * 4 + bcap / 8;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    unsigned int na = 0;
+    add_pdl_attr(ctx, attr, na);
+    cfg.attrs = attr;
+    cfg.numAttrs = na;
+    LaunchScope ls(ctx, IC_K_TOPK, stream);
+    cudaLaunchKernelEx(&cfg, k_topk<THREADS, CAND, MINB>, scores, static_cast<long long>(ld), k,
+                       causal_base, row_len, max_len, idx_out, static_cast<long long>(ld_out), bcap);
+    cudaError_t e = ls.done();
+    if (e != cudaSuccess) return cuda_fail(ctx, e, "topk launch");
+    return IC_OK;
+}
+
 bool topk_uses_cluster(const ic_ctx* ctx, int rows, bool has_row_len, int max_len) {
     // few long rows (decode): a cluster of CTAs per row keeps many SMs busy
     return has_row_len && rows > 0 &&
@@ -801,33 +851,15 @@ int launch_topk(ic_ctx* ctx, const float* scores, int64_t ld, int rows, int k, i
                                    ld_out, stream, hist);
     if (hist != nullptr)
         return fail(ctx, IC_ERR_INVALID_ARG, "topk: a histogram is only used by the cluster form");
-    static PerDeviceOnce attr_once;
-    cudaError_t ea = attr_once.run(ctx->device, [] {
-        return cudaFuncSetAttribute(k_topk, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                    kCandCap * 4 + kBitmapCap / 8);
-    });
-    if (ea != cudaSuccess) return cuda_fail(ctx, ea, "cudaFuncSetAttribute(topk)");
     // causal row r has n = causal_base + r + 1 keys; rows longer than the
     // bitmap holds take the general path
     const long long nmax = row_len ? max_len : static_cast<long long>(causal_base) + rows;
     const int bcap = static_cast<int>(((nmax < kBitmapCap ? nmax : kBitmapCap) + 127) / 128 * 128);
-    const int smem = kCandCap * 4 + bcap / 8;
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(rows, 1, 1);
-    cfg.blockDim = dim3(kTopkThreads, 1, 1);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
-    cudaLaunchAttribute attr[1];
-    unsigned int na = 0;
-    add_pdl_attr(ctx, attr, na);
-    cfg.attrs = attr;
-    cfg.numAttrs = na;
-    LaunchScope ls(ctx, IC_K_TOPK, stream);
-    cudaLaunchKernelEx(&cfg, k_topk, scores, static_cast<long long>(ld), k, causal_base, row_len,
-                       max_len, idx_out, static_cast<long long>(ld_out), bcap);
-    cudaError_t e = ls.done();
-    if (e != cudaSuccess) return cuda_fail(ctx, e, "topk launch");
-    return IC_OK;
+    if (nmax <= kShortRow)
+        return launch_topk_rows<256, 2048, 8>(ctx, scores, ld, rows, k, causal_base, row_len,
+                                              max_len, idx_out, ld_out, bcap, stream);
+    return launch_topk_rows<512, 4096, 0>(ctx, scores, ld, rows, k, causal_base, row_len, max_len,
+                                          idx_out, ld_out, bcap, stream);
 }
 
 }  // namespace ic

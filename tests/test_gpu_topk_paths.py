@@ -1,11 +1,20 @@
-"""The top-k kernel's branches, each forced by a constructed row and
+"""The top-k kernels' branches, each forced by a constructed row and
 checked bit-exact against the oracle's top-k (positions of the k largest,
-ascending, ties to the lower position):
+ascending, ties to the lower position).
+
+The row kernel comes in two shapes, chosen by the longest row of a launch
+(16 warps and 4096 candidate slots above 32768 keys, 8 warps and 2048 slots
+up to it); a launch of few long rows with given lengths takes the cluster
+form instead.  Each set of rows runs in the launch shape that reaches the
+intended kernel, padded with Gaussian rows of assorted lengths where the
+row kernel needs more rows than the cluster form takes (every row checked):
   - the bitmap path on Gaussian rows, including one at the bitmap's
-    capacity (131072 keys), and one tie at T taken whole;
+    capacity (131072 keys) and one at the short shape's limit (32768), and
+    one tie at T taken whole;
   - the general path: a row longer than the bitmap holds, a candidate bin
     larger than the candidate list, a warp slice that overflows, and a tie
-    at T that is split by position."""
+    at T that is split by position;
+  - rows of at most k keys (all taken, -1 padding)."""
 import numpy as np
 import pytest
 import torch
@@ -23,7 +32,9 @@ def ic():
     return indexcache
 
 
-def _rows():
+def _long_rows():
+    """Rows for the long-row shape (and the cluster form): 4096 slots, and
+    a warp's slice of 256 slots over segments of n / 16 keys."""
     rng = np.random.default_rng(2024)
     rows = {}
     rows["gauss_20000"] = rng.standard_normal(20000)
@@ -56,15 +67,55 @@ def _rows():
     return {n: v.astype(np.float32) for n, v in rows.items()}
 
 
-def test_topk_every_path_bit_exact(ic):
-    ctx = ic.Context(0)
-    rows = _rows()
+def _short_rows():
+    """Rows for the short-row shape: 2048 slots, and a warp's slice of 256
+    slots over segments of n / 8 keys (2560 keys at n = 20000)."""
+    rng = np.random.default_rng(2025)
+    rows = {}
+    rows["gauss_16384"] = rng.standard_normal(16384)
+    rows["gauss_at_short_limit"] = rng.standard_normal(32768)
+    rows["gauss_2049"] = rng.standard_normal(2049)
+    rows["few_keys"] = rng.standard_normal(700)
+    # 1000 keys far above, 2500 keys in [1.0, 1.25) (one 11-bit bin): more
+    # than the list's 2048 slots
+    r = np.full(20000, -1.0) - rng.random(20000)
+    r[rng.permutation(20000)[:1000]] = 100.0 + rng.random(1000)
+    free = np.flatnonzero(r < 0)
+    r[rng.permutation(free)[:2500]] = 1.0 + 0.25 * rng.random(2500)
+    rows["bin_over_list"] = r
+    # 1500 keys far above, 1000 threshold-bin keys packed at the start: they
+    # fit the list but not the first warp's slice
+    r = np.full(20000, -1.0) - rng.random(20000)
+    r[:1000] = 1.0 + 0.25 * rng.random(1000)
+    r[1000 + rng.permutation(19000)[:1500]] = 100.0 + rng.random(1500)
+    rows["slice_overflow"] = r
+    # 2045 keys above 10, then the k-th value 5.0 three times (all taken) or
+    # six times (three taken, the lowest positions)
+    for name, ties in (("tie_taken_whole", 3), ("tie_split", 6)):
+        r = -rng.random(9000)
+        pos = rng.permutation(9000)
+        r[pos[:2045]] = 10.0 + rng.random(2045)
+        r[pos[2045:2045 + ties]] = 5.0
+        rows[name] = r
+    return {n: v.astype(np.float32) for n, v in rows.items()}
+
+
+def _check_launch(ic, rows, min_rows, filler_max, seed):
+    """One ic_topk launch over `rows` (padded to min_rows with Gaussian
+    rows of up to filler_max keys), every row compared with the oracle."""
+    rng = np.random.default_rng(seed)
+    rows = dict(rows)
+    i = 0
+    while len(rows) < min_rows:
+        rows["filler_%d" % i] = rng.standard_normal(int(rng.integers(1, filler_max + 1))).astype(np.float32)
+        i += 1
     names = list(rows)
     ld = (max(len(v) for v in rows.values()) + 3) // 4 * 4
     sc = torch.full((len(names), ld), -1e30, dtype=torch.float32)
     for i, n in enumerate(names):
         sc[i, :len(rows[n])] = torch.from_numpy(rows[n])
     lens = torch.tensor([len(rows[n]) for n in names], dtype=torch.int32)
+    ctx = ic.Context(0)
     idx = torch.empty((len(names), K), dtype=torch.int32, device="cuda")
     ic.ic_topk(ctx, sc.cuda(), K, idx, row_len=lens.cuda(), ld=ld)
     ctx.sync_status()
@@ -73,3 +124,28 @@ def test_topk_every_path_bit_exact(ic):
         want = oracle.topk_row(rows[n].astype(np.float64), K)
         assert got[i].tolist() == want.tolist(), n
     ctx.close()
+    return ld
+
+
+# rows * 8 CTAs above 4 per SM of a 148-SM part (and of any up to 192 SMs):
+# the launch cannot take the cluster form
+ROW_KERNEL_ROWS = 97
+
+
+def test_topk_cluster_form_every_path_bit_exact(ic):
+    """The constructed long rows alone: seven rows of up to 140000 keys
+    with given lengths take the cluster form."""
+    _check_launch(ic, _long_rows(), 0, 0, 0)
+
+
+def test_topk_long_row_kernel_every_path_bit_exact(ic):
+    """The same rows among 97: the row kernel's long-row shape."""
+    ld = _check_launch(ic, _long_rows(), ROW_KERNEL_ROWS, 140000, 1)
+    assert ld > 32768
+
+
+def test_topk_short_row_kernel_every_path_bit_exact(ic):
+    """Rows of at most 32768 keys among 97: the short-row shape, at its
+    limit."""
+    ld = _check_launch(ic, _short_rows(), ROW_KERNEL_ROWS, 32768, 2)
+    assert ld == 32768
