@@ -320,6 +320,13 @@ def run_ours(args, rank, world, local_rank):
                         "peak_kind": "HBM copy, " + peak_src,
                         "ms_per_f_layer": round(per_f, 4), "bytes_per_f_layer": bytes_f}
     overlap = measure_overlap(ctx, layers, cfg, stream)
+    # the same stack with the F layers' indexers issued ahead on a second
+    # stream (the multi-layer indexer page's scheduling); not the headline:
+    # it relies on each F layer's inputs being given
+    ahead = {"ms_per_step": round(time_stack_ahead(ctx, pat, dims, cache, arr, max(args.steps, 5),
+                                                   stream, flush), 4),
+             "stack_ms_per_step": round(ms_per_step, 4),
+             "what": "ic_run_stack_ahead on the same layers, L2 flushed between steps"}
     dominant = max(("index_score", "sparse_attn"), key=lambda n: ktimes[n]["ms"])
     roofline = dict(roof.get(dominant, {}))
     roofline["kernel"] = dominant
@@ -334,6 +341,7 @@ def run_ours(args, rank, world, local_rank):
         "roofline_all": roof,
         "l2_gather_ceiling": extra_ceiling,
         "cross_layer_overlap": overlap,
+        "stack_ahead": ahead,
     }
 
     # ------------------------------------------------ e2e through the C ABI with host buffers
@@ -665,7 +673,8 @@ def run_decode(args, ctx, peaks, peak_src, local_rank):
         ic.ic_run_stack(ctx, pat, None, dims, cache, layer_array=arr)
     ctx.sync_status()
     steps = max(args.steps, 5)
-    t = _time_stack(ctx, pat, dims, cache, arr, steps, torch.cuda.current_stream(), flush)
+    t = _time_stack(ctx, pat, dims, cache, arr, steps, torch.cuda.current_stream(), flush,
+                    ahead=True)
     kt = t.pop("kernels")
     n_f = cfg.pattern.count("F")
     scan_bytes = B * S * (cfg.d_I + 4) + B * S * 4  # e4m3 keys + scales read, fp32 scores written
@@ -767,7 +776,7 @@ def _attn_graph_launch_ms(ctx, layers, cache, S, d, reps, flush):
     return _graph_launch_ms(ctx, all_layers, len(layers), reps, flush)
 
 
-def _time_stack(ctx, pat, dims, cache, arr, steps, stream, flush=None, graph=True):
+def _time_stack(ctx, pat, dims, cache, arr, steps, stream, flush=None, graph=True, ahead=False):
     """One step of the stack timed three ways, each over `steps`
     steps with CUDA events around the step only: "step_ms" through
     ic_run_stack, "graph_step_ms" as a replay of the stack captured with
@@ -775,7 +784,8 @@ def _time_stack(ctx, pat, dims, cache, arr, steps, stream, flush=None, graph=Tru
     per-kernel timing events on (the per-kernel breakdown, "kernels", comes
     from that pass; its events add launch gaps to a step of many small
     kernels).  `flush`, when given, is rewritten before every step;
-    graph=False skips the graph pass."""
+    graph=False skips the graph pass; ahead=True adds "ahead_step_ms",
+    through ic_run_stack_ahead (F layers' indexers on a second stream)."""
     from cross_layer_top_b200 import indexcache as ic
 
     def timed(run):
@@ -797,6 +807,8 @@ def _time_stack(ctx, pat, dims, cache, arr, steps, stream, flush=None, graph=Tru
 
     plain = timed(eager)
     res = {"step_ms": plain}
+    if ahead:
+        res["ahead_step_ms"] = time_stack_ahead(ctx, pat, dims, cache, arr, steps, stream, flush)
     if graph:
         g = ic.ic_stack_graph_create(ctx, pat, None, dims, cache, layer_array=arr)
         for _ in range(2):
@@ -811,6 +823,34 @@ def _time_stack(ctx, pat, dims, cache, arr, steps, stream, flush=None, graph=Tru
     res["events_step_ms"] = with_events
     res["kernels"] = {n: ctx.get_timing(i) for i, n in enumerate(ic.KERNEL_NAMES)}
     return res
+
+
+def time_stack_ahead(ctx, pat, dims, cache, arr, steps, stream, flush=None):
+    """ms per step of ic_run_stack_ahead on the same layers (a second index
+    buffer beside `cache`), after two untimed steps; CUDA events on the
+    caller's stream, whose completion covers the side stream's work."""
+    from cross_layer_top_b200 import indexcache as ic
+    cache2 = torch.empty_like(cache)
+
+    def run():
+        ic.ic_run_stack_ahead(ctx, pat, None, dims, cache, cache2, stream=stream, layer_array=arr)
+
+    for _ in range(2):
+        run()
+    ctx.sync_status(stream)
+    tot = 0.0
+    for i in range(steps):
+        if flush is not None:
+            flush.fill_(float(i))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        run()
+        b.record(stream)
+        b.synchronize()
+        tot += a.elapsed_time(b)
+    ctx.sync_status(stream)
+    del cache2
+    return tot / steps
 
 
 def run_long_prefill(args, ctx, peaks, local_rank):

@@ -190,6 +190,14 @@ extern "C" int ic_ctx_destroy(ic_ctx* ctx) {
         cudaStreamDestroy(ctx->hs.in);
         cudaStreamDestroy(ctx->hs.out);
     }
+    if (ctx->ahead.ready) {
+        cudaEventDestroy(ctx->ahead.start);
+        for (int i = 0; i < 2; ++i) {
+            cudaEventDestroy(ctx->ahead.indexed[i]);
+            cudaEventDestroy(ctx->ahead.freed[i]);
+        }
+        cudaStreamDestroy(ctx->ahead.side);
+    }
     for (auto& p : ctx->pool) {
         cudaEventDestroy(p.start);
         cudaEventDestroy(p.stop);

@@ -60,6 +60,13 @@ struct ic_ctx {
         void* slot[kHostSlots] = {};
         size_t slot_cap = 0;  // bytes per slot
     } hs;
+    // ic_run_stack_ahead: the side stream that runs the F layers' indexers,
+    // and its fork and buffer events (created on first use)
+    struct Ahead {
+        bool ready = false;
+        cudaStream_t side = nullptr;
+        cudaEvent_t start = nullptr, indexed[2] = {}, freed[2] = {};
+    } ahead;
 };
 
 struct ic_pattern {

@@ -89,6 +89,8 @@ _SIGS = {
                       _vp], _i),
     "ic_run_stack_host": ([_vp, _vp, ctypes.POINTER(ic_layer_io), ctypes.POINTER(ic_stack_dims),
                            _vp, _vp], _i),
+    "ic_run_stack_ahead": ([_vp, _vp, ctypes.POINTER(ic_layer_io), ctypes.POINTER(ic_stack_dims),
+                            _vp, _vp, _vp], _i),
     "ic_run_stack_rows": ([_vp, _vp, ctypes.POINTER(ic_layer_io), ctypes.POINTER(ic_stack_dims),
                            ctypes.POINTER(ctypes.c_int32), _i, _vp, _vp], _i),
     "ic_prefill_partition": ([_i, _i, _i, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(_i)], _i),
@@ -380,6 +382,16 @@ def ic_run_stack(ctx: Context, pattern: Pattern, layers, dims: ic_stack_dims, id
     arr = layer_array if layer_array is not None else make_stack_layers(layers, dims.mode)
     _check(_lib.ic_run_stack(ctx.handle, pattern.handle, arr, ctypes.byref(dims),
                              _ptr(idx_cache), _stream(stream)), ctx)
+
+
+def ic_run_stack_ahead(ctx: Context, pattern: Pattern, layers, dims: ic_stack_dims, idx_cache,
+                       idx_cache2, stream=None, layer_array=None):
+    """ic_run_stack with each F layer's indexer issued ahead on a second
+    stream; the j-th F layer's indices go to idx_cache (j even) or
+    idx_cache2 (j odd)."""
+    arr = layer_array if layer_array is not None else make_stack_layers(layers, dims.mode)
+    _check(_lib.ic_run_stack_ahead(ctx.handle, pattern.handle, arr, ctypes.byref(dims),
+                                   _ptr(idx_cache), _ptr(idx_cache2), _stream(stream)), ctx)
 
 
 def ic_run_stack_host(ctx: Context, pattern: Pattern, layers_host, dims: ic_stack_dims, idx_cache,

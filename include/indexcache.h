@@ -333,6 +333,25 @@ typedef struct ic_stack_dims {
 int ic_run_stack(ic_ctx *ctx, const ic_pattern *pattern, const ic_layer_io *layers,
                  const ic_stack_dims *dims, int32_t *idx_cache, void *stream);
 
+/* The same stack with every F layer's indexer and top-k issued ahead on a
+ * second, context-owned stream, so that it runs while the attention of the
+ * layers before it runs (the scheduling idea of the multi-layer indexer
+ * page, "MLI", on this method's own indices).  Valid only because each F
+ * layer's indexer inputs are given: in a model whose layer l reads layer
+ * l-1's output this order would not exist.  The j-th F layer (0-based)
+ * writes its index tensor to idx_cache when j is even and to idx_cache2
+ * when j is odd (both device int32 [rows, k], distinct, overwritten), and
+ * it and the S layers after it attend from there; F layer j's indexer
+ * waits until the layers of F layer j-2's group have attended.  Every
+ * output, snapshot and index tensor is bit-identical to ic_run_stack's.
+ * The side stream first waits for the work `stream` held at the call, and
+ * `stream` ends after the last layer, so its completion covers all work.
+ * No programmatic launches or cross-layer prefetch.  Errors as ic_run_stack,
+ * plus IC_ERR_INVALID_ARG when idx_cache2 is NULL or equals idx_cache. */
+int ic_run_stack_ahead(ic_ctx *ctx, const ic_pattern *pattern, const ic_layer_io *layers,
+                       const ic_stack_dims *dims, int32_t *idx_cache, int32_t *idx_cache2,
+                       void *stream);
+
 /* The prefill stack of one rank of a row split ([IC] Figure 2 over the
  * rank's rows).  `ranges` (HOST int32 [2*n_ranges], half-open, disjoint,
  * e.g. from ic_prefill_partition) are the rank's query rows.  In layers[l],
