@@ -785,7 +785,8 @@ def _time_stack(ctx, pat, dims, cache, arr, steps, stream, flush=None, graph=Tru
     from that pass; its events add launch gaps to a step of many small
     kernels).  `flush`, when given, is rewritten before every step;
     graph=False skips the graph pass; ahead=True adds "ahead_step_ms",
-    through ic_run_stack_ahead (F layers' indexers on a second stream)."""
+    through ic_run_stack_ahead (F layers' indexers on a second stream), and
+    with the graph pass "ahead_graph_step_ms", a replay of its graph."""
     from cross_layer_top_b200 import indexcache as ic
 
     def timed(run):
@@ -809,6 +810,15 @@ def _time_stack(ctx, pat, dims, cache, arr, steps, stream, flush=None, graph=Tru
     res = {"step_ms": plain}
     if ahead:
         res["ahead_step_ms"] = time_stack_ahead(ctx, pat, dims, cache, arr, steps, stream, flush)
+        if graph:
+            cache2 = torch.empty_like(cache)
+            g = ic.ic_stack_graph_create_ahead(ctx, pat, None, dims, cache, cache2,
+                                               layer_array=arr)
+            for _ in range(2):
+                g.launch(stream)
+            res["ahead_graph_step_ms"] = timed(lambda: g.launch(stream))
+            g.close()
+            del cache2
     if graph:
         g = ic.ic_stack_graph_create(ctx, pat, None, dims, cache, layer_array=arr)
         for _ in range(2):
@@ -968,7 +978,7 @@ def run_decode_sweep(args, ctx, local_rank):
         pat = ic.ic_pattern_uniform(cfg.n_layers, r)
         for _ in range(2):
             ic.ic_run_stack(ctx, pat, None, dims, cache, layer_array=arr)
-        t = _time_stack(ctx, pat, dims, cache, arr, 5, stream)
+        t = _time_stack(ctx, pat, dims, cache, arr, 5, stream, ahead=True)
         kt = t.pop("kernels")
         res["r%d" % r] = {"pattern_F_layers": str(pat).count("F"), **t,
                           "tokens_per_s": B / (t["step_ms"] / 1e3),
@@ -979,7 +989,7 @@ def run_decode_sweep(args, ctx, local_rank):
         pat = ic.ic_create_pattern(c)
         for _ in range(2):
             ic.ic_run_stack(ctx, pat, None, dims, cache, layer_array=arr)
-        t = _time_stack(ctx, pat, dims, cache, arr, 5, stream)
+        t = _time_stack(ctx, pat, dims, cache, arr, 5, stream, ahead=True)
         kt = t.pop("kernels")
         res["searched_" + ret.replace("/", "_")] = {
             "pattern_F_layers": c.count("F"), **t, "tokens_per_s": B / (t["step_ms"] / 1e3),

@@ -11,6 +11,11 @@
 // idx_cache and dims->seq_len alive and changes their contents, not their
 // addresses, between replays.  While any graph exists, the context refuses
 // to regrow the scratch buffers the graph uses.
+//
+// ic_stack_graph_create_ahead captures ic_run_stack_ahead instead: the side
+// stream joins the capture through the fork event and rejoins it through
+// the last F layer's event, so the graph holds both streams' kernels with
+// the same dependencies.
 #include "ic_internal.h"
 
 using namespace ic;
@@ -22,9 +27,20 @@ struct ic_graph {
     int64_t kernels = 0;  // kernel launches in one replay
 };
 
-extern "C" int ic_stack_graph_create(ic_ctx* ctx, const ic_pattern* pattern,
-                                     const ic_layer_io* layers, const ic_stack_dims* dims,
-                                     int32_t* idx_cache, ic_graph** out) {
+namespace {
+
+// the stack in the chosen schedule: ic_run_stack, or ic_run_stack_ahead
+// when idx_cache2 is given
+int run_schedule(ic_ctx* ctx, const ic_pattern* pattern, const ic_layer_io* layers,
+                 const ic_stack_dims* dims, int32_t* idx_cache, int32_t* idx_cache2,
+                 cudaStream_t s) {
+    if (idx_cache2) return ic_run_stack_ahead(ctx, pattern, layers, dims, idx_cache, idx_cache2, s);
+    return ic_run_stack(ctx, pattern, layers, dims, idx_cache, s);
+}
+
+int graph_create(ic_ctx* ctx, const ic_pattern* pattern, const ic_layer_io* layers,
+                 const ic_stack_dims* dims, int32_t* idx_cache, int32_t* idx_cache2,
+                 ic_graph** out) {
     if (!out) return fail(ctx, IC_ERR_INVALID_ARG, "stack_graph_create: out is NULL");
     *out = nullptr;
     int rc = check_stack_args(ctx, pattern, layers, dims, idx_cache);
@@ -36,7 +52,7 @@ extern "C" int ic_stack_graph_create(ic_ctx* ctx, const ic_pattern* pattern,
     const bool timing = ctx->timing;
     ctx->timing = false;  // no timing events inside the graph
     // eager pass: scratch sizes, kernel attributes, cluster-occupancy queries
-    rc = ic_run_stack(ctx, pattern, layers, dims, idx_cache, s);
+    rc = run_schedule(ctx, pattern, layers, dims, idx_cache, idx_cache2, s);
     if (!rc) {
         e = cudaStreamSynchronize(s);
         if (e != cudaSuccess) rc = cuda_fail(ctx, e, "stack_graph_create: eager pass");
@@ -50,7 +66,7 @@ extern "C" int ic_stack_graph_create(ic_ctx* ctx, const ic_pattern* pattern,
         if (e != cudaSuccess) {
             rc = cuda_fail(ctx, e, "stack_graph_create: begin capture");
         } else {
-            rc = ic_run_stack(ctx, pattern, layers, dims, idx_cache, s);
+            rc = run_schedule(ctx, pattern, layers, dims, idx_cache, idx_cache2, s);
             cudaGraph_t graph = nullptr;
             e = cudaStreamEndCapture(s, &graph);  // always ends the capture
             g->graph = graph;
@@ -77,6 +93,24 @@ extern "C" int ic_stack_graph_create(ic_ctx* ctx, const ic_pattern* pattern,
     ctx->graphs_alive++;
     *out = g;
     return IC_OK;
+}
+
+}  // namespace
+
+extern "C" int ic_stack_graph_create(ic_ctx* ctx, const ic_pattern* pattern,
+                                     const ic_layer_io* layers, const ic_stack_dims* dims,
+                                     int32_t* idx_cache, ic_graph** out) {
+    return graph_create(ctx, pattern, layers, dims, idx_cache, nullptr, out);
+}
+
+extern "C" int ic_stack_graph_create_ahead(ic_ctx* ctx, const ic_pattern* pattern,
+                                           const ic_layer_io* layers, const ic_stack_dims* dims,
+                                           int32_t* idx_cache, int32_t* idx_cache2,
+                                           ic_graph** out) {
+    if (!idx_cache2 || idx_cache2 == idx_cache)
+        return fail(ctx, IC_ERR_INVALID_ARG, "stack_graph_create_ahead: idx_cache2 must be a "
+                                             "second buffer");
+    return graph_create(ctx, pattern, layers, dims, idx_cache, idx_cache2, out);
 }
 
 extern "C" int ic_stack_graph_launch(ic_graph* g, void* stream) {

@@ -97,6 +97,9 @@ _SIGS = {
     "ic_index_fp_rows": ([_vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _i, _vp, _vp], _i),
     "ic_stack_graph_create": ([_vp, _vp, ctypes.POINTER(ic_layer_io),
                                ctypes.POINTER(ic_stack_dims), _vp, ctypes.POINTER(_vp)], _i),
+    "ic_stack_graph_create_ahead": ([_vp, _vp, ctypes.POINTER(ic_layer_io),
+                                     ctypes.POINTER(ic_stack_dims), _vp, _vp,
+                                     ctypes.POINTER(_vp)], _i),
     "ic_stack_graph_launch": ([_vp, _vp], _i),
     "ic_stack_graph_kernels": ([_vp], _i64),
     "ic_stack_graph_destroy": ([_vp], _i),
@@ -445,18 +448,25 @@ class StackGraph:
     """ic_stack_graph_*: the stack captured once and replayed.  The graph
     keeps the device addresses of the layer tensors, dims.seq_len and
     idx_cache, so this object holds references to them; change their
-    contents in place between launches."""
+    contents in place between launches.  With idx_cache2, the schedule of
+    ic_run_stack_ahead is captured (ic_stack_graph_create_ahead)."""
 
     def __init__(self, ctx: Context, pattern: Pattern, layers, dims: ic_stack_dims, idx_cache,
-                 layer_array=None):
+                 layer_array=None, idx_cache2=None):
         arr = layer_array if layer_array is not None else make_stack_layers(layers, dims.mode)
         h = _vp()
-        _check(_lib.ic_stack_graph_create(ctx.handle, pattern.handle, arr, ctypes.byref(dims),
-                                          _ptr(idx_cache), ctypes.byref(h)), ctx)
+        if idx_cache2 is None:
+            rc = _lib.ic_stack_graph_create(ctx.handle, pattern.handle, arr, ctypes.byref(dims),
+                                            _ptr(idx_cache), ctypes.byref(h))
+        else:
+            rc = _lib.ic_stack_graph_create_ahead(ctx.handle, pattern.handle, arr,
+                                                  ctypes.byref(dims), _ptr(idx_cache),
+                                                  _ptr(idx_cache2), ctypes.byref(h))
+        _check(rc, ctx)
         self.handle = h
         self.ctx = ctx
         ctx._graphs.add(self)
-        self._keep = (pattern, layers, dims, idx_cache, arr)
+        self._keep = (pattern, layers, dims, idx_cache, idx_cache2, arr)
 
     def launch(self, stream=None):
         _check(_lib.ic_stack_graph_launch(self.handle, _stream(stream)), self.ctx)
@@ -479,6 +489,11 @@ class StackGraph:
 def ic_stack_graph_create(ctx: Context, pattern: Pattern, layers, dims: ic_stack_dims, idx_cache,
                           layer_array=None) -> StackGraph:
     return StackGraph(ctx, pattern, layers, dims, idx_cache, layer_array)
+
+
+def ic_stack_graph_create_ahead(ctx: Context, pattern: Pattern, layers, dims: ic_stack_dims,
+                                idx_cache, idx_cache2, layer_array=None) -> StackGraph:
+    return StackGraph(ctx, pattern, layers, dims, idx_cache, layer_array, idx_cache2)
 
 
 def stack_dims(mode, H_I, d_I, k, Hq, d, L=0, B=0, S_max=0, seq_len=None, scale=0.0):

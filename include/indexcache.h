@@ -380,6 +380,13 @@ int ic_run_stack_rows(ic_ctx *ctx, const ic_pattern *pattern, const ic_layer_io 
 typedef struct ic_graph ic_graph;
 int ic_stack_graph_create(ic_ctx *ctx, const ic_pattern *pattern, const ic_layer_io *layers,
                           const ic_stack_dims *dims, int32_t *idx_cache, ic_graph **out);
+/* The same for the schedule of ic_run_stack_ahead (its two index buffers;
+ * the side stream's kernels are captured into the same graph with their
+ * dependencies).  Errors as ic_stack_graph_create, plus IC_ERR_INVALID_ARG
+ * when idx_cache2 is NULL or equals idx_cache. */
+int ic_stack_graph_create_ahead(ic_ctx *ctx, const ic_pattern *pattern, const ic_layer_io *layers,
+                                const ic_stack_dims *dims, int32_t *idx_cache, int32_t *idx_cache2,
+                                ic_graph **out);
 int ic_stack_graph_launch(ic_graph *graph, void *stream);
 int64_t ic_stack_graph_kernels(const ic_graph *graph);
 int ic_stack_graph_destroy(ic_graph *graph);

@@ -1,7 +1,8 @@
 """ic_run_stack_ahead: the layer stack with every F layer's indexer issued
-ahead on a second stream (the multi-layer indexer page's scheduling).  The
-order of the kernels changes, not their inputs, so every index tensor and
-output must equal ic_run_stack's bit for bit; on the integer tiny workload
+ahead on a second stream (the multi-layer indexer page's scheduling), run
+eagerly and as a captured graph (ic_stack_graph_create_ahead).  The order
+of the kernels changes, not their inputs, so every index tensor and output
+must equal ic_run_stack's bit for bit; on the integer tiny workload
 the indices are also checked against the oracle's stack and the attention
 against the oracle within the attention bars of tests/attn_check.py.
 
@@ -47,13 +48,28 @@ def _with_outputs(layers, rows, cfg):
     return out
 
 
-def _run_both(ic, ctx, pattern, glayers_a, glayers_b, dims, rows, k):
+def _run_both(ic, ctx, pattern, glayers_a, glayers_b, dims, rows, k, graph=False):
+    """ic_run_stack into glayers_a, ic_run_stack_ahead into glayers_b (with
+    graph=True: its captured graph, replayed twice with the outputs and
+    buffers reset in between), then every output and index tensor compared."""
     pat = ic.ic_create_pattern(pattern)
     cache = torch.empty((rows, k), dtype=torch.int32, device="cuda")
     ic.ic_run_stack(ctx, pat, glayers_a, dims, cache)
     c0 = torch.full((rows, k), -9, dtype=torch.int32, device="cuda")
     c1 = torch.full((rows, k), -9, dtype=torch.int32, device="cuda")
-    ic.ic_run_stack_ahead(ctx, pat, glayers_b, dims, c0, c1)
+    if graph:
+        g = ic.ic_stack_graph_create_ahead(ctx, pat, glayers_b, dims, c0, c1)
+        for _ in range(2):
+            for lay in glayers_b:
+                lay["out"].fill_(float("nan"))
+                lay["idx_snapshot"].fill_(-7)
+            c0.fill_(-9)
+            c1.fill_(-9)
+            g.launch()
+        ctx.sync_status()
+        g.close()
+    else:
+        ic.ic_run_stack_ahead(ctx, pat, glayers_b, dims, c0, c1)
     ctx.sync_status()
     for l in range(len(pattern)):
         assert torch.equal(glayers_a[l]["idx_snapshot"], glayers_b[l]["idx_snapshot"]), l
@@ -68,7 +84,8 @@ def _run_both(ic, ctx, pattern, glayers_a, glayers_b, dims, rows, k):
             assert torch.all(buf == -9)
 
 
-def test_stack_ahead_tiny_against_oracle(ic):
+@pytest.mark.parametrize("graph", [False, True])
+def test_stack_ahead_tiny_against_oracle(ic, graph):
     cfg = synth.CONFIGS["tiny"]
     pattern = "FSFFSSFS"
     L, k = cfg.L, cfg.k
@@ -77,7 +94,7 @@ def test_stack_ahead_tiny_against_oracle(ic):
     ga = _with_outputs(layers, L, cfg)
     gb = _with_outputs(layers, L, cfg)
     dims = ic.stack_dims(ic.IC_PREFILL, cfg.H_I, cfg.d_I, k, cfg.Hq, cfg.d, L=L)
-    _run_both(ic, ctx, pattern, ga, gb, dims, L, k)
+    _run_both(ic, ctx, pattern, ga, gb, dims, L, k, graph=graph)
     olayers = [{n: f32(v) for n, v in lay.items()} for lay in layers]
     oidx, oout = oracle.run_stack(pattern, olayers, k)
     for l in range(len(pattern)):
@@ -104,8 +121,10 @@ def test_stack_ahead_prefill_equals_stack(ic):
     ctx.close()
 
 
-def test_stack_ahead_decode_equals_stack(ic):
-    """The batched-decode stack (32 x 65537, 16 layers FSSS x4)."""
+@pytest.mark.parametrize("graph", [False, True])
+def test_stack_ahead_decode_equals_stack(ic, graph):
+    """The batched-decode stack (32 x 65537, 16 layers FSSS x4), eagerly and
+    as a captured graph."""
     cfg = synth.CONFIGS["decode"]
     B, S, k = cfg.B, cfg.S, cfg.k
     ctx = ic.Context(0)
@@ -123,11 +142,12 @@ def test_stack_ahead_decode_equals_stack(ic):
             out.append(g)
         return out
 
-    _run_both(ic, ctx, cfg.pattern, outputs(), outputs(), dims, B, k)
+    _run_both(ic, ctx, cfg.pattern, outputs(), outputs(), dims, B, k, graph=graph)
     ctx.close()
 
 
 def test_stack_ahead_needs_two_buffers(ic):
+    """Both the eager call and the graph capture refuse one buffer twice."""
     cfg = synth.CONFIGS["tiny"]
     L, k = cfg.L, cfg.k
     ctx = ic.Context(0)
@@ -136,5 +156,9 @@ def test_stack_ahead_needs_two_buffers(ic):
     cache = torch.empty((L, k), dtype=torch.int32, device="cuda")
     with pytest.raises(ic.ICError) as e:
         ic.ic_run_stack_ahead(ctx, ic.ic_create_pattern(cfg.pattern), layers, dims, cache, cache)
+    assert e.value.code == ic.IC_ERR_INVALID_ARG
+    with pytest.raises(ic.ICError) as e:
+        ic.ic_stack_graph_create_ahead(ctx, ic.ic_create_pattern(cfg.pattern), layers, dims,
+                                       cache, cache)
     assert e.value.code == ic.IC_ERR_INVALID_ARG
     ctx.close()
