@@ -315,10 +315,26 @@ def run_ours(args, rank, world, local_rank):
         bytes_f = sum(4 * (t + 1) for t in range(k, L)) + 4 * k * L
         per_f = top_k["ms"] / (args.steps * n_f)
         gbs = bytes_f / (per_f / 1e3) / 1e9
-        roof["topk"] = {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
-                        "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4), "traffic": None,
-                        "peak_kind": "HBM copy, " + peak_src,
-                        "ms_per_f_layer": round(per_f, 4), "bytes_per_f_layer": bytes_f}
+        # The kernel is bound by instruction issue (ncu: issue active 79%):
+        # the warp-instructions one launch over the scored rows executes (from
+        # the capture of the current kernel), per second, against one
+        # instruction per clock on each of the SM's 4 schedulers at the clock
+        # sampled during the timed steps.
+        mhz = clk.get("sm_mhz") or clk.get("sm_max_mhz") or 1965.0
+        sms = torch.cuda.get_device_properties(stream.device).multi_processor_count
+        issue_peak = 4 * sms * mhz * 1e6 / 1e9
+        roof["topk"] = {"bound": "issue", "achieved": None, "peak": round(issue_peak, 1),
+                        "unit": "G warp-instructions/s", "frac": None, "traffic": TOPK_PREFILL_DRAM_BYTES,
+                        "peak_kind": "4 schedulers x %d SMs x %.0f MHz (sampled)" % (sms, mhz),
+                        "ms_per_f_layer": round(per_f, 4), "bytes_per_f_layer": bytes_f,
+                        "hbm": {"achieved": round(gbs, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                "frac": round(gbs / peaks["hbm_gbs"], 4),
+                                "peak_kind": "HBM copy, " + peak_src}}
+        if TOPK_PREFILL_WARP_INSTR:
+            ginst = TOPK_PREFILL_WARP_INSTR / (per_f / 1e3) / 1e9
+            roof["topk"]["achieved"] = round(ginst, 1)
+            roof["topk"]["frac"] = round(ginst / issue_peak, 4)
+            roof["topk"]["warp_instructions_per_launch"] = TOPK_PREFILL_WARP_INSTR
     overlap = measure_overlap(ctx, layers, cfg, stream)
     # the same stack with the F layers' indexers issued ahead on a second
     # stream (the multi-layer indexer page's scheduling); not the headline:
@@ -398,6 +414,10 @@ def run_ours(args, rank, world, local_rank):
 # None once a kernel changes until it is captured again.
 ATTN_PREFILL_DRAM_BYTES = 210.32e6 + 50.96e6
 INDEX_SCORE_PREFILL_DRAM_BYTES = 249.13e6 + 487.47e6
+TOPK_PREFILL_DRAM_BYTES = 530.31e6 + 107.22e6
+# warp-instructions of one prefill top-k launch over the scored rows (the
+# same capture: smsp__inst_executed.sum)
+TOPK_PREFILL_WARP_INSTR = 310.89e6
 
 
 def measure_gather_ceiling(cache, lay, L, k, stream):

@@ -1,9 +1,9 @@
 """Edge cases of the path on the GPU against the oracle: degenerate stacks
 (L <= k, where every row keeps all of its causal keys and sparse attention
 is ordinary causal attention; L = 1; k = 1; a single F layer), empty launches,
-one-candidate decode rows, and the longest decode rows, whose top-k leaves
+one-candidate decode rows, the longest decode rows, whose top-k leaves
 the cluster form for the single-CTA kernel's general path (rows past its
-shared selection bitmap)."""
+shared selection bitmap), and decode stacks of ragged sequence lengths."""
 import numpy as np
 import pytest
 import torch
@@ -124,3 +124,54 @@ def test_decode_rows_past_the_cluster_form(ic, ctx):
         n = int(lt[b])
         ref = oracle.decode_scores(f32(q[b]), f32(w[b]), k8[b].numpy(), sc[b].numpy(), S=n)
         assert got[b].tolist() == oracle.topk_row(ref, k).tolist(), b
+
+
+@pytest.mark.parametrize("S_max", [9000, 40001])
+def test_decode_stack_ragged_lengths(ic, ctx, S_max):
+    """A decode stack whose sequences hold different numbers of candidates
+    (1, k + 1, a middle length and the full capacity), with the single-CTA
+    top-k (9000) and the cluster top-k (40001): F-layer selections within
+    the oracle's bar (rows of at most k candidates take all of them), the
+    reuse invariant, and every layer's attention against the oracle."""
+    import dataclasses
+    k = 2048
+    cfg = dataclasses.replace(synth.CONFIGS["decode"], B=4, ctx=S_max - 1, pattern="FSFS", k=k,
+                              seed=17)
+    B, S = cfg.B, cfg.S
+    lens = [S, 1, k + 1, S // 2]
+    seq_len = torch.tensor(lens, dtype=torch.int32, device="cuda")
+    layers = []
+    for l in range(cfg.n_layers):
+        lay = synth.decode_layer(cfg, l, "cuda")
+        lay["seq_len"] = seq_len
+        lay["out"] = torch.empty((B, cfg.Hq, cfg.d), dtype=torch.bfloat16, device="cuda")
+        lay["idx_snapshot"] = torch.full((B, k), -7, dtype=torch.int32, device="cuda")
+        layers.append(lay)
+    dims = ic.stack_dims(ic.IC_DECODE, cfg.H_I, cfg.d_I, k, cfg.Hq, cfg.d, B=B, S_max=S,
+                         seq_len=seq_len)
+    cache = torch.empty((B, k), dtype=torch.int32, device="cuda")
+    ic.ic_run_stack(ctx, ic.ic_create_pattern(cfg.pattern), layers, dims, cache)
+    ctx.sync_status()
+    src = oracle.pattern_src(cfg.pattern)
+    snaps = [lay["idx_snapshot"].cpu().numpy() for lay in layers]
+    for l, c in enumerate(cfg.pattern):
+        assert np.array_equal(snaps[l], snaps[src[l]]), l
+        lay = layers[l]
+        if c == "F":
+            for b in range(B):
+                n = lens[b]
+                ref = oracle.decode_scores(f32(lay["q"][b]), f32(lay["w"][b]),
+                                           lay["kI8"][b].cpu().numpy(),
+                                           lay["kI_scale"][b].cpu().numpy(), S=n)
+                row = snaps[l][b]
+                m = min(n, k)
+                assert np.all(row[m:] == -1) and np.all(np.diff(row[:m]) > 0)
+                assert row[:m].min() >= 0 and row[:m].max() < n
+                if n <= k:
+                    assert row[:m].tolist() == list(range(n))
+                else:
+                    kth = oracle.kth_score(ref, k)
+                    assert ref[row[:m]].min() >= kth - 1e-3 * abs(kth)
+        got = lay["out"].float().cpu().numpy().astype(np.float64)
+        attn_check.check(got, f32(lay["Q"]), f32(lay["K"]), f32(lay["V"]), snaps[l],
+                         rows_per_seq=1, what="ragged decode S_max=%d layer %d" % (S_max, l))
