@@ -267,6 +267,11 @@ __global__ void __launch_bounds__(kRowThreads, kRowMinCtas)
     const int c0 = sliced ? warp * kSlice + lane : tid;
     const int c1 = sliced ? warp * kSlice + static_cast<int>(S.wcand[warp]) : ncand;
     const int cstep = sliced ? 32 : kRowThreads;
+    // On the bitmap path the third digit is skipped when the second
+    // digit's bin is taken whole (the usual case for real-valued scores):
+    // T is then that bin's smallest key, and the keys >= T are exactly the
+    // selection.
+    bool whole = false;
 #pragma unroll 1
     for (int pass = 0; pass < 2; ++pass) {
         const int shift = pass == 0 ? 10 : 0;
@@ -285,13 +290,20 @@ __global__ void __launch_bounds__(kRowThreads, kRowMinCtas)
         prefix |= S.bin << shift;
         mask |= dmask << shift;
         krem -= S.above;
+        const bool taken_whole = pass == 0 && sliced && krem == S.bin_count;  // the same in every thread
         __syncthreads();
+        if (taken_whole) {
+            whole = true;
+            break;
+        }
     }
     const uint32_t T = prefix;
 
     // ---- C (bitmap): when every key equal to T is taken, mark the
-    // candidates >= T in the bitmap and write its set positions in order
-    if (sliced && krem == S.hist[T & 0x3FFu]) {
+    // candidates >= T in the bitmap, gather its set positions in order in
+    // shared memory (over the candidates' positions, no longer needed),
+    // then write the row's k positions with coalesced stores
+    if (sliced && (whole || krem == S.hist[T & 0x3FFu])) {
         for (int j = c0; j < c1; j += 32)
             if (S.cand[j] >= T) {
                 const int pos = cpos[j];
@@ -321,9 +333,16 @@ __global__ void __launch_bounds__(kRowThreads, kRowMinCtas)
         }
         const uint32_t before = __shfl_sync(0xffffffffu, ws, warp > 0 ? warp - 1 : 0);
         uint32_t at = incl - cnt + (warp > 0 ? before : 0u);
+        uint32_t* opos = cpos;  // k <= kRowCandCap slots
         for (int w = w0; w < w1; ++w)
-            for (uint32_t x = bits[w]; x; x &= x - 1u) o[at++] = (w << 5) + (__ffs(x) - 1);
-        return;  // exactly k positions were written
+            for (uint32_t x = bits[w]; x; x &= x - 1u) {
+                // exactly k bits are set; the bound only guards the buffer
+                if (at < static_cast<uint32_t>(k)) opos[at] = (w << 5) + (__ffs(x) - 1);
+                ++at;
+            }
+        __syncthreads();
+        for (int i = tid; i < k; i += kRowThreads) o[i] = static_cast<int32_t>(opos[i]);
+        return;
     }
 
     // ---- C (ordered passes): per-warp segments, counts, offsets, writes
@@ -673,7 +692,12 @@ __global__ void __launch_bounds__(kTopkThreads)
         prefix |= S.bin << shift;
         mask |= dmask << shift;
         krem -= S.above;
+        // the second digit's bin taken whole (the usual case): T = its
+        // smallest key, every key >= T is selected and the third digit is
+        // not needed (the same answer in every thread and CTA)
+        const bool taken_whole = pass == 1 && use_cand && krem == S.bin_count;
         __syncthreads();
+        if (taken_whole) break;
     }
     const uint32_t T = prefix;
 
