@@ -520,16 +520,20 @@ __global__ void __launch_bounds__(kTopkThreads)
             total += nq[q];
         }
         for (int i4 = 4 * tid; i4 < kCandCap; i4 += 4 * kTopkThreads) {
-            uint4 cv[kClusterCtas];
+            // two rounds of loads from half the CTAs each
 #pragma unroll
-            for (uint32_t q = 0; q < kClusterCtas; ++q)
-                if (i4 < nq[q]) cv[q] = dsmem_ld_u4(dsmem_addr(&S.cand[i4], q));
+            for (uint32_t h = 0; h < kClusterCtas; h += kClusterCtas / 2) {
+                uint4 cv[kClusterCtas / 2];
 #pragma unroll
-            for (uint32_t q = 0; q < kClusterCtas; ++q) {
-                const uint32_t c4[4] = {cv[q].x, cv[q].y, cv[q].z, cv[q].w};
+                for (uint32_t q = 0; q < kClusterCtas / 2; ++q)
+                    if (i4 < nq[h + q]) cv[q] = dsmem_ld_u4(dsmem_addr(&S.cand[i4], h + q));
 #pragma unroll
-                for (int e = 0; e < 4; ++e)
-                    if (i4 + e < nq[q]) cand_all[off[q] + i4 + e] = c4[e];
+                for (uint32_t q = 0; q < kClusterCtas / 2; ++q) {
+                    const uint32_t c4[4] = {cv[q].x, cv[q].y, cv[q].z, cv[q].w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        if (i4 + e < nq[h + q]) cand_all[off[h + q] + i4 + e] = c4[e];
+                }
             }
         }
         // No CTA rewrites its S.ncand or S.cand after this, so other CTAs may
@@ -664,6 +668,7 @@ __global__ void __launch_bounds__(kTopkThreads)
             ncand = merge_candidates();
         }
     }  // the path without a histogram (or with too many keys in its bin)
+    bool whole = false;  // the second digit's bin taken whole (below)
 #pragma unroll 1
     for (int pass = first_pass; pass < 3; ++pass) {
         const int shift = pass == 0 ? 21 : (pass == 1 ? 10 : 0);
@@ -697,9 +702,87 @@ __global__ void __launch_bounds__(kTopkThreads)
         // not needed (the same answer in every thread and CTA)
         const bool taken_whole = pass == 1 && use_cand && krem == S.bin_count;
         __syncthreads();
-        if (taken_whole) break;
+        if (taken_whole) {
+            whole = true;
+            break;
+        }
     }
     const uint32_t T = prefix;
+
+    // ---- C (bitmap): when every key equal to T is taken (the same answer in
+    // every CTA: it follows from the merged candidates), the selection is
+    // the keys >= T.  One pass marks this segment's in a bitmap (over the
+    // merged candidates, no longer needed), a block scan of the words'
+    // popcounts gives each thread its offset, the segment's total goes to
+    // the later CTAs, and the positions are gathered in order in shared
+    // memory (over this CTA's candidate list, which no CTA reads after the
+    // barrier) and written with coalesced stores.
+    if (use_cand && (whole || krem == S.hist[T & 0x3FFu])) {
+        uint32_t* bits = cand_all;  // ceil(m / 32) <= kCandCap words
+        for (int base = 128 * warp; base < m; base += 128 * kTopkWarps) {
+            const int i0 = base + 4 * lane;
+            uint32_t nib = 0;
+            if (i0 + 3 < m) {
+                const uint4 v = *reinterpret_cast<const uint4*>(srow + i0);
+                nib = static_cast<uint32_t>(v.x >= T) | static_cast<uint32_t>(v.y >= T) << 1 |
+                      static_cast<uint32_t>(v.z >= T) << 2 | static_cast<uint32_t>(v.w >= T) << 3;
+            } else {
+                for (int j = 0; j < 4 && i0 + j < m; ++j)
+                    nib |= static_cast<uint32_t>(srow[i0 + j] >= T) << j;
+            }
+            // word w of the block holds lanes 8w .. 8w+7's nibbles
+            uint32_t word = nib << (4 * (lane & 7));
+            word |= __shfl_xor_sync(0xffffffffu, word, 1);
+            word |= __shfl_xor_sync(0xffffffffu, word, 2);
+            word |= __shfl_xor_sync(0xffffffffu, word, 4);
+            if ((lane & 7) == 0 && i0 < m) bits[(base >> 5) + (lane >> 3)] = word;
+        }
+        __syncthreads();
+        const int nw = (m + 31) >> 5;
+        const int wpt = (nw + kTopkThreads - 1) / kTopkThreads;  // words per thread
+        const int w0 = min(nw, tid * wpt), w1 = min(nw, w0 + wpt);
+        uint32_t cnt = 0;
+        for (int w = w0; w < w1; ++w) cnt += __popc(bits[w]);
+        uint32_t incl = cnt;  // inclusive scan of the counts in thread order
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const uint32_t x = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += x;
+        }
+        if (lane == 31) S.wsum[warp] = incl;
+        __syncthreads();
+        // positions in the warps before this one, and the segment's total
+        uint32_t ws = lane < kTopkWarps ? S.wsum[lane] : 0u;
+#pragma unroll
+        for (int off = 1; off < kTopkWarps; off <<= 1) {
+            const uint32_t x = __shfl_up_sync(0xffffffffu, ws, off);
+            if (lane >= off) ws += x;
+        }
+        const uint32_t before = __shfl_sync(0xffffffffu, ws, warp > 0 ? warp - 1 : 0);
+        const uint32_t total = __shfl_sync(0xffffffffu, ws, kTopkWarps - 1);
+        // thread q > rank stores this segment's total into CTA q's slot `rank`
+        if (tid < kClusterCtas && tid > static_cast<int>(rank))
+            dsmem_st_u32(dsmem_addr(&CS.cnt_g[rank], tid), total);
+        // The last cluster barrier, as on the path below.
+        cluster_sync_all();
+        uint32_t G = 0;  // selected positions in the segments before this one
+        for (uint32_t q = 0; q < rank; ++q) G += CS.cnt_g[q];
+        uint32_t at = incl - cnt + (warp > 0 ? before : 0u);
+        uint32_t* opos = S.cand;
+        for (int w = w0; w < w1; ++w)
+            for (uint32_t x = bits[w]; x; x &= x - 1u) {
+                // the segment holds at most k selected keys; the bound only
+                // guards the buffer against counts that were not the row's
+                if (at < static_cast<uint32_t>(kCandCap))
+                    opos[at] = static_cast<uint32_t>(s0 + (w << 5) + (__ffs(x) - 1));
+                ++at;
+            }
+        __syncthreads();
+        const uint32_t nout = min(total, static_cast<uint32_t>(kCandCap));
+        for (uint32_t i = tid; i < nout; i += kTopkThreads)
+            if (G + i < static_cast<uint32_t>(k)) o[G + i] = static_cast<int32_t>(opos[i]);
+        return;
+    }
 
     // ---- C: counts of this segment, offsets from the segments before it.
     // Each warp walks a contiguous part of the segment in blocks of 128 keys,
