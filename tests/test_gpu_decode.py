@@ -181,6 +181,39 @@ def test_decode_index_histogram_paths_bit_exact(ic, ctx):
     assert kinds == {"fits", "overflows"}
 
 
+def test_decode_index_few_ties_bit_exact(ic, ctx):
+    """The decode F layer (scan with first-digit histograms, cluster top-k)
+    on wide integer inputs (q in [-31, 31], keys in [-16, 16]): every score
+    is exact in fp32 (as in test_decode_scores_wide_integer_exact) and the
+    scores are spread widely, so the k-th largest is mostly unique.  Rows
+    whose keys equal to the threshold are all taken select through the
+    top-k's bitmap output; every row must equal the oracle's top-k bit for
+    bit, and most rows must be of that kind."""
+    B, S_max, k, H_I = 4, 70001, 2048, 64
+    gen = torch.Generator().manual_seed(29)
+    q = torch.randint(-31, 32, (B, H_I, 128), generator=gen).float()
+    q[:, 0, 0] = 31.0
+    table = torch.tensor([_e4m3_byte_of_int(v) for v in range(-16, 17)], dtype=torch.uint8)
+    k8 = table[torch.randint(0, 33, (B, S_max, 128), generator=gen)]
+    w = torch.tensor([-1.0, -0.5, 0.5, 1.0])[torch.randint(0, 4, (B, H_I), generator=gen)]
+    sc = torch.tensor([1.0, 0.5, 2.0, 0.25])[torch.randint(0, 4, (B, S_max), generator=gen)]
+    lens = [S_max, 65537, 40000, 2049]
+    q, w = q.bfloat16(), w.bfloat16()
+    idx = torch.full((B, k), -7, dtype=torch.int32, device="cuda")
+    ic.ic_index_fp_decode(ctx, q.cuda(), w.cuda(), k8.cuda(), sc.float().cuda(),
+                          torch.tensor(lens, dtype=torch.int32).cuda(), k, idx)
+    ctx.sync_status()
+    got = idx.cpu().numpy()
+    unique_kth = 0
+    for b in range(B):
+        n = lens[b]
+        ref = oracle.decode_scores(f32(q[b]), f32(w[b]), k8[b].numpy(), sc[b].float().numpy(), S=n)
+        assert got[b].tolist() == oracle.topk_row(ref, k).tolist(), b
+        kth = np.sort(ref)[::-1][k - 1]
+        unique_kth += int(np.sum(ref == kth) == 1)
+    assert unique_kth >= 3
+
+
 def test_decode_workload_sampled(ic, ctx):
     """Decode workload shapes (32 sequences x 65537 candidates, H_I=64,
     k=2048): one F layer, 6 sequences checked against the oracle."""
