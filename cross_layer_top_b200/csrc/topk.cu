@@ -711,10 +711,10 @@ __global__ void __launch_bounds__(kTopkThreads)
 
     // ---- C (bitmap): when every key equal to T is taken (the same answer in
     // every CTA: it follows from the merged candidates), the selection is
-    // the keys >= T.  One pass marks this segment's in a bitmap (over the
-    // merged candidates, no longer needed), a block scan of the words'
-    // popcounts gives each thread its offset, the segment's total goes to
-    // the later CTAs, and the positions are gathered in order in shared
+    // the keys >= T.  One pass marks this segment's keys >= T in a bitmap
+    // (over the merged candidates, no longer needed), a block scan of the
+    // words' popcounts gives each thread its offset, the segment's total goes
+    // to the later CTAs, and the positions are gathered in order in shared
     // memory (over this CTA's candidate list, which no CTA reads after the
     // barrier) and written with coalesced stores.
     if (use_cand && (whole || krem == S.hist[T & 0x3FFu])) {
