@@ -5,7 +5,8 @@
 // Accelerating Sparse Attention via Cross-Layer Index Reuse", Figure 2 step
 // SPARSEATTN).  One K/V head is shared by all Hq <= 16 query heads.
 //
-// Design: one CTA (4 warps, three CTAs per SM) per (query row, key split).
+// Design: one CTA per (query row, key split): 3 warps and four CTAs per SM
+// for whole rows (prefill), 4 warps and two CTAs per SM for split rows.
 // The 16 query heads form the M = 16 rows of mma.m16n8k16 tiles, so one
 // gathered K/V row serves every head.  Each warp owns chunks of 16 index
 // slots and a 2-deep ring: lane l always copies the same 16-byte piece
@@ -27,9 +28,13 @@
 #include "ic_device.cuh"
 #include "ic_internal.h"
 
-// Warps per CTA and gather-ring depth (compile-time tuning knobs).
+// Warps per CTA of the split (decode) and the row (prefill) kernel, and the
+// gather-ring depth (compile-time tuning knobs).
 #ifndef IC_ATTN_WARPS
 #define IC_ATTN_WARPS 4
+#endif
+#ifndef IC_ATTN_ROW_WARPS
+#define IC_ATTN_ROW_WARPS 3
 #endif
 #ifndef IC_ATTN_STAGES
 #define IC_ATTN_STAGES 2
@@ -41,9 +46,9 @@ namespace ic {
 // every nsplit from 2 to 8 (at most 21, for nsplit = 7)
 constexpr int kRecvRows = 24;
 
-template <int D>
+template <int D, int W>
 struct AttnShape {
-    static constexpr int WARPS = IC_ATTN_WARPS;
+    static constexpr int WARPS = W;
     static constexpr int THREADS = WARPS * 32;
     static constexpr int CH = 16;  // index slots per warp chunk
     static constexpr int STAGES = IC_ATTN_STAGES;
@@ -54,21 +59,25 @@ struct AttnShape {
     static constexpr int Q_BYTES = 16 * ROWP;
     static constexpr int MAXK = 2048;
     static constexpr int OFF_IDX = 0;
-    static constexpr int OFF_LAST = OFF_IDX + MAXK * 4;
-    static constexpr int OFF_ST = OFF_LAST + 128;
-    // Q is staged in the last warp's second ring buffer: every warp reads it
-    // into registers before any gather fills that buffer
+    static constexpr int OFF_ST = OFF_IDX + MAXK * 4;
+    // Q is staged in the last warp's second ring buffer, followed by the
+    // CTA's last-valid-slot word: every warp reads both before any gather
+    // fills that buffer
     static constexpr int OFF_Q = OFF_ST + (WARPS - 1) * WARP_BYTES + STAGE_BYTES;
+    static constexpr int OFF_LAST = OFF_Q + Q_BYTES;
     static constexpr int SMEM = OFF_ST + WARPS * WARP_BYTES;
-    // resident CTAs per SM (228 KB of shared memory, 1 KB reserved per CTA);
-    // three 4-warp CTAs keep three rows' prologues and merges in flight
-    static constexpr int CTAS_PER_SM = 3 * (SMEM + 1024) <= 233472 ? 3 : 2;
+    // resident CTAs per SM (228 KB of shared memory, 1 KB reserved per CTA):
+    // several CTAs keep several rows' prologues and merges in flight (three
+    // 4-warp CTAs, or four 3-warp CTAs for the row kernel)
+    static constexpr int CTAS_FIT = 233472 / (SMEM + 1024);
+    static constexpr int CTAS_PER_SM = CTAS_FIT < 4 ? CTAS_FIT : 4;
+    static_assert(CTAS_PER_SM >= 2, "shared memory per CTA");
     // split rows: a receive area of its own past the ring, for the cluster
     // merge ([kRecvRows][D] partial O, then [kRecvRows][2] M, L)
     static constexpr int OFF_RECV = SMEM;
     static constexpr int SMEM_SPLIT = OFF_RECV + (kRecvRows * D + kRecvRows * 2) * 4;
     static constexpr int CTAS_SPLIT = 233472 / (SMEM_SPLIT + 1024) < 3 ? 233472 / (SMEM_SPLIT + 1024) : 3;
-    static_assert(Q_BYTES <= STAGE_BYTES && STAGES >= 2, "Q lives in a second ring buffer");
+    static_assert(Q_BYTES + 4 <= STAGE_BYTES && STAGES >= 2, "Q and the last-slot word live in a second ring buffer");
     // per-warp O and (m, l), then the per-head factors, M and L
     // per-warp partial O rows are OS = D + 8 floats apart (OS = 8 mod 32 banks):
     // a warp's float2 fragment stores then take the minimal two wavefronts
@@ -198,9 +207,14 @@ __device__ __forceinline__ void attn_chunk(uint32_t kb, uint32_t vb, uint32_t cm
 
 // SPLIT: rows split across a cluster of CTAs (few rows, decode); otherwise
 // one CTA per row, and the cluster merge is not compiled in.
+// the shape of the split (decode) and of the row (prefill) kernel
 template <int D, bool SPLIT>
-__global__ void __launch_bounds__(AttnShape<D>::THREADS,
-                                  SPLIT ? AttnShape<D>::CTAS_SPLIT : AttnShape<D>::CTAS_PER_SM)
+using AttnShapeOf = AttnShape<D, SPLIT ? IC_ATTN_WARPS : IC_ATTN_ROW_WARPS>;
+
+template <int D, bool SPLIT>
+__global__ void __launch_bounds__(AttnShapeOf<D, SPLIT>::THREADS,
+                                  SPLIT ? AttnShapeOf<D, SPLIT>::CTAS_SPLIT
+                                        : AttnShapeOf<D, SPLIT>::CTAS_PER_SM)
     k_sparse_attn(const __nv_bfloat16* __restrict__ Q, const __nv_bfloat16* __restrict__ K,
                   const __nv_bfloat16* __restrict__ V, const int32_t* __restrict__ idx, int Hq,
                   int k, int rows_per_seq, long long kv_seq_stride, int kv_len, float scale_log2,
@@ -208,7 +222,7 @@ __global__ void __launch_bounds__(AttnShape<D>::THREADS,
                   const __nv_bfloat16* __restrict__ nK, const __nv_bfloat16* __restrict__ nV,
                   __nv_bfloat16* __restrict__ out,
                   int* __restrict__ err) {
-    using S = AttnShape<D>;
+    using S = AttnShapeOf<D, SPLIT>;
     extern __shared__ __align__(128) uint8_t smem[];
     const int r = blockIdx.x, split = blockIdx.y;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -545,14 +559,15 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
                          const int32_t* idx, int rows, int Hq, int k, int rows_per_seq,
                          int64_t kv_seq_stride, int kv_len, float scale, void* out,
                          cudaStream_t stream) {
-    using S = AttnShape<D>;
+    using SR = AttnShapeOf<D, false>;  // the row kernel
+    using SS = AttnShapeOf<D, true>;   // the split kernel
     static PerDeviceOnce attr_once;
     cudaError_t ea = attr_once.run(ctx->device, [] {
         cudaError_t e = cudaFuncSetAttribute(k_sparse_attn<D, false>,
-                                             cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM);
+                                             cudaFuncAttributeMaxDynamicSharedMemorySize, SR::SMEM);
         if (e == cudaSuccess)
             e = cudaFuncSetAttribute(k_sparse_attn<D, true>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, S::SMEM_SPLIT);
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, SS::SMEM_SPLIT);
         return e;
     });
     if (ea != cudaSuccess) return cuda_fail(ctx, ea, "cudaFuncSetAttribute(sparse_attn)");
@@ -570,8 +585,8 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
         if (n == 0) {
             cudaLaunchConfig_t q = {};
             q.gridDim = dim3(1, cs, 1);
-            q.blockDim = dim3(S::THREADS, 1, 1);
-            q.dynamicSmemBytes = S::SMEM_SPLIT;
+            q.blockDim = dim3(SS::THREADS, 1, 1);
+            q.dynamicSmemBytes = SS::SMEM_SPLIT;
             cudaLaunchAttribute qa[1];
             qa[0].id = cudaLaunchAttributeClusterDimension;
             qa[0].val.clusterDim.x = 1;
@@ -586,17 +601,17 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
         return n;
     };
     int nsplit = 1;
-    const int target = S::CTAS_PER_SM * ctx->num_sms;
+    const int target = SR::CTAS_PER_SM * ctx->num_sms;
     if (rows < target) {
         nsplit = target / rows;
-        const int max_split = (k + S::CH - 1) / S::CH;
+        const int max_split = (k + SS::CH - 1) / SS::CH;
         if (nsplit > max_split) nsplit = max_split;
         if (nsplit > kMaxClusterSplits) nsplit = kMaxClusterSplits;
         while (nsplit > 1 && resident_clusters(nsplit) < rows) --nsplit;
         if (nsplit < 1) nsplit = 1;
     }
     int kps = (k + nsplit - 1) / nsplit;
-    kps = (kps + S::CH - 1) / S::CH * S::CH;
+    kps = (kps + SS::CH - 1) / SS::CH * SS::CH;
     nsplit = (k + kps - 1) / kps;
     const float scale_log2 = scale * 1.4426950408889634f;
     // slot rows start 16-byte aligned when idx does and k, kps are multiples of 4
@@ -613,8 +628,8 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
     if (nsplit == 1) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(rows, 1, 1);
-        cfg.blockDim = dim3(S::THREADS, 1, 1);
-        cfg.dynamicSmemBytes = S::SMEM;
+        cfg.blockDim = dim3(SR::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = SR::SMEM;
         cfg.stream = stream;
         cudaLaunchAttribute attr[1];
         unsigned int na = 0;
@@ -622,13 +637,13 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
         cfg.attrs = attr;
         cfg.numAttrs = na;
         cudaLaunchKernelEx(&cfg, k_sparse_attn<D, false>, Qp, Kp, Vp, idx, Hq, k, rows_per_seq, kvs,
-                           kv_len, scale_log2, 1, kps, S::CTAS_PER_SM * ctx->num_sms, vec_idx,
+                           kv_len, scale_log2, 1, kps, SR::CTAS_PER_SM * ctx->num_sms, vec_idx,
                            ctx->pdl, pfK, pfV, op, ctx->dev_err);
     } else {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(rows, nsplit, 1);
-        cfg.blockDim = dim3(S::THREADS, 1, 1);
-        cfg.dynamicSmemBytes = S::SMEM_SPLIT;
+        cfg.blockDim = dim3(SS::THREADS, 1, 1);
+        cfg.dynamicSmemBytes = SS::SMEM_SPLIT;
         cfg.stream = stream;
         cudaLaunchAttribute attr[2];
         attr[0].id = cudaLaunchAttributeClusterDimension;
