@@ -412,7 +412,7 @@ def run_ours(args, rank, world, local_rank):
 # the prefill kernels, from one ncu capture of the current kernel each (the
 # summaries under profiles/ for the L=16384 prefill attention and indexer);
 # None once a kernel changes until it is captured again.
-ATTN_PREFILL_DRAM_BYTES = 210.32e6 + 50.96e6
+ATTN_PREFILL_DRAM_BYTES = 209.91e6 + 55.03e6
 INDEX_SCORE_PREFILL_DRAM_BYTES = 249.13e6 + 487.47e6
 TOPK_PREFILL_DRAM_BYTES = 530.30e6 + 107.56e6
 # warp-instructions of one prefill top-k launch over the scored rows (the
