@@ -65,6 +65,10 @@ struct AttnShape {
     // fills that buffer
     static constexpr int OFF_Q = OFF_ST + (WARPS - 1) * WARP_BYTES + STAGE_BYTES;
     static constexpr int OFF_LAST = OFF_Q + Q_BYTES;
+    // split rows (at most MAXK / 2 slots each) stage Q in the second half of
+    // the slot area instead, so their first gathers need not wait for it
+    static constexpr int OFF_Q_SPLIT = OFF_IDX + MAXK * 2;
+    static_assert(Q_BYTES <= MAXK * 2, "Q fits half the slot area");
     static constexpr int SMEM = OFF_ST + WARPS * WARP_BYTES;
     // resident CTAs per SM (228 KB of shared memory, 1 KB reserved per CTA):
     // several CTAs keep several rows' prologues and merges in flight (three
@@ -230,7 +234,7 @@ __global__ void __launch_bounds__(AttnShapeOf<D, SPLIT>::THREADS,
     const int nk = max(0, min(k, slot0 + kps) - slot0);
     int32_t* sIdx = reinterpret_cast<int32_t*>(smem + S::OFF_IDX);
     int* s_last = reinterpret_cast<int*>(smem + S::OFF_LAST);
-    const uint32_t sQ = smem_u32(smem + S::OFF_Q);
+    const uint32_t sQ = smem_u32(smem + (SPLIT ? S::OFF_Q_SPLIT : S::OFF_Q));
     const long long seq = rows_per_seq > 0 ? r / rows_per_seq : 0;
     const __nv_bfloat16* Kb = K + seq * kv_seq_stride;
     const __nv_bfloat16* Vb = V + seq * kv_seq_stride;
@@ -325,19 +329,24 @@ __global__ void __launch_bounds__(AttnShapeOf<D, SPLIT>::THREADS,
         stage_q();
     }
     griddep_launch_dependents();
-    cp_async_wait<0>();
+    if constexpr (!SPLIT) cp_async_wait<0>();  // Q, in a ring buffer, is read before any gather
     __syncthreads();
     const int nk_eff = *s_last + 1;  // slots after the last valid one hold nothing
 
     uint32_t qa[D / 16][4];
+    auto load_q = [&]() {
 #pragma unroll
-    for (int kk = 0; kk < D / 16; ++kk) {
-        const int m = lane >> 3;
-        const int row = (m & 1) * 8 + (lane & 7);
-        const int c = 2 * kk + (m >> 1);
-        ldsm_x4(sQ + swz<D>(row, c), qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
-    }
-    __syncthreads();  // every warp holds Q: its staging buffer may now be filled
+        for (int kk = 0; kk < D / 16; ++kk) {
+            const int m = lane >> 3;
+            const int row = (m & 1) * 8 + (lane & 7);
+            const int c = 2 * kk + (m >> 1);
+            ldsm_x4(sQ + swz<D>(row, c), qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3]);
+        }
+    };
+    if constexpr (!SPLIT) load_q();
+    // every warp holds Q (row kernel) and has read the last-slot word, which
+    // lies in a ring buffer: the gathers may now fill the ring
+    __syncthreads();
 
     const uint32_t wst = smem_u32(smem + S::OFF_ST + warp * S::WARP_BYTES);
     const int nch = (nk_eff + S::CH - 1) / S::CH;
@@ -411,6 +420,13 @@ __global__ void __launch_bounds__(AttnShapeOf<D, SPLIT>::THREADS,
     // j + STAGES) as soon as chunk j has been consumed
 #pragma unroll
     for (int j = 0; j < S::STAGES; ++j) issue(j);
+    if constexpr (SPLIT) {
+        // split rows stage Q outside the ring, so the first gathers went out
+        // before it landed; its cp.async group is older than theirs
+        cp_async_wait<S::STAGES>();
+        __syncthreads();
+        load_q();
+    }
     for (int j = 0; j < my_n; ++j) {
         const int st = j % S::STAGES;
         cp_async_wait<S::STAGES - 1>();  // chunk j has landed
@@ -625,6 +641,9 @@ static int launch_attn_t(ic_ctx* ctx, const void* Q, const void* K, const void* 
     const auto* pfK = ctx->pf_V ? static_cast<const __nv_bfloat16*>(ctx->pf_K) : nullptr;
     const auto* pfV = pfK ? static_cast<const __nv_bfloat16*>(ctx->pf_V) : nullptr;
     const long long kvs = static_cast<long long>(kv_seq_stride);
+    // a split row's slots share the slot area with Q (k <= 2048 over >= 2 splits)
+    if (nsplit > 1 && kps > SS::MAXK / 2)
+        return fail(ctx, IC_ERR_UNSUPPORTED, "sparse_attn: %d slots per split", kps);
     if (nsplit == 1) {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(rows, 1, 1);
