@@ -409,6 +409,7 @@ struct alignas(16) TopkClusterShared {
     // key range, and (for the later segments) its counts of keys > T and == T
     uint32_t rng_min[kClusterCtas], rng_max[kClusterCtas];
     uint32_t cnt_g[kClusterCtas], cnt_e[kClusterCtas];
+    alignas(8) uint64_t stage_bar;  // completion of the segment's bulk copy
 };
 static_assert(offsetof(TopkShared, hist) % 16 == 0 && offsetof(TopkShared, cand) % 16 == 0,
               "16-byte loads of the histogram and candidates");
@@ -418,7 +419,7 @@ __global__ void __launch_bounds__(kTopkThreads)
     k_topk_cluster(const float* __restrict__ scores, long long ld, int k,
                    const int32_t* __restrict__ row_len, int max_len, int causal_base,
                    int32_t* __restrict__ out, long long ld_out, int seg_cap,
-                   uint32_t* __restrict__ ghist) {
+                   uint32_t* __restrict__ ghist, int* __restrict__ err) {
     // dynamic shared memory: the staged segment, then the merged candidates
     extern __shared__ uint32_t srow[];
     uint32_t* cand_all = srow + seg_cap;
@@ -459,30 +460,43 @@ __global__ void __launch_bounds__(kTopkThreads)
     auto stage = [&](uint32_t& kmin, uint32_t& kmax) {
         kmin = 0xFFFFFFFFu;
         kmax = 0u;
+        // The segment's whole float4s arrive by one bulk copy that completes
+        // on an mbarrier (the row start and the segment start are 16-byte
+        // aligned; at most 45000 keys, within the transaction count), the
+        // last m mod 4 scores by plain loads; then every float becomes its
+        // order key in place.
         const int m4 = m >> 2;
-        const float4* row4 = reinterpret_cast<const float4*>(row);
-        auto put = [&](int i, const float4& v) {
-            const uint32_t u0 = order_key(v.x), u1 = order_key(v.y);
-            const uint32_t u2 = order_key(v.z), u3 = order_key(v.w);
-            *reinterpret_cast<uint4*>(srow + 4 * i) = make_uint4(u0, u1, u2, u3);
-            kmin = min(kmin, min(min(u0, u1), min(u2, u3)));
-            kmax = max(kmax, max(max(u0, u1), max(u2, u3)));
-        };
-        // four 16-byte loads in flight per thread before any is used
-        int i = tid;
-        for (; i + 3 * kTopkThreads < m4; i += 4 * kTopkThreads) {
-            float4 v[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) v[q] = __ldg(row4 + i + q * kTopkThreads);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) put(i + q * kTopkThreads, v[q]);
+        const uint32_t bytes = static_cast<uint32_t>(m4) * 16u;
+        if (tid == 0) {
+            mbar_init(&CS.stage_bar, 1);
+            fence_mbar_init();
         }
-        for (; i < m4; i += kTopkThreads) put(i, __ldg(row4 + i));
+        __syncthreads();
+        if (tid == 0 && bytes > 0) {
+            mbar_arrive_expect_tx(&CS.stage_bar, bytes);
+            asm volatile(
+                "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                ::"r"(smem_u32(srow)), "l"(row), "r"(bytes), "r"(smem_u32(&CS.stage_bar))
+                : "memory");
+        }
         for (int i = 4 * m4 + tid; i < m; i += kTopkThreads) {
             const uint32_t u = order_key(__ldg(row + i));
             srow[i] = u;
             kmin = min(kmin, u);
             kmax = max(kmax, u);
+        }
+        if (bytes > 0 && !mbar_wait_drain(&CS.stage_bar, 0)) {
+            // bounded: the keys are then not the row's; the error is latched
+            if (tid == 0 && err != nullptr) atomicCAS(err, 0, kDevTimeoutProducer);
+        }
+        uint4* srow4 = reinterpret_cast<uint4*>(srow);
+        for (int i = tid; i < m4; i += kTopkThreads) {
+            const uint4 v = srow4[i];
+            const uint32_t u0 = order_key(__uint_as_float(v.x)), u1 = order_key(__uint_as_float(v.y));
+            const uint32_t u2 = order_key(__uint_as_float(v.z)), u3 = order_key(__uint_as_float(v.w));
+            srow4[i] = make_uint4(u0, u1, u2, u3);
+            kmin = min(kmin, min(min(u0, u1), min(u2, u3)));
+            kmax = max(kmax, max(max(u0, u1), max(u2, u3)));
         }
     };
     // The histogram's counts are loaded before the segment, so that their
@@ -904,7 +918,7 @@ static int launch_topk_cluster(ic_ctx* ctx, const float* scores, int64_t ld, int
     LaunchScope ls(ctx, IC_K_TOPK, stream);
     cudaLaunchKernelEx(&cfg, k_topk_cluster, scores, static_cast<long long>(ld), k, row_len,
                        max_len, causal_base, idx_out, static_cast<long long>(ld_out), seg_cap,
-                       hist);
+                       hist, ctx->dev_err);
     e = ls.done();
     if (e != cudaSuccess) return cuda_fail(ctx, e, "topk_cluster launch");
     return IC_OK;
