@@ -17,11 +17,13 @@
 //     b1 go with their positions to the warp's own slice of a candidate
 //     list.  Two more radix digits (11 + 10 bits) are resolved on the
 //     candidates: the threshold key T and krem, the number of keys equal to
-//     T still to take;
+//     T still to take (the third digit is skipped when the second digit's
+//     bin is taken whole: T is then that bin's smallest key);
 //  C. when every key equal to T is taken (no tie split), the candidates
-//     >= T are OR-ed into the bitmap and its set positions are written in
-//     ascending order (a block scan of the words' popcounts gives each
-//     warp's offset).  Otherwise (a tie split, a candidate bin too large
+//     >= T are OR-ed into the bitmap and its set positions are gathered in
+//     ascending order in shared memory (a block scan of the words'
+//     popcounts gives each thread its offset), then written with coalesced
+//     stores.  Otherwise (a tie split, a candidate bin too large
 //     for the list, or a row longer than the bitmap) the general path:
 //     digits resolved on the full row, then per-warp counts of keys > T and
 //     == T, a block scan, and an ordered walk that takes a key == T while
@@ -390,16 +392,19 @@ __global__ void __launch_bounds__(kRowThreads, kRowMinCtas)
 // ------------------------------------------------------------------------
 // Cluster variant for few long rows (the decode step: B rows of up to
 // ~200K candidates).  One thread-block cluster of kClusterCtas CTAs per row;
-// its first-level histogram has 2048 bins uniform in VALUE between the
-// row's min and max (a monotone function of the score, so every key in a
-// higher bin is larger), which narrows bin b1 to a short candidate list;
 // CTA `rank` stages the row segment [rank*seg, (rank+1)*seg) in its shared
-// memory.  The row-wide quantities (min/max, histograms, candidate lists,
-// per-segment counts) are exchanged through distributed shared memory
-// (mapa + ld.shared::cluster) between cluster barriers; every CTA then takes
-// the same decisions, and each writes the selected positions of its own
-// segment at the offsets of the segments before it.  Same output contract
-// as k_topk.
+// memory (one bulk copy).  With the scan's first-digit histogram of the row
+// the bin b1 of the k-th largest key is known before the row is read, and
+// its keys form a short candidate list; without it, a first-level
+// histogram of 2048 bins uniform in VALUE between the row's min and max (a
+// monotone function of the score, so every key in a higher bin is larger)
+// narrows bin b1.  The row-wide quantities (min/max, histograms, candidate
+// lists, per-segment counts) are exchanged through distributed shared
+// memory (mapa + ld.shared::cluster) between cluster barriers; every CTA
+// then takes the same decisions, and each writes the selected positions of
+// its own segment (through a selection bitmap when every key equal to the
+// threshold is taken) at the offsets of the segments before it.  Same
+// output contract as k_topk.
 constexpr int kClusterCtas = 8;
 
 struct alignas(16) TopkClusterShared {
