@@ -64,6 +64,18 @@ extern "C" int ic_run_stack_ahead(ic_ctx* ctx, const ic_pattern* pattern, const 
     cudaError_t e = cudaEventRecord(a.start, main);
     if (e == cudaSuccess) e = cudaStreamWaitEvent(a.side, a.start, 0);
     if (e != cudaSuccess) return cuda_fail(ctx, e, "run_stack_ahead: fork");
+    // On an error below, the caller's stream still waits for what the side
+    // stream holds, so that nothing writes the caller's buffers after the
+    // caller's stream has passed this call.
+    struct Join {
+        ic_ctx::Ahead& a;
+        cudaStream_t main;
+        bool armed = true;
+        ~Join() {
+            if (armed && cudaEventRecord(a.start, a.side) == cudaSuccess)
+                cudaStreamWaitEvent(main, a.start, 0);
+        }
+    } join{a, main};
     const int N = static_cast<int>(pattern->c.size());
     int j = -1;  // F layers seen
     for (int l = 0; l < N; ++l) {
@@ -109,5 +121,6 @@ extern "C" int ic_run_stack_ahead(ic_ctx* ctx, const ic_pattern* pattern, const 
                                 dims->scale, io.out, main);
         if (rc) return rc;
     }
+    join.armed = false;  // the last layer waited for the last indexer
     return IC_OK;
 }

@@ -347,7 +347,9 @@ int ic_run_stack(ic_ctx *ctx, const ic_pattern *pattern, const ic_layer_io *laye
  * The side stream first waits for the work `stream` held at the call, and
  * `stream` ends after the last layer, so its completion covers all work.
  * No programmatic launches or cross-layer prefetch.  Errors as ic_run_stack,
- * plus IC_ERR_INVALID_ARG when idx_cache2 is NULL or equals idx_cache. */
+ * plus IC_ERR_INVALID_ARG when idx_cache2 is NULL or equals idx_cache; on an
+ * error after work was issued, `stream` still waits for the side stream's
+ * work, so completion of `stream` covers it. */
 int ic_run_stack_ahead(ic_ctx *ctx, const ic_pattern *pattern, const ic_layer_io *layers,
                        const ic_stack_dims *dims, int32_t *idx_cache, int32_t *idx_cache2,
                        void *stream);

@@ -162,3 +162,28 @@ def test_stack_ahead_needs_two_buffers(ic):
                                        cache, cache)
     assert e.value.code == ic.IC_ERR_INVALID_ARG
     ctx.close()
+
+
+def test_stack_ahead_error_leaves_context_usable(ic):
+    """A layer that fails its argument checks (no Q) after F layers' indexers
+    were issued on the side stream: the call returns IC_ERR_INVALID_ARG, the
+    caller's stream covers the side stream's work, and the next call on the
+    same context is bit-identical to ic_run_stack."""
+    cfg = synth.CONFIGS["tiny"]
+    pattern = "FSFS"
+    L, k = cfg.L, cfg.k
+    layers = _prefill_layers(cfg, pattern, "cpu")
+    ctx = ic.Context(0)
+    dims = ic.stack_dims(ic.IC_PREFILL, cfg.H_I, cfg.d_I, k, cfg.Hq, cfg.d, L=L)
+    bad = _with_outputs(layers, L, cfg)
+    bad[3]["Q"] = None
+    c0 = torch.empty((L, k), dtype=torch.int32, device="cuda")
+    c1 = torch.empty((L, k), dtype=torch.int32, device="cuda")
+    with pytest.raises(ic.ICError) as e:
+        ic.ic_run_stack_ahead(ctx, ic.ic_create_pattern(pattern), bad, dims, c0, c1)
+    assert e.value.code == ic.IC_ERR_INVALID_ARG
+    torch.cuda.current_stream().synchronize()
+    ctx.sync_status()
+    _run_both(ic, ctx, pattern, _with_outputs(layers, L, cfg), _with_outputs(layers, L, cfg), dims,
+              L, k)
+    ctx.close()
