@@ -111,6 +111,21 @@ extern "C" int ic_run_stack_host(ic_ctx* ctx, const ic_pattern* pattern,
         hs.slot_cap = need;
     }
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    // On an error below, `stream` still waits for every copy already issued
+    // on the context's streams, so that none reads or writes the caller's
+    // host buffers after the caller's stream has passed this call.
+    struct Join {
+        ic_ctx::HostStack& hs;
+        cudaStream_t s;
+        bool armed = true;
+        ~Join() {
+            if (!armed) return;
+            if (cudaEventRecord(hs.in_ready[0], hs.in) == cudaSuccess)
+                cudaStreamWaitEvent(s, hs.in_ready[0], 0);
+            if (cudaEventRecord(hs.out_done[0], hs.out) == cudaSuccess)
+                cudaStreamWaitEvent(s, hs.out_done[0], 0);
+        }
+    } join{hs, s};
     const int N = static_cast<int>(pattern->c.size());
     for (int l = 0; l < N; ++l) {
         const int sl = l % ic_ctx::kHostSlots;
@@ -174,5 +189,6 @@ extern "C" int ic_run_stack_host(ic_ctx* ctx, const ic_pattern* pattern,
     for (int i = 0; i < ic_ctx::kHostSlots && e == cudaSuccess; ++i)
         e = cudaStreamWaitEvent(s, hs.out_done[i], 0);
     if (e != cudaSuccess) return cuda_fail(ctx, e, "run_stack_host: final wait");
+    join.armed = false;  // the caller's stream has waited for every copy already
     return IC_OK;
 }

@@ -407,7 +407,8 @@ int ic_stack_graph_destroy(ic_graph *graph);
  * layers compute.  Asynchronous: when `stream` reaches the point after this
  * call, every output is in host memory; the host inputs must not change
  * before then.  Errors as ic_run_stack, plus IC_ERR_NOMEM when the four
- * slots cannot be allocated. */
+ * slots cannot be allocated; on an error after copies were issued, `stream`
+ * still waits for them, so its completion means no copy is left. */
 int ic_run_stack_host(ic_ctx *ctx, const ic_pattern *pattern, const ic_layer_io *layers_host,
                       const ic_stack_dims *dims, int32_t *idx_cache, void *stream);
 

@@ -106,3 +106,31 @@ def test_host_stack_prefill_workload(ic):
     host = _run_both(ic, ctx, cfg.pattern, layers, dims, L, k)
     _check_equal(layers, host)
     ctx.close()
+
+
+def test_host_stack_error_leaves_context_usable(ic):
+    """A layer without an output buffer fails its checks after earlier layers'
+    copies were issued: the call returns IC_ERR_INVALID_ARG, the caller's
+    stream covers the copies already issued, and the next call on the same
+    context matches ic_run_stack bit for bit."""
+    ctx = ic.Context(0)
+    cfg = synth.PrefillConfig("host_prefill_err", 1500, "FSSF", 64, 128, 256, 16, 128, 14)
+    L, k = cfg.L, cfg.k
+    layers = []
+    for l in range(cfg.n_layers):
+        lay = synth.prefill_layer(cfg, l, "cuda")
+        lay["out"] = torch.empty((L, cfg.Hq, cfg.d), dtype=torch.bfloat16, device="cuda")
+        lay["idx_snapshot"] = torch.empty((L, k), dtype=torch.int32, device="cuda")
+        layers.append(lay)
+    dims = ic.stack_dims(ic.IC_PREFILL, cfg.H_I, cfg.d_I, k, cfg.Hq, cfg.d, L=L)
+    bad = _host_layers(layers)
+    bad[2]["out"] = None
+    cache = torch.empty((L, k), dtype=torch.int32, device="cuda")
+    with pytest.raises(ic.ICError) as e:
+        ic.ic_run_stack_host(ctx, ic.ic_create_pattern(cfg.pattern), bad, dims, cache)
+    assert e.value.code == ic.IC_ERR_INVALID_ARG
+    torch.cuda.current_stream().synchronize()
+    ctx.sync_status()
+    host = _run_both(ic, ctx, cfg.pattern, layers, dims, L, k)
+    _check_equal(layers, host)
+    ctx.close()
