@@ -161,33 +161,45 @@ __global__ void __launch_bounds__(kRowThreads, kRowMinCtas)
     }
     const float* row = scores + static_cast<long long>(r) * ld;
     auto key_at = [&](int i) -> uint32_t { return order_key(__ldg(row + i)); };
-    // ---- A: keys + histogram of the top 11 bits
-    for (int i = tid; i < 2048; i += kRowThreads) S.hist[i] = 0;
-    if (tid == 0) S.ncand = 0;
-    __syncthreads();
-    {
+    // ---- A: histogram of the keys' top 11 bits.  It is counted on the raw
+    // float bits: raw top bits r lie in key bin r + 1024 (r < 1024) or
+    // 2047 - r, for every score but -0.0, whose raw bits fall in bin 1023
+    // while its key (that of +0.0) is in bin 1024.  Only a threshold in bin
+    // 1023 or 1024 depends on that: such a row is counted again on keys.
+    auto count_keys = [&](bool raw) {
+        for (int i = tid; i < 2048; i += kRowThreads) S.hist[i] = 0;
+        __syncthreads();
         const int n4 = n >> 2;
         const float4* row4 = reinterpret_cast<const float4*>(row);
+        auto bin = [&](float x) { return (raw ? __float_as_uint(x) : order_key(x)) >> 21; };
         for (int i = tid; i < n4; i += kRowThreads) {
             const float4 v = __ldg(row4 + i);
-            const uint32_t u0 = order_key(v.x), u1 = order_key(v.y);
-            const uint32_t u2 = order_key(v.z), u3 = order_key(v.w);
-            atomicAdd(&S.hist[u0 >> 21], 1u);
-            atomicAdd(&S.hist[u1 >> 21], 1u);
-            atomicAdd(&S.hist[u2 >> 21], 1u);
-            atomicAdd(&S.hist[u3 >> 21], 1u);
+            atomicAdd(&S.hist[bin(v.x)], 1u);
+            atomicAdd(&S.hist[bin(v.y)], 1u);
+            atomicAdd(&S.hist[bin(v.z)], 1u);
+            atomicAdd(&S.hist[bin(v.w)], 1u);
         }
-        for (int i = 4 * n4 + tid; i < n; i += kRowThreads) {
-            const uint32_t u = order_key(__ldg(row + i));
-            atomicAdd(&S.hist[u >> 21], 1u);
+        for (int i = 4 * n4 + tid; i < n; i += kRowThreads) atomicAdd(&S.hist[bin(__ldg(row + i))], 1u);
+        __syncthreads();
+        constexpr int PER = 2048 / kRowThreads;
+        uint32_t c[PER];
+#pragma unroll
+        for (int b = 0; b < PER; ++b) {
+            const int key_bin = tid * PER + b;
+            c[b] = S.hist[!raw ? key_bin : (key_bin >= 1024 ? key_bin - 1024 : 2047 - key_bin)];
         }
+        find_bin_counts<2048>(S, static_cast<uint32_t>(k), c);
+    };
+    if (tid == 0) S.ncand = 0;
+    count_keys(true);
+    if (S.bin == 1023u || S.bin == 1024u) {  // the same in every thread
+        __syncthreads();  // everyone has read S.bin
+        count_keys(false);
     }
-    __syncthreads();
-    find_bin<2048>(S, static_cast<uint32_t>(k));
     const uint32_t b1 = S.bin;
     uint32_t krem = static_cast<uint32_t>(k) - S.above;
-    const uint32_t in_bin = S.hist[b1];
-    __syncthreads();  // everyone has read S.bin / S.above / S.hist[b1]
+    const uint32_t in_bin = S.bin_count;
+    __syncthreads();  // everyone has read S.bin / S.above / S.bin_count
 
     // ---- B: resolve bits 20..10 and 9..0 within bin b1
     uint32_t prefix = b1 << 21, mask = 0xFFE00000u;

@@ -14,7 +14,9 @@ row kernel needs more rows than the cluster form takes (every row checked):
   - the general path: a row longer than the bitmap holds, a candidate bin
     larger than the candidate list, a warp slice that overflows, and a tie
     at T that is split by position;
-  - rows of at most k keys (all taken, -1 padding)."""
+  - rows of at most k keys (all taken, -1 padding);
+  - rows whose threshold lies among signed zeros and denormals (the first
+    digit's bins 1023 and 1024)."""
 import numpy as np
 import pytest
 import torch
@@ -38,6 +40,7 @@ def _long_rows():
     rng = np.random.default_rng(2024)
     rows = {}
     rows["gauss_20000"] = rng.standard_normal(20000)
+    rows.update(_zero_threshold_rows(rng, 40000))
     rows["gauss_at_bitmap_cap"] = rng.standard_normal(131072)
     rows["longer_than_bitmap"] = rng.standard_normal(140000)
     # 1000 keys far above, then 5000 keys in [1.0, 1.25) (one 11-bit bin), the rest below:
@@ -67,12 +70,36 @@ def _long_rows():
     return {n: v.astype(np.float32) for n, v in rows.items()}
 
 
+def _zero_threshold_rows(rng, n):
+    """Rows whose k-th largest score lies in the bins around zero (key bins
+    1023 and 1024): signed zeros and denormals, where the first digit counted
+    on raw float bits differs from the order keys (-0.0) and the kernel
+    counts again."""
+    tiny = np.float32(1e-42)  # a denormal
+    # the k-th largest is 0: 1000 positives, 3000 zeros of both signs, negatives
+    r = np.concatenate([rng.random(1000) + 1.0, np.zeros(3000), -(rng.random(n - 4000) + 1.0)])
+    r = rng.permutation(r).astype(np.float32)
+    r[rng.permutation(np.flatnonzero(r == 0))[:1500]] = np.float32(-0.0)
+    rows = {"threshold_at_zero": r}
+    # the k-th largest is a negative denormal: 1000 positives, 500 zeros, 2000
+    # negative denormals, negatives
+    r = np.concatenate([rng.random(1000) + 1.0, np.zeros(500),
+                        -tiny * (1 + rng.integers(0, 50, 2000)), -(rng.random(n - 3500) + 1.0)])
+    rows["threshold_negative_denormal"] = rng.permutation(r).astype(np.float32)
+    # the k-th largest is a positive denormal, next to -0.0 keys
+    r = np.concatenate([rng.random(1000) + 1.0, tiny * (1 + rng.integers(0, 50, 2000)),
+                        np.full(1000, -0.0), -(rng.random(n - 4000) + 1.0)])
+    rows["threshold_positive_denormal"] = rng.permutation(r).astype(np.float32)
+    return rows
+
+
 def _short_rows():
     """Rows for the short-row shape: 2048 slots, and a warp's slice of 256
     slots over segments of n / 8 keys (2560 keys at n = 20000)."""
     rng = np.random.default_rng(2025)
     rows = {}
     rows["gauss_16384"] = rng.standard_normal(16384)
+    rows.update(_zero_threshold_rows(rng, 9000))
     rows["gauss_at_short_limit"] = rng.standard_normal(32768)
     rows["gauss_2049"] = rng.standard_normal(2049)
     rows["few_keys"] = rng.standard_normal(700)
