@@ -414,10 +414,10 @@ def run_ours(args, rank, world, local_rank):
 # None once a kernel changes until it is captured again.
 ATTN_PREFILL_DRAM_BYTES = 209.91e6 + 55.03e6
 INDEX_SCORE_PREFILL_DRAM_BYTES = 249.13e6 + 487.47e6
-TOPK_PREFILL_DRAM_BYTES = None
+TOPK_PREFILL_DRAM_BYTES = 532.31e6 + 107.21e6
 # warp-instructions of one prefill top-k launch over the scored rows (the
 # same capture: smsp__inst_executed.sum)
-TOPK_PREFILL_WARP_INSTR = None
+TOPK_PREFILL_WARP_INSTR = 291.70e6
 
 
 def measure_gather_ceiling(cache, lay, L, k, stream):
