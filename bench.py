@@ -666,13 +666,14 @@ def run_e2e(args, ctx, pat, dims, cfg, layers, cache, world, pairs_step, stream)
 
 def run_decode(args, ctx, peaks, peak_src, local_rank):
     """One decode step of the batched-decode workload (32 sequences x 65537
-    candidates, 16 layers FSSS x4): step ms, FP8 indexer-key scan GB/s and
-    the attention gather GB/s against the HBM peak.  --decode-layers N keeps
-    the first N layers (for profiling captures that must stay small)."""
+    candidates, 16 layers FSSS x4; --decode-config picks a 200K-context
+    workload of the retention sweep instead): step ms, FP8 indexer-key scan
+    GB/s and the attention gather GB/s against the HBM peak.  --decode-layers
+    N keeps the first N layers (for profiling captures that must stay small)."""
     import dataclasses
     from cross_layer_top_b200 import indexcache as ic
     from cross_layer_top_b200 import synth
-    cfg = synth.CONFIGS["decode"]
+    cfg = synth.CONFIGS[getattr(args, "decode_config", "decode")]
     if args.decode_layers:
         cfg = dataclasses.replace(cfg, pattern=cfg.pattern[:args.decode_layers])
     dev = torch.device("cuda", local_rank)
@@ -701,8 +702,9 @@ def run_decode(args, ctx, peaks, peak_src, local_rank):
     scan_ms, scan_n = kt["index_score_decode"]
     att_ms, att_n = kt["sparse_attn"]
     gather_bytes = B * k * 2 * cfg.d * 2
-    res = {"workload": "decode: 32 sequences x (65536 cached + 1 new) tokens, 16 layers FSSS x4, "
-                       "FP8 e4m3 indexer keys + fp32 per-token scale, k=2048",
+    res = {"workload": "decode: %d sequences x (%d cached + 1 new) tokens, %d layers %s, "
+                       "FP8 e4m3 indexer keys + fp32 per-token scale, k=%d"
+                       % (B, S - 1, cfg.n_layers, cfg.pattern, k),
            **t,
            "kernels_ms_per_step": {n: round(v[0] / steps, 4) for n, v in kt.items()}}
     if scan_n:
@@ -1150,6 +1152,10 @@ def main():
     ap.add_argument("--decode-only", action="store_true",
                     help="time only the decode workload (not the contract line)")
     ap.add_argument("--decode-layers", type=int, default=0)
+    ap.add_argument("--decode-config", default="decode",
+                    choices=["decode", "decode_sweep_r1", "decode_sweep_r2", "decode_sweep_r4",
+                             "decode_sweep_r8"],
+                    help="the decode workload of --decode-only")
     ap.add_argument("--profile-kernel", default=None, choices=PROFILE_KERNELS,
                     help="harness for ncu captures: only this kernel's inputs, then exit")
     ap.add_argument("--prefill-split", action="store_true",
